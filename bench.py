@@ -1,0 +1,476 @@
+"""Benchmark: one decode step (append + paged attention over every layer) on one or more B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+
+A step is the whole hot path over one batch: for each layer, scatter the new
+token's K/V into its slot, then decode attention over every sequence's paged
+cache (with the split-K merge). Inputs are synthetic and seeded, shaped like
+the pages' models (see paged_kv_cache_470_b200/workloads.py); the default is
+the 0.5B GQA model's decode step (24 layers, Hq=20, Hkv=4, D=64, batch 64,
+context U[128,2048]).
+
+Reported (one JSON line on rank 0):
+  value      achieved HBM GB/s = algorithmic bytes of the step / step time,
+             summed over GPUs (inputs resident in HBM, CUDA-graph replay)
+  e2e        the same metric through the C ABI with host buffers: pinned-host
+             -> device copies of the step's inputs and a device -> host copy of
+             its outputs inside the timed region
+  roofline   the decode kernel alone: its algorithmic bytes per launch over its
+             CUDA-event duration, against the measured HBM copy bandwidth
+  cpu_baseline  the float64 oracle on this host's cores, on a bounded sample
+
+With --gpus N > 1 (under torchrun) each rank runs an independent replica of
+the workload on its own GPU (the path needs no exchange between GPUs); the
+step time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_470_b200 import workloads  # noqa: E402  (no CUDA library needed)
+
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_0p5b_gqa.txt")
+DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_470_b200", "csrc", "decode.cu")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what one decode step must move at least once)
+# ---------------------------------------------------------------------------
+def layer_bytes(cfg, lens, shares_prefix=None, unique_prefix=False):
+    """Bytes one layer's append + attention must move, from the drawn lengths.
+
+    KV read: 2 (K and V) x c x Hkv x D x 2 per sequence; q read and out write:
+    2 x Hq x D x 2 per sequence; table entries 4 x ceil(c/16) and the length
+    (4); append: the new K/V rows read and written (4 x Hkv x D x 2) and the
+    slot (8). With unique_prefix, a shared prefix's blocks count once.
+    """
+    B = len(lens)
+    kv = 0
+    for b, c in enumerate(lens):
+        own = c
+        if unique_prefix and shares_prefix is not None and shares_prefix[b]:
+            own = c - cfg.shared_prefix_tokens
+        kv += 2 * own * cfg.Hkv * cfg.D * 2
+    if unique_prefix and shares_prefix is not None and any(shares_prefix):
+        kv += 2 * cfg.shared_prefix_tokens * cfg.Hkv * cfg.D * 2
+    qo = 2 * B * cfg.Hq * cfg.D * 2
+    tables = sum(4 * -(-c // 16) + 4 for c in lens)
+    append = B * (4 * cfg.Hkv * cfg.D * 2 + 8)
+    return {"kv": kv, "q_out": qo, "tables": tables, "append": append,
+            "decode_kernel": kv + qo + tables, "total": kv + qo + tables + append}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it matches the current kernel source."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+        src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
+        m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        h = re.search(r"decode\.cu sha256\[:16\]:\s*([0-9a-f]+)", text)
+        if m and h and h.group(1) == src_hash:
+            return float(m.group(1))
+    except OSError:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle"}
+
+    def __init__(self, device_index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            bus = getattr(props, "pci_bus_id", None)
+            if bus is not None:
+                dom = getattr(props, "pci_domain_id", 0)
+                dev = getattr(props, "pci_device_id", 0)
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(f"{dom:08x}:{bus:02x}:{dev:02x}.0".encode())
+            else:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report what is missing
+            self.error = str(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nvml.nvmlDeviceGetClockInfo(self._h, self._nvml.NVML_CLOCK_SM))
+                mask = self._nvml.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t.is_alive():
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0, "note": getattr(self, "error", "no samples")}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# ---------------------------------------------------------------------------
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if (torch.cuda.is_available() and args.impl == "ours") else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def dist_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_done(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+class Workload:
+    def __init__(self, cfg, device, rank=0):
+        import paged_kv_cache_470_b200 as pkv
+        self.pkv = pkv
+        self.cfg = cfg
+        self.layout = workloads.draw_layout(cfg)
+        gen = workloads.device_generator(cfg.seed + 1000 * rank, device)
+        self.k, self.v = [], []
+        for _ in range(cfg.n_layers):
+            k, v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device)
+            self.k.append(k)
+            self.v.append(v)
+        self.q, self.k_new, self.v_new = workloads.make_step_inputs(cfg, gen, device)
+        self.tables = self.layout.block_tables.to(device)
+        self.lens = self.layout.context_lens.to(device)
+        self.slots = self.layout.slot_mapping().to(device)
+        self.out = torch.empty_like(self.q)
+        self.ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D, device)
+
+    def step(self, stream=None):
+        pkv, cfg = self.pkv, self.cfg
+        for layer in range(cfg.n_layers):
+            pkv.kv_cache_append(self.k_new[layer], self.v_new[layer], self.k[layer], self.v[layer], self.slots,
+                                stream=stream)
+            pkv.paged_attention_decode(self.out[layer], self.q[layer], self.k[layer], self.v[layer], self.tables,
+                                       self.lens, cfg.scale, self.ws, stream=stream)
+
+
+def capture(fn):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # warm up outside the graph once (library set-up)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_replays(graph, steps, world):
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        graph.replay()
+    end.record()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    return start.elapsed_time(end) / steps
+
+
+def decode_kernel_duration_ms(wl, reps=5):
+    """Average duration of one paged_attention_decode launch, by CUDA events on its stream, cycling layers."""
+    pkv, cfg = wl.pkv, wl.cfg
+    stream = torch.cuda.current_stream()
+    evs = []
+    for _ in range(reps):
+        for layer in range(cfg.n_layers):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            pkv.paged_attention_decode(wl.out[layer], wl.q[layer], wl.k[layer], wl.v[layer], wl.tables, wl.lens,
+                                       cfg.scale, wl.ws, stream=stream)
+            b.record(stream)
+            evs.append((a, b))
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in evs]
+    return sum(times) / len(times), len(times)
+
+
+def e2e_measure(wl, steps, warmup, world):
+    """The same step through the C ABI with host buffers: H2D of the step's inputs, D2H of its outputs."""
+    cfg = wl.cfg
+    host_in = {name: t.cpu().pin_memory() for name, t in
+               (("q", wl.q), ("k_new", wl.k_new), ("v_new", wl.v_new), ("tables", wl.tables),
+                ("lens", wl.lens), ("slots", wl.slots))}
+    dev_in = {"q": wl.q, "k_new": wl.k_new, "v_new": wl.v_new, "tables": wl.tables, "lens": wl.lens,
+              "slots": wl.slots}
+    host_out = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out.numel() * host_out.element_size()
+
+    def one():
+        for name, t in host_in.items():
+            dev_in[name].copy_(t, non_blocking=True)
+        wl.step()
+        host_out.copy_(wl.out, non_blocking=True)
+
+    g = capture(one)
+    for _ in range(warmup):
+        g.replay()
+    ms = time_replays(g, steps, world)
+    return ms, h2d, d2h
+
+
+class OracleSampler:
+    """The float64 oracle on whole layers of the workload (append + attention), on this host's cores."""
+
+    def __init__(self, cfg, layout):
+        import oracle
+        self.oracle, self.cfg, self.layout = oracle, cfg, layout
+        gen = workloads.device_generator(cfg.seed, "cpu")
+        self.k, self.v = workloads.make_layer_cache(layout.num_blocks, cfg.Hkv, cfg.D, gen, "cpu")
+        q, kn, vn = workloads.make_step_inputs(cfg, gen, "cpu", n_layers=1)
+        self.q, self.kn, self.vn = q[0], kn[0], vn[0]
+        self.slots = layout.slot_mapping().numpy()
+        self.tables = layout.block_tables.numpy()
+        self.lens = layout.context_lens.numpy()
+        lens = [int(c) for c in self.lens]
+        self.layer_bytes = layer_bytes(cfg, lens, layout.shares_prefix.tolist(), unique_prefix=True)["total"]
+        self.cores = oracle.num_threads()
+
+    def run(self, seconds: float):
+        """Whole layers until `seconds` have passed (at least one). Returns (bytes, seconds, seq-layers)."""
+        done_bytes, done_layers, t0 = 0, 0, time.perf_counter()
+        while True:
+            k2, v2 = self.oracle.kv_cache_append(self.k, self.v, self.kn, self.vn, self.slots)
+            self.oracle.paged_attention_decode(self.q, k2, v2, self.tables, self.lens, self.cfg.scale)
+            done_bytes += self.layer_bytes
+            done_layers += 1
+            if time.perf_counter() - t0 >= seconds:
+                break
+        return done_bytes, time.perf_counter() - t0, done_layers * self.cfg.batch
+
+
+def run_ours(args, world, rank, local):
+    import paged_kv_cache_470_b200 as pkv
+    cfg = workloads.CONFIGS[args.config]
+    device = torch.device("cuda", local if world > 1 else 0)
+    if args.compute:
+        pkv.set_option(pkv.KV_OPT_COMPUTE, {"tensor": 1, "cuda": 2}[args.compute])
+    wl = Workload(cfg, device, rank)
+    lens = [int(c) for c in wl.layout.context_lens]
+    share = wl.layout.shares_prefix.tolist()
+    lb_logical = layer_bytes(cfg, lens, share, unique_prefix=False)
+    lb_unique = layer_bytes(cfg, lens, share, unique_prefix=True)
+    step_bytes = lb_unique["total"] * cfg.n_layers
+
+    graph = capture(wl.step)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    with ClockSampler(device.index or 0) as clk:
+        ms = time_replays(graph, args.steps, world)
+    ms = dist_max(ms, world)
+    status = pkv.read_status(wl.ws)
+
+    # the decode kernel alone, for the roofline
+    kern_ms, n_launch = decode_kernel_duration_ms(wl)
+    kern_ms = dist_max(kern_ms, world)
+    peak, peak_kind = measured_peak()
+    kern_bytes = lb_unique["decode_kernel"]
+    achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
+    traffic = profiled_traffic()
+
+    e2e_ms, h2d, d2h = e2e_measure(wl, max(args.steps // 4, 3), args.warmup, world)
+    e2e_ms = dist_max(e2e_ms, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        sampler = OracleSampler(cfg, wl.layout)
+        b, s, nsl = sampler.run(args.cpu_seconds)
+        cpu = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": sampler.cores, "kind": "oracle",
+               "seq_layers_per_s": round(nsl / s, 2),
+               "sample": f"{nsl // cfg.batch} layer(s) of this workload (all {cfg.batch} sequences, append + "
+                         f"attention) in float64 on the host, {s:.1f} s"}
+
+    value = step_bytes * world / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "decode-attention achieved HBM GB/s (% of B200 peak); seq·layers/sec per step",
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "seq_layers_per_s": round(cfg.batch * cfg.n_layers * world / (ms * 1e-3), 1),
+        "pct_of_nominal_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
+        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+        "config": {"workload": cfg.name, "config_id": cfg.cid, "layers": cfg.n_layers, "batch": cfg.batch,
+                   "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "block_tokens": 16,
+                   "mean_context": round(sum(lens) / len(lens), 1),
+                   "kv_bytes_per_step": lb_unique["kv"] * cfg.n_layers,
+                   "kv_bytes_per_step_logical": lb_logical["kv"] * cfg.n_layers,
+                   "algorithmic_bytes_per_step": step_bytes,
+                   "l2": "inputs larger than L2: every step reads all layers' distinct caches "
+                         f"({lb_unique['kv'] * cfg.n_layers / 1e9:.2f} GB of KV vs 126 MB L2)",
+                   "timing": "CUDA-graph replay of the whole step, CUDA events, max over ranks",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": kern_bytes, "kernel_ms": round(kern_ms, 5),
+                     "launches_timed": n_launch, "peak_kind": f"{peak_kind} HBM copy bandwidth",
+                     "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)},
+        "e2e": {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "api": "kv_cache_append + paged_attention_decode per layer, captured in a CUDA graph with the copies"},
+        "gpu_launches": (2 if pkv.get_option(pkv.KV_OPT_COMBINE) == 0 else 3) * cfg.n_layers * args.steps,
+        "clocks": clk.summary(),
+        "device_status": status,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, world, rank):
+    """The oracle on the host cores, on bounded samples of the same workload."""
+    if rank != 0:
+        return
+    cfg = workloads.CONFIGS[args.config]
+    layout = workloads.draw_layout(cfg)
+    total_steps = args.steps + args.warmup
+    per_step = max(0.05, min(2.0, args.reference_budget / max(total_steps, 1)))
+    sampler = OracleSampler(cfg, layout)
+    cores = sampler.cores
+    for _ in range(args.warmup):
+        sampler.run(0.0)
+    b_all = s_all = n_all = 0
+    for _ in range(args.steps):
+        b, s, n = sampler.run(per_step)
+        b_all, s_all, n_all = b_all + b, s_all + s, n_all + n
+    value = b_all / s_all / 1e9
+    sample = (f"each step: whole layers of this workload (append + attention, all {cfg.batch} sequences) "
+              f"for about {per_step:.2f} s")
+    line = {"impl": "reference", "metric": "decode-attention achieved HBM GB/s (% of B200 peak); seq·layers/sec per step",
+            "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * s_all / args.steps, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "seq_layers_per_s": round(n_all / s_all, 2),
+            "config": {"workload": cfg.name, "config_id": cfg.cid},
+            "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", type=int, default=2, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--compute", choices=["tensor", "cuda"], default=None)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-budget", type=float, default=120.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

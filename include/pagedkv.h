@@ -1,0 +1,228 @@
+/*
+ * pagedkv.h -- C ABI of the paged KV cache decode library (libpagedkv.so).
+ *
+ * One decode step of a transformer layer over a paged KV cache:
+ *
+ *   kv_cache_append         scatter each new token's K and V rows into its slot
+ *   paged_attention_decode  out = softmax(scale * q K^T) V per query head,
+ *                           reading K/V through per-sequence block tables
+ *   kv_pool_*               host bookkeeping of physical blocks: allocate,
+ *                           free, and reference counts for shared prefixes
+ *
+ * Sources for what is computed:
+ *   - "Module 23: Serving", section 23.4 (Paged Attention): the cache lives in
+ *     fixed-size blocks of 16 tokens, allocated as a sequence grows, with a
+ *     per-sequence table mapping positions to blocks; sequences that share a
+ *     prefix can share its blocks.
+ *   - "Designing an LLM serving system", section "Paged attention": a page
+ *     table per sequence; logical positions map to physical blocks through an
+ *     indirection; shared blocks for a common prompt.
+ *   - "Scaling LLM serving", section "The KV cache" (Share key/value heads):
+ *     grouped-query attention, each key/value head shared by a group of query
+ *     heads. Groups are contiguous: query head h reads kv head h / (Hq / Hkv).
+ *   - "Module 23: Serving", section 23.2 (Prefill and Decode): a decode step
+ *     reads the whole KV cache for one new token per sequence.
+ *
+ * Conventions for every call:
+ *   - Device pointers are CUDA global-memory addresses on the current device.
+ *     The caller owns every buffer, the workspace included. The library never
+ *     allocates or frees device memory and never synchronises, except where a
+ *     call says so (paged_attention_read_status).
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Work is
+ *     enqueued on it; kernels are launched with programmatic dependent launch,
+ *     so consecutive calls on one stream may overlap their prologues. All calls
+ *     that launch work can be captured into a CUDA graph.
+ *   - Return value: KV_OK (0) or a negative kv_status. Argument checks happen on
+ *     the host before anything is enqueued; on KV_ERR_ARG nothing is launched.
+ *     KV_ERR_CUDA means a launch failed (cudaGetLastError was not cudaSuccess).
+ *   - Element type: dtype must be KV_DTYPE_BF16. Head dimension D must be 64 or
+ *     128. Block size is fixed at KV_BLOCK_TOKENS = 16 tokens.
+ *
+ * Layouts (row-major):
+ *   k_cache, v_cache   [num_blocks][16][Hkv][D]  bf16, one tensor each for K, V
+ *   q, out             [B][Hq][D]               bf16
+ *   k_new, v_new       [T][Hkv][D]              bf16
+ *   slot_mapping       [T]                      int64; slot = block*16 + offset,
+ *                                                negative = padding (skipped)
+ *   block_tables       [B][W]                   int32 physical block ids; row b
+ *                                                holds ceil(context_lens[b]/16)
+ *                                                valid entries, the rest unread
+ *   context_lens       [B]                      int32 tokens cached for sequence
+ *                                                b, this step's token included
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KV_API __attribute__((visibility("default")))
+#else
+#define KV_API
+#endif
+
+typedef int kv_status;
+
+#define KV_OK 0
+#define KV_ERR_ARG (-1)    /* bad argument; nothing was done                       */
+#define KV_ERR_OOM (-2)    /* block pool has too few free blocks; nothing changed  */
+#define KV_ERR_STATE (-3)  /* pool state forbids it (free of a free block, ...)    */
+#define KV_ERR_CUDA (-4)   /* a CUDA runtime call failed                           */
+
+#define KV_DTYPE_BF16 0
+#define KV_BLOCK_TOKENS 16
+
+/* Bits of the device status word kept in the attention workspace. */
+#define KV_STATUS_BAD_BLOCK_ID 1   /* a table entry was outside [0, num_blocks)   */
+#define KV_STATUS_BAD_CONTEXT 2    /* a context length was < 0 or > 16 * W        */
+#define KV_STATUS_WAIT_TIMEOUT 4   /* an internal pipeline wait gave up (~1 s)    */
+#define KV_STATUS_BAD_SLOT 8       /* an append slot was >= num_blocks * 16       */
+
+typedef struct CUstream_st *kv_stream_t; /* same type as cudaStream_t */
+
+/* ------------------------------------------------------------------------ */
+/* Append ("Module 23: Serving", 23.4: blocks are filled as a sequence grows) */
+/* ------------------------------------------------------------------------ */
+/*
+ * For every i in [0, T) with slot_mapping[i] >= 0:
+ *   k_cache[slot/16][slot%16][:][:] = k_new[i][:][:]   (all Hkv heads, bitwise)
+ *   v_cache[slot/16][slot%16][:][:] = v_new[i][:][:]
+ * Every other cache byte is left unchanged. Non-negative slots must be
+ * distinct (two tokens writing one slot race). A slot >= num_blocks*16 is not
+ * written; if error_flag is non-NULL (a device int32), KV_STATUS_BAD_SLOT is
+ * OR-ed into it. All pointers are device pointers, 16-byte aligned.
+ * T = 0 is a no-op.
+ */
+KV_API kv_status kv_cache_append(const void *k_new, const void *v_new,
+                          void *k_cache, void *v_cache,
+                          const int64_t *slot_mapping, int T,
+                          int num_blocks, int Hkv, int D, int dtype,
+                          int32_t *error_flag, kv_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Decode attention ("Module 23: Serving", 23.2 and 23.4; "Scaling LLM       */
+/* serving", "The KV cache")                                                 */
+/* ------------------------------------------------------------------------ */
+/*
+ * Bytes of device workspace paged_attention_decode needs for these sizes on
+ * the current device (it depends on the device's SM count). Returns 0 for
+ * invalid sizes. The workspace holds a status word, split-K partial results
+ * and one counter per (sequence, kv head) work item.
+ */
+KV_API size_t paged_attention_workspace_size(int B, int Hq, int Hkv, int D);
+
+/*
+ * Zero a workspace (cudaMemsetAsync on `stream`). A workspace must be zeroed
+ * once before its first use, and again after a call reported
+ * KV_STATUS_WAIT_TIMEOUT; between calls it stays valid by itself.
+ */
+KV_API kv_status paged_attention_workspace_init(void *workspace, size_t workspace_bytes,
+                                         kv_stream_t stream);
+
+/*
+ * For each sequence b with c = context_lens[b], each query head h in [0, Hq)
+ * and j = h / (Hq / Hkv):
+ *   K_t = k_cache[block_tables[b][t/16]][t%16][j][:],  V_t likewise, t < c
+ *   out[b][h][:] = sum_t softmax_t(scale * <q[b][h], K_t>) V_t
+ * computed with fp32 arithmetic (bf16 inputs, bf16 output). c = 0 gives
+ * out[b][h][:] = 0. The result does not depend on which physical blocks hold
+ * the tokens, only on the logical order, and is bitwise reproducible.
+ *
+ * q, out, k_cache, v_cache, block_tables, context_lens, workspace: device
+ * pointers (the first four 16-byte aligned, workspace 256-byte aligned).
+ * workspace_bytes must be >= paged_attention_workspace_size(B, Hq, Hkv, D).
+ * Requirements: B >= 0, W >= 1, num_blocks >= 1, Hq % Hkv == 0, D in {64, 128}.
+ * Bad table entries or context lengths are not checked on the host (the data
+ * is on the device): the kernel never reads outside the cache or the table
+ * row, and records KV_STATUS_BAD_BLOCK_ID / KV_STATUS_BAD_CONTEXT in the
+ * workspace status word (see paged_attention_read_status); the output of an
+ * affected sequence is then unspecified.
+ * Concurrent calls must not share a workspace.
+ */
+KV_API kv_status paged_attention_decode(void *out, const void *q,
+                                 const void *k_cache, const void *v_cache,
+                                 const int32_t *block_tables, int max_blocks_per_seq,
+                                 const int32_t *context_lens, int B,
+                                 int num_blocks, int Hq, int Hkv, int D,
+                                 float scale, int dtype,
+                                 void *workspace, size_t workspace_bytes,
+                                 kv_stream_t stream);
+
+/*
+ * Copy the workspace status word to *status_out (host int32), synchronising
+ * `stream` first; if clear != 0, reset it to 0 afterwards. 0 = no error seen.
+ */
+KV_API kv_status paged_attention_read_status(const void *workspace, int32_t *status_out,
+                                      int clear, kv_stream_t stream);
+
+/*
+ * Process-wide tuning switches (defaults are the tuned choices).
+ *   KV_OPT_COMPUTE:   0 auto, 1 tensor cores (mma.sync bf16), 2 CUDA cores
+ *   KV_OPT_COMBINE:   0 split-K merge fused into the last CTA of each work
+ *                     item, 1 separate combine kernel
+ *   KV_OPT_GRID:      0 auto (CTAs resident on all SMs), n > 0 launch n CTAs
+ *                     (n is capped by what the workspace was sized for)
+ *   KV_OPT_MIN_CHUNK: 0 auto, n > 0 minimum KV blocks per CTA
+ * Returns KV_ERR_ARG for an unknown key or value.
+ */
+#define KV_OPT_COMPUTE 1
+#define KV_OPT_COMBINE 2
+#define KV_OPT_GRID 3
+#define KV_OPT_MIN_CHUNK 4
+KV_API kv_status kv_decode_set_option(int key, int value);
+KV_API int kv_decode_get_option(int key);
+
+/* ------------------------------------------------------------------------ */
+/* Host block pool ("Module 23: Serving", 23.4; "Designing an LLM serving    */
+/* system", "Paged attention" and "Caching and shortcuts": prefix caching)   */
+/* ------------------------------------------------------------------------ */
+/*
+ * An opaque host object tracking which of num_blocks physical blocks are free
+ * and how many sequences reference each used block. It owns no device memory.
+ * Calls on one pool are serialised by an internal mutex.
+ */
+KV_API kv_status kv_pool_create(int num_blocks, void **pool_out);
+KV_API void kv_pool_destroy(void *pool);
+
+/* n fresh blocks (refcount 1 each) into ids_out[0..n), or KV_ERR_OOM with no
+ * change if fewer than n are free. */
+KV_API kv_status kv_pool_alloc(void *pool, int n, int32_t *ids_out);
+
+/* One more reference to each listed block (a sequence sharing a prefix).
+ * KV_ERR_STATE, with no change, if any listed block is free or out of range. */
+KV_API kv_status kv_pool_incref(void *pool, const int32_t *ids, int n);
+
+/* Drop one reference per listed entry; a block whose count reaches 0 becomes
+ * free. KV_ERR_STATE, with no change, if that would take any count below 0. */
+KV_API kv_status kv_pool_free(void *pool, const int32_t *ids, int n);
+
+KV_API int kv_pool_num_free(const void *pool);
+KV_API int kv_pool_num_blocks(const void *pool);
+/* Reference count of block id, or -1 if id is out of range. */
+KV_API int kv_pool_refcount(const void *pool, int32_t id);
+
+/*
+ * Host bookkeeping for one decode step of B sequences (host arrays):
+ * sequence b currently caches context_lens[b] = c tokens; its new token goes
+ * to position c. If c % 16 == 0 a fresh block is allocated and stored at
+ * block_tables[b*W + c/16]. slot_mapping_out[b] = block*16 + c%16, and
+ * context_lens[b] becomes c + 1. All or nothing: KV_ERR_OOM if the pool lacks
+ * the blocks, KV_ERR_ARG if a sequence would exceed W blocks, KV_ERR_STATE if
+ * the new token would land in a block shared with another sequence (refcount
+ * > 1; copy-on-write is the caller's job). Nothing changes on error.
+ * Afterwards each sequence holds exactly ceil(c'/16) blocks.
+ */
+KV_API kv_status kv_pool_append_slots(void *pool, int32_t *block_tables, int W,
+                               int32_t *context_lens, int B,
+                               int64_t *slot_mapping_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

@@ -1,0 +1,211 @@
+"""Python binding of libpagedkv.so (the C ABI declared in include/pagedkv.h).
+
+Argument marshalling only: every step of a decode (append, attention, split-K
+merge) runs in the library's CUDA kernels, and the block pool runs in its C++
+code. PyTorch supplies device memory and the stream. There is no fallback: if
+the shared library is missing, importing this package raises ImportError.
+
+Build it with ``python paged_kv_cache_470_b200/build.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python paged_kv_cache_470_b200/build.py`")
+_lib = ctypes.CDLL(LIB_PATH)
+
+KV_OK, KV_ERR_ARG, KV_ERR_OOM, KV_ERR_STATE, KV_ERR_CUDA = 0, -1, -2, -3, -4
+KV_DTYPE_BF16 = 0
+BLOCK_TOKENS = 16
+KV_STATUS_BAD_BLOCK_ID, KV_STATUS_BAD_CONTEXT, KV_STATUS_WAIT_TIMEOUT, KV_STATUS_BAD_SLOT = 1, 2, 4, 8
+KV_OPT_COMPUTE, KV_OPT_COMBINE, KV_OPT_GRID, KV_OPT_MIN_CHUNK = 1, 2, 3, 4
+COMPUTE_AUTO, COMPUTE_TENSOR_CORES, COMPUTE_CUDA_CORES = 0, 1, 2
+
+_P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_sig = {
+    "kv_cache_append": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "paged_attention_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "paged_attention_workspace_init": (_I, [_P, _SZ, _P]),
+    "paged_attention_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _SZ,
+                                    _P]),
+    "paged_attention_read_status": (_I, [_P, _P, _I, _P]),
+    "kv_decode_set_option": (_I, [_I, _I]),
+    "kv_decode_get_option": (_I, [_I]),
+    "kv_pool_create": (_I, [_I, ctypes.POINTER(ctypes.c_void_p)]),
+    "kv_pool_destroy": (None, [_P]),
+    "kv_pool_alloc": (_I, [_P, _I, _P]),
+    "kv_pool_incref": (_I, [_P, _P, _I]),
+    "kv_pool_free": (_I, [_P, _P, _I]),
+    "kv_pool_num_free": (_I, [_P]),
+    "kv_pool_num_blocks": (_I, [_P]),
+    "kv_pool_refcount": (_I, [_P, ctypes.c_int32]),
+    "kv_pool_append_slots": (_I, [_P, _P, _I, _P, _I, _P]),
+}
+for _name, (_res, _args) in _sig.items():
+    _f = getattr(_lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+EXPORTED = tuple(_sig)
+
+
+class KVError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        names = {KV_ERR_ARG: "KV_ERR_ARG", KV_ERR_OOM: "KV_ERR_OOM", KV_ERR_STATE: "KV_ERR_STATE",
+                 KV_ERR_CUDA: "KV_ERR_CUDA"}
+        super().__init__(f"{call} failed: {names.get(status, status)}")
+        self.status = status
+
+
+def _check(call: str, status: int) -> None:
+    if status != KV_OK:
+        raise KVError(call, status)
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream or None
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream or None
+    return int(stream) or None
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+# ---------------------------------------------------------------------------
+# kernels
+# ---------------------------------------------------------------------------
+def kv_cache_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                    slot_mapping: torch.Tensor, error_flag: torch.Tensor | None = None, stream=None) -> None:
+    """Scatter k_new/v_new [T,Hkv,D] into the caches [num_blocks,16,Hkv,D] at slot_mapping [T] (int64)."""
+    T, Hkv, D = k_new.shape
+    num_blocks = k_cache.shape[0]
+    ef = _dev(error_flag, "error_flag", torch.int32) if error_flag is not None else None
+    _check("kv_cache_append", _lib.kv_cache_append(
+        _dev(k_new, "k_new", torch.bfloat16), _dev(v_new, "v_new", torch.bfloat16),
+        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(slot_mapping, "slot_mapping", torch.int64), T, num_blocks, Hkv, D, KV_DTYPE_BF16, ef,
+        _stream_handle(stream)))
+
+
+def workspace_size(B: int, Hq: int, Hkv: int, D: int) -> int:
+    n = _lib.paged_attention_workspace_size(B, Hq, Hkv, D)
+    if n == 0:
+        raise KVError("paged_attention_workspace_size", KV_ERR_ARG)
+    return int(n)
+
+
+def make_workspace(B: int, Hq: int, Hkv: int, D: int, device=None) -> torch.Tensor:
+    """A zeroed workspace (uint8) sized for these shapes on the current device."""
+    return torch.zeros(workspace_size(B, Hq, Hkv, D), dtype=torch.uint8, device=device or "cuda")
+
+
+def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                           block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                           workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """out[B,Hq,D] = softmax(scale * q K^T) V over each sequence's paged cache."""
+    B, Hq, D = q.shape
+    num_blocks, _, Hkv, Dk = k_cache.shape
+    if Dk != D or tuple(out.shape) != (B, Hq, D) or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch")
+    _check("paged_attention_decode", _lib.paged_attention_decode(
+        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
+        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), KV_DTYPE_BF16,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
+    return out
+
+
+def read_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
+    """Synchronise the stream and return (optionally clearing) the device status word."""
+    v = ctypes.c_int32(0)
+    _check("paged_attention_read_status", _lib.paged_attention_read_status(
+        _dev(workspace, "workspace", torch.uint8), ctypes.byref(v), int(clear), _stream_handle(stream)))
+    return int(v.value)
+
+
+def set_option(key: int, value: int) -> None:
+    _check("kv_decode_set_option", _lib.kv_decode_set_option(key, value))
+
+
+def get_option(key: int) -> int:
+    return int(_lib.kv_decode_get_option(key))
+
+
+# ---------------------------------------------------------------------------
+# host block pool
+# ---------------------------------------------------------------------------
+def _i32(a) -> ctypes.Array:
+    return (ctypes.c_int32 * len(a))(*[int(x) for x in a])
+
+
+class BlockPool:
+    """Reference-counted physical block ids (host only; owns no device memory)."""
+
+    def __init__(self, num_blocks: int):
+        h = ctypes.c_void_p()
+        _check("kv_pool_create", _lib.kv_pool_create(num_blocks, ctypes.byref(h)))
+        self._h = h
+
+    def close(self) -> None:
+        if self._h:
+            _lib.kv_pool_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    @property
+    def handle(self):
+        return self._h
+
+    def alloc(self, n: int) -> list[int]:
+        buf = (ctypes.c_int32 * max(n, 1))()
+        _check("kv_pool_alloc", _lib.kv_pool_alloc(self._h, n, buf))
+        return list(buf[:n])
+
+    def incref(self, ids) -> None:
+        ids = list(ids)
+        _check("kv_pool_incref", _lib.kv_pool_incref(self._h, _i32(ids), len(ids)))
+
+    def free(self, ids) -> None:
+        ids = list(ids)
+        _check("kv_pool_free", _lib.kv_pool_free(self._h, _i32(ids), len(ids)))
+
+    def num_free(self) -> int:
+        return int(_lib.kv_pool_num_free(self._h))
+
+    def num_blocks(self) -> int:
+        return int(_lib.kv_pool_num_blocks(self._h))
+
+    def refcount(self, block_id: int) -> int:
+        return int(_lib.kv_pool_refcount(self._h, block_id))
+
+    def append_slots(self, block_tables: torch.Tensor, context_lens: torch.Tensor, slot_mapping: torch.Tensor) -> None:
+        """One decode step of bookkeeping on host tensors (int32 [B,W], int32 [B], int64 [B]), in place."""
+        for t, name, dt in ((block_tables, "block_tables", torch.int32), (context_lens, "context_lens", torch.int32),
+                            (slot_mapping, "slot_mapping", torch.int64)):
+            if t.is_cuda or not t.is_contiguous() or t.dtype != dt:
+                raise ValueError(f"{name} must be a contiguous host {dt} tensor")
+        B, W = block_tables.shape
+        _check("kv_pool_append_slots", _lib.kv_pool_append_slots(
+            self._h, block_tables.data_ptr(), W, context_lens.data_ptr(), B, slot_mapping.data_ptr()))

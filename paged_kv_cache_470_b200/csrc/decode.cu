@@ -1,0 +1,1101 @@
+// paged_attention_decode: one decode step of grouped-query attention over a
+// paged KV cache, for sm_100a.
+//
+// What is computed ("Module 23: Serving", sections 23.2 and 23.4; "Scaling LLM
+// serving", section "The KV cache"): for sequence b with c cached tokens and
+// query head h, with kv head j = h / (Hq / Hkv),
+//     out[b][h] = sum_t softmax_t(scale * <q[b][h], K_t>) V_t,   t < c,
+// where token t lives in physical block block_tables[b][t / 16], row t % 16.
+//
+// Work decomposition. A work item is (sequence b, kv head j, chunk of at most
+// 8 query heads of j's group); its work units are the ceil(c/16) KV blocks of
+// the sequence. All units of all items are laid end to end and cut into
+// equal contiguous ranges, one per CTA (the grid is sized to be resident on
+// every SM at once). A CTA therefore handles whole items and at most two
+// partial items; an item cut between CTAs is a split-K item: each piece
+// produces (running max, running sum, unnormalised accumulator) in fp32 and a
+// log-sum-exp merge joins them. The merge runs in the last CTA to finish a
+// piece of that item (an atomic counter, no spinning), or, as an option, in a
+// separate combine kernel.
+//
+// Inside a CTA: warp 4 is the producer. It reads block ids from the table and
+// issues TMA tile loads of the item's 16 K rows and 16 V rows (one 128-byte
+// swizzled box per 64 columns) into a ring of shared-memory stages guarded by
+// mbarriers. Warps 0-3 consume units round robin, each keeping an fp32 online
+// softmax (running max and sum per query head) and its own accumulator; at the
+// end of an item the four warps are merged through shared memory.
+//
+// Two consumer arithmetic paths:
+//  * tensor cores: S^T[16 tokens x 8 heads] = K_blk * Q^T with
+//    mma.sync.m16n8k16 (bf16 in, fp32 accumulate; the 16 tokens of a block are
+//    the M dimension, the group's query heads the N dimension), then
+//    O^T[D x 8] += V_blk^T * P^T, with the probabilities split into a bf16
+//    high part and a bf16 residual so that P keeps ~16 significant bits.
+//  * CUDA cores: fp32 FMAs on values unpacked from bf16.
+#include "pkv_device.cuh"
+#include "pagedkv.h"
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+namespace pkv {
+
+constexpr int kThreads = 160;
+constexpr int kConsumerWarps = 4;
+constexpr int kConsumerThreads = kConsumerWarps * 32;
+constexpr int kProducerWarp = 4;
+constexpr int kGroupMax = 8;             // query heads per work item
+constexpr int kTileBytes = 16 * 128;     // one TMA box: 16 rows x 64 bf16, 128B-swizzled
+constexpr int kCtasPerSm = 2;
+constexpr int kStatusBytes = 256;
+constexpr unsigned kFull = 0xffffffffu;
+
+enum ComputePath { kPathMma = 1, kPathSimt = 2 };
+
+template <int D>
+struct Geo {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int kTiles = D / 64;
+    static constexpr int kStageBytes = 2 * kTiles * kTileBytes;   // K and V of one block
+    // A multiple of the consumer-warp count, so stage s is always consumed by
+    // warp s % 4, in order: a warp never waits on round r+1 of a stage whose
+    // round r another warp has not consumed yet (the parity wait could not
+    // tell those two rounds apart).
+    static constexpr int kStages = ((80 * 1024) / kStageBytes) / kConsumerWarps * kConsumerWarps;  // 20 or 8
+    static_assert(kStages % kConsumerWarps == 0, "stage ownership must be fixed per warp");
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kAccStride = D + 4;                      // padded: conflict-free scratch writes
+    static constexpr int kQStride = D + 8;                        // second half shifted by 4 floats
+    static constexpr int kOffAcc = kRingBytes;
+    static constexpr int kOffMl = kOffAcc + kConsumerWarps * kGroupMax * kAccStride * 4;
+    static constexpr int kOffQ = kOffMl + kConsumerWarps * kGroupMax * 2 * 4;
+    static constexpr int kOffP = kOffQ + kGroupMax * kQStride * 4;
+    static constexpr int kOffBar = kOffP + kConsumerWarps * 16 * kGroupMax * 4;
+    static constexpr int kOffMisc = kOffBar + 2 * kStages * 8;
+    static constexpr int kMiscInts = 16;
+    static constexpr int kSmemBytes = kOffMisc + kMiscInts * 4 + 1024;  // + room to align the base
+};
+
+struct DecodeArgs {
+    __nv_bfloat16 *out;
+    const __nv_bfloat16 *q;
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    float *part_acc;     // [slots][8][D]
+    float *part_ml;      // [slots][8][2]  (max in log2 units, sum)
+    int32_t *counters;   // [items]
+    int32_t *status;
+    int B, W, Hq, Hkv, group, hchunks, items_per_seq, num_blocks;
+    int min_chunk;
+    int fused;
+    float scale_log2;    // scale * log2(e)
+};
+
+// misc ints in shared memory
+enum { kMiscAbort = 0, kMiscLocB = 1, kMiscLocR = 2, kMiscLast = 3, kMiscZero = 4, kMiscWarpSums = 8 };
+
+__device__ __forceinline__ int clamp_ctx(int c, int W)
+{
+    return c < 0 ? 0 : (c > W * kBlockTokens ? W * kBlockTokens : c);
+}
+__device__ __forceinline__ int seq_ctx(const DecodeArgs &a, int b) { return clamp_ctx(__ldg(a.context_lens + b), a.W); }
+__device__ __forceinline__ int ctx_blocks(int c) { return (c + kBlockTokens - 1) / kBlockTokens; }
+
+// Inclusive scan over the 160 threads; *total receives the sum of all values.
+__device__ __forceinline__ int block_scan_incl(int v, volatile int *warp_sums, int *total)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o)
+            x += y;
+    }
+    if (lane == 31)
+        warp_sums[warp] = x;
+    __syncthreads();
+    int pre = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) {
+        const int s = warp_sums[w];
+        pre += (w < warp) ? s : 0;
+        tot += s;
+    }
+    __syncthreads();
+    *total = tot;
+    return x + pre;
+}
+
+struct Cursor {
+    int b;     // sequence
+    int k;     // item within the sequence: j * hchunks + head chunk
+    int off;   // block offset within the sequence
+    int ctx;   // tokens of sequence b (clamped)
+    int n;     // blocks of sequence b
+};
+
+__device__ __forceinline__ void cursor_next_item(const DecodeArgs &a, Cursor &c)
+{
+    c.off = 0;
+    if (++c.k == a.items_per_seq) {
+        c.k = 0;
+        do {
+            ++c.b;
+            c.ctx = (c.b < a.B) ? seq_ctx(a, c.b) : 0;
+            c.n = ctx_blocks(c.ctx);
+        } while (c.n == 0 && c.b < a.B);
+    }
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t addr)
+{
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t addr)
+{
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+__device__ __forceinline__ void sts128_zero(uint32_t addr)
+{
+    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(addr), "r"(0) : "memory");
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128B-swizzled box.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+// ---------------------------------------------------------------------------
+// Per-warp consumer state and arithmetic.
+// ---------------------------------------------------------------------------
+template <int D, int PATH, int NH>
+struct Consumer;
+
+// Tensor-core path. Lane (r = lane/4, c = lane%4) holds scores of tokens r and
+// r+8 for heads 2c and 2c+1, and the accumulator O^T rows d = 16*mt + r (+8)
+// for the same two heads.
+template <int D, int NH>
+struct Consumer<D, kPathMma, NH> {
+    static constexpr int kTiles = D / 64;
+    static constexpr int kMt = D / 16;
+    uint32_t qf[kMt][2];
+    float acc[kMt][4];
+    float m0, m1, l0, l1;
+
+    __device__ __forceinline__ void begin_item(const DecodeArgs &a, int b, int h0, int gc, float *)
+    {
+        const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q + (static_cast<size_t>(b) * a.Hq + h0 + r) * D);
+#pragma unroll
+        for (int kk = 0; kk < kMt; ++kk) {
+            qf[kk][0] = (r < gc) ? __ldg(qrow + kk * 8 + c) : 0u;
+            qf[kk][1] = (r < gc) ? __ldg(qrow + kk * 8 + 4 + c) : 0u;
+        }
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt)
+            acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
+    }
+
+    __device__ __forceinline__ void unit(uint32_t kbase, uint32_t vbase, int valid, float sl2, float *)
+    {
+        const int lane = threadIdx.x & 31, r = lane >> 2, mi = lane >> 3, rr = lane & 7;
+        if (valid < 16) {
+            // rows past the context hold whatever the pool holds; zero them so 0 * V stays 0
+            const int rows = 16 - valid;
+            for (int idx = lane; idx < rows * 8 * kTiles; idx += 32) {
+                const int t = idx / (8 * kTiles);
+                const int rem = idx - t * 8 * kTiles;
+                const int tile = rem >> 3, ch = rem & 7;
+                sts128_zero(vbase + tile * kTileBytes + (valid + t) * 128 + ch * 16);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+        }
+        // S^T = K_blk [16 x D] * Q^T [D x 8]
+        float s[4] = {0.f, 0.f, 0.f, 0.f};
+        {
+            const int row = ((mi & 1) << 3) + rr;
+#pragma unroll
+            for (int kk = 0; kk < kMt; ++kk) {
+                const int tile = kk >> 2, kc = kk & 3;
+                uint32_t af[4];
+                ldmatrix_x4(af, kbase + tile * kTileBytes + swz(row, (kc << 1) + (mi >> 1)));
+                mma_bf16_16816(s, af, qf[kk][0], qf[kk][1]);
+            }
+        }
+        const bool v0 = r < valid, v1 = (r + 8) < valid;
+        const float s0 = v0 ? s[0] * sl2 : -INFINITY;
+        const float s1 = v0 ? s[1] * sl2 : -INFINITY;
+        const float s2 = v1 ? s[2] * sl2 : -INFINITY;
+        const float s3 = v1 ? s[3] * sl2 : -INFINITY;
+        float bm0 = fmaxf(s0, s2), bm1 = fmaxf(s1, s3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, o));
+            bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, o));
+        }
+        const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
+        const float al0 = exp2f(m0 - mn0), al1 = exp2f(m1 - mn1);
+        m0 = mn0;
+        m1 = mn1;
+        const float p0 = exp2f(s0 - mn0), p1 = exp2f(s1 - mn1);
+        const float p2 = exp2f(s2 - mn0), p3 = exp2f(s3 - mn1);
+        l0 = l0 * al0 + (p0 + p2);
+        l1 = l1 * al1 + (p1 + p3);
+        // P^T as bf16 high part plus bf16 residual, transposed into B fragments
+        const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
+        const uint32_t r01 = pack_bf16x2(p0 - bf16lo_to_f32(h01), p1 - bf16hi_to_f32(h01));
+        const uint32_t r23 = pack_bf16x2(p2 - bf16lo_to_f32(h23), p3 - bf16hi_to_f32(h23));
+        const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
+        const uint32_t bl0 = movmatrix_trans(r01), bl1 = movmatrix_trans(r23);
+        // O^T [D x 8] += V_blk^T [D x 16] * P^T [16 x 8]
+        const int vrow = ((mi >> 1) << 3) + rr;
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt) {
+            acc[mt][0] *= al0;
+            acc[mt][1] *= al1;
+            acc[mt][2] *= al0;
+            acc[mt][3] *= al1;
+            const int tile = mt >> 2, kc = mt & 3;
+            uint32_t af[4];
+            ldmatrix_x4_trans(af, vbase + tile * kTileBytes + swz(vrow, (kc << 1) + (mi & 1)));
+            mma_bf16_16816(acc[mt], af, bh0, bh1);
+            mma_bf16_16816(acc[mt], af, bl0, bl1);
+        }
+    }
+
+    // Write this warp's (m, l, acc) for heads 0..7 into the merge scratch.
+    __device__ __forceinline__ void finish(float *acc_w, float *ml_w)
+    {
+        const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            l0 += __shfl_xor_sync(kFull, l0, o);
+            l1 += __shfl_xor_sync(kFull, l1, o);
+        }
+        constexpr int AS = Geo<D>::kAccStride;
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt) {
+            const int d = mt * 16 + r;
+            acc_w[(2 * c) * AS + d] = acc[mt][0];
+            acc_w[(2 * c + 1) * AS + d] = acc[mt][1];
+            acc_w[(2 * c) * AS + d + 8] = acc[mt][2];
+            acc_w[(2 * c + 1) * AS + d + 8] = acc[mt][3];
+        }
+        if (r == 0) {
+            ml_w[(2 * c) * 2] = m0;
+            ml_w[(2 * c) * 2 + 1] = l0;
+            ml_w[(2 * c + 1) * 2] = m1;
+            ml_w[(2 * c + 1) * 2 + 1] = l1;
+        }
+    }
+};
+
+// CUDA-core path. QK: lane (t = lane/2, half = lane%2) dots token t's half row
+// with every head; PV: lane owns D/32 output columns for every head.
+template <int D, int NH>
+struct Consumer<D, kPathSimt, NH> {
+    static constexpr int E = D / 32;
+    static constexpr int CPH = D / 16;
+    float acc[NH][E];
+    float m[NH], l[NH];
+
+    __device__ __forceinline__ void begin_item(const DecodeArgs &, int, int, int, float *)
+    {
+#pragma unroll
+        for (int n = 0; n < NH; ++n) {
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                acc[n][e] = 0.f;
+            m[n] = -INFINITY;
+            l[n] = 0.f;
+        }
+    }
+
+    // q_s: [8][kQStride] fp32 (filled by the CTA), p_s: this warp's [16][8] fp32
+    __device__ __forceinline__ void unit(uint32_t kbase, uint32_t vbase, int valid, float sl2, float *qp)
+    {
+        constexpr int QS = Geo<D>::kQStride;
+        const float *q_s = qp;
+        float *p_s = qp + kGroupMax * QS + (threadIdx.x >> 5) * 16 * kGroupMax;
+        const int lane = threadIdx.x & 31, t = lane >> 1, half = lane & 1;
+        float dot[NH];
+#pragma unroll
+        for (int n = 0; n < NH; ++n)
+            dot[n] = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < CPH; ++cc) {
+            const int dcol = half * (D / 2) + cc * 8;
+            const uint4 kv = lds128(kbase + (dcol >> 6) * kTileBytes + swz(t, (dcol & 63) >> 3));
+            const float k0 = bf16lo_to_f32(kv.x), k1 = bf16hi_to_f32(kv.x), k2 = bf16lo_to_f32(kv.y),
+                        k3 = bf16hi_to_f32(kv.y), k4 = bf16lo_to_f32(kv.z), k5 = bf16hi_to_f32(kv.z),
+                        k6 = bf16lo_to_f32(kv.w), k7 = bf16hi_to_f32(kv.w);
+            const float *qs = q_s + dcol + half * 4;
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                const float4 qa = *reinterpret_cast<const float4 *>(qs + n * QS);
+                const float4 qb = *reinterpret_cast<const float4 *>(qs + n * QS + 4);
+                float x = dot[n];
+                x = fmaf(k0, qa.x, x);
+                x = fmaf(k1, qa.y, x);
+                x = fmaf(k2, qa.z, x);
+                x = fmaf(k3, qa.w, x);
+                x = fmaf(k4, qb.x, x);
+                x = fmaf(k5, qb.y, x);
+                x = fmaf(k6, qb.z, x);
+                x = fmaf(k7, qb.w, x);
+                dot[n] = x;
+            }
+        }
+        float al[NH];
+#pragma unroll
+        for (int n = 0; n < NH; ++n) {
+            const float full_dot = dot[n] + __shfl_xor_sync(kFull, dot[n], 1);
+            const float sv = (t < valid) ? full_dot * sl2 : -INFINITY;
+            float bm = sv;
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1)
+                bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, o));
+            const float mn = fmaxf(m[n], bm);
+            al[n] = exp2f(m[n] - mn);
+            m[n] = mn;
+            const float p = exp2f(sv - mn);
+            l[n] = l[n] * al[n] + p;
+            if (half == 0)
+                p_s[t * kGroupMax + n] = p;
+        }
+        __syncwarp();
+        const int d0 = lane * E;
+        const uint32_t vcol = (d0 >> 6) * kTileBytes;
+        const int chunk = (d0 & 63) >> 3, within = d0 & 7;
+#pragma unroll
+        for (int n = 0; n < NH; ++n)
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                acc[n][e] *= al[n];
+        for (int tt = 0; tt < valid; ++tt) {
+            const uint32_t addr = vbase + vcol + swz(tt, chunk) + within * 2;
+            float v[E];
+            if constexpr (E == 4) {
+                const uint2 w = lds64(addr);
+                v[0] = bf16lo_to_f32(w.x);
+                v[1] = bf16hi_to_f32(w.x);
+                v[2] = bf16lo_to_f32(w.y);
+                v[3] = bf16hi_to_f32(w.y);
+            } else {
+                const uint32_t w = lds32(addr);
+                v[0] = bf16lo_to_f32(w);
+                v[1] = bf16hi_to_f32(w);
+            }
+            const float *pr = p_s + tt * kGroupMax;
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                const float pn = pr[n];
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    acc[n][e] = fmaf(pn, v[e], acc[n][e]);
+            }
+        }
+        __syncwarp();
+    }
+
+    __device__ __forceinline__ void finish(float *acc_w, float *ml_w)
+    {
+        const int lane = threadIdx.x & 31;
+        constexpr int AS = Geo<D>::kAccStride;
+#pragma unroll
+        for (int n = 0; n < kGroupMax; ++n) {
+            float ln = 0.f, mn = -INFINITY;
+            if (n < NH) {
+                ln = l[n];
+#pragma unroll
+                for (int o = 2; o < 32; o <<= 1)
+                    ln += __shfl_xor_sync(kFull, ln, o);
+                mn = m[n];
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                acc_w[n * AS + lane * E + e] = (n < NH) ? acc[n < NH ? n : 0][e] : 0.f;
+            if (lane == 0) {
+                ml_w[n * 2] = mn;
+                ml_w[n * 2 + 1] = ln;
+            }
+        }
+    }
+};
+
+// Log-sum-exp merge of split-K pieces of one item, read from global memory.
+template <int D>
+__device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int item, int first_cta, int last_cta,
+                                                    int b, int h0, int gc, int tid, int nthreads)
+{
+    for (int idx = tid; idx < gc * D; idx += nthreads) {
+        const int n = idx / D, d = idx - n * D;
+        float M = -INFINITY;
+        for (int c = first_cta; c <= last_cta; ++c)
+            M = fmaxf(M, __ldcg(a.part_ml + ((static_cast<size_t>(c) + item) * kGroupMax + n) * 2));
+        float L = 0.f, O = 0.f;
+        for (int c = first_cta; c <= last_cta; ++c) {
+            const size_t slot = static_cast<size_t>(c) + item;
+            const float sc = exp2f(__ldcg(a.part_ml + (slot * kGroupMax + n) * 2) - M);
+            L = fmaf(sc, __ldcg(a.part_ml + (slot * kGroupMax + n) * 2 + 1), L);
+            O = fmaf(sc, __ldcg(a.part_acc + (slot * kGroupMax + n) * D + d), O);
+        }
+        a.out[(static_cast<size_t>(b) * a.Hq + h0 + n) * D + d] = __float2bfloat16(O / L);
+    }
+}
+
+template <int D, int PATH, int NH>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const DecodeArgs a)
+{
+    using G = Geo<D>;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    unsigned char *base = smem_raw + (base_s - raw_s);
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + G::kOffBar);
+    uint64_t *empty = full + G::kStages;
+    volatile int *misc = reinterpret_cast<volatile int *>(base + G::kOffMisc);
+    float *acc_scratch = reinterpret_cast<float *>(base + G::kOffAcc);
+    float *ml_scratch = reinterpret_cast<float *>(base + G::kOffMl);
+    float *qp_scratch = reinterpret_cast<float *>(base + G::kOffQ);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    if (tid == 0) {
+        for (int s = 0; s < G::kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_fence_init();
+        misc[kMiscAbort] = 0;
+        misc[kMiscLocB] = -1;
+        misc[kMiscLocR] = 0;
+        misc[kMiscZero] = 0;
+    }
+    if (warp == kProducerWarp && lane == 0) {
+        tma_prefetch_descriptor(&tmK);
+        tma_prefetch_descriptor(&tmV);
+    }
+    __syncthreads();
+
+    // ---- split plan (reads only tables and lengths: no wait needed yet) ----
+    int my_blocks = 0;
+    for (int b = tid; b < a.B; b += kThreads)
+        my_blocks += ctx_blocks(seq_ctx(a, b));
+    int sum_blocks;
+    block_scan_incl(my_blocks, misc + kMiscWarpSums, &sum_blocks);
+    const int total = sum_blocks * a.items_per_seq;
+    int chunk = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+    if (chunk < a.min_chunk)
+        chunk = a.min_chunk;
+    const int start = static_cast<int>(blockIdx.x) * chunk;
+    const int count = min(chunk, total - start);
+
+    if (count > 0) {
+        int running = 0;
+        for (int base_b = 0; base_b < a.B; base_b += kThreads) {
+            const int b = base_b + tid;
+            const int n = (b < a.B) ? ctx_blocks(seq_ctx(a, b)) : 0;
+            int tot;
+            const int incl = block_scan_incl(n, misc + kMiscWarpSums, &tot);
+            const int lo = (running + incl - n) * a.items_per_seq;
+            const int hi = (running + incl) * a.items_per_seq;
+            if (n > 0 && start >= lo && start < hi) {
+                misc[kMiscLocB] = b;
+                misc[kMiscLocR] = start - lo;
+            }
+            running += tot;
+            __syncthreads();
+            if (misc[kMiscLocB] >= 0)
+                break;
+        }
+    }
+
+    // Everything below may touch what the previous kernel in the stream writes.
+    grid_dependency_wait();
+    grid_launch_dependents();
+
+    if (blockIdx.x == 0) {
+        // outputs of empty sequences, and the length check
+        for (int b = tid; b < a.B; b += kThreads) {
+            const int c = __ldg(a.context_lens + b);
+            if (c < 0 || c > a.W * kBlockTokens)
+                atomicOr(a.status, KV_STATUS_BAD_CONTEXT);
+            if (clamp_ctx(c, a.W) == 0) {
+                __nv_bfloat16 *o = a.out + static_cast<size_t>(b) * a.Hq * D;
+                for (int i = 0; i < a.Hq * D; ++i)
+                    o[i] = __float2bfloat16(0.f);
+            }
+        }
+    }
+    if (count <= 0)
+        return;
+
+    Cursor cur0;
+    cur0.b = misc[kMiscLocB];
+    cur0.ctx = seq_ctx(a, cur0.b);
+    cur0.n = ctx_blocks(cur0.ctx);
+    {
+        const int r = misc[kMiscLocR];
+        cur0.k = r / cur0.n;
+        cur0.off = r - cur0.k * cur0.n;
+    }
+    volatile int *abort_flag = misc + kMiscAbort;
+    const uint32_t ring = base_s;
+
+    if (warp == kProducerWarp) {
+        // ---------------- producer: block ids -> TMA loads ----------------
+        const uint64_t policy = l2_policy_evict_first();
+        Cursor cur = cur0;
+        int u = 0, issued = 0;
+        bool stop = false;
+        while (u < count && !stop) {
+            const int run = min(cur.n - cur.off, count - u);
+            const int j = cur.k / a.hchunks;
+            const int32_t *row = a.block_tables + static_cast<size_t>(cur.b) * a.W + cur.off;
+            for (int bi = 0; bi < run && !stop; bi += 32) {
+                const int m = min(32, run - bi);
+                int blk = 0;
+                if (lane < m) {
+                    blk = __ldg(row + bi + lane);
+                    if (blk < 0 || blk >= a.num_blocks) {
+                        atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
+                        blk = 0;
+                    }
+                }
+                for (int i = 0; i < m; ++i) {
+                    const int phys = __shfl_sync(kFull, blk, i);
+                    const int uu = u + bi + i;
+                    const int s = uu % G::kStages;
+                    int ok = 1;
+                    if (lane == 0) {
+                        ok = mbar_wait_bounded(&empty[s], ((uu / G::kStages) & 1) ^ 1, abort_flag);
+                        if (ok) {
+                            mbar_arrive_expect_tx(&full[s], G::kStageBytes);
+                            const uint32_t dst = ring + s * G::kStageBytes;
+#pragma unroll
+                            for (int t = 0; t < G::kTiles; ++t)
+                                tma_load_4d(dst + t * kTileBytes, &tmK, t * 64, j, 0, phys, &full[s], policy);
+#pragma unroll
+                            for (int t = 0; t < G::kTiles; ++t)
+                                tma_load_4d(dst + (G::kTiles + t) * kTileBytes, &tmV, t * 64, j, 0, phys, &full[s],
+                                            policy);
+                        } else {
+                            *abort_flag = 1;
+                            atomicOr(a.status, KV_STATUS_WAIT_TIMEOUT);
+                        }
+                    }
+                    ok = __shfl_sync(kFull, ok, 0);
+                    if (!ok) {
+                        stop = true;
+                        break;
+                    }
+                    issued = uu + 1;
+                }
+            }
+            u += run;
+            if (u < count)
+                cursor_next_item(a, cur);
+        }
+        // No load may land after this CTA exits: wait (bounded) for the last ones.
+        if (lane == 0) {
+            for (int v = max(0, issued - G::kStages); v < issued; ++v)
+                mbar_wait_bounded(&full[v % G::kStages], (v / G::kStages) & 1, misc + kMiscZero);
+        }
+        return;
+    }
+
+    // -------------------- consumers: warps 0..3 --------------------
+    Consumer<D, PATH, NH> st;
+    Cursor cur = cur0;
+    int u = 0;
+    float *acc_w = acc_scratch + warp * kGroupMax * G::kAccStride;
+    float *ml_w = ml_scratch + warp * kGroupMax * 2;
+    while (u < count) {
+        const int run = min(cur.n - cur.off, count - u);
+        const int item = cur.b * a.items_per_seq + cur.k;
+        const int j = cur.k / a.hchunks, hc = cur.k - (cur.k / a.hchunks) * a.hchunks;
+        const int h0 = j * a.group + hc * kGroupMax;
+        const int gc = min(kGroupMax, a.group - hc * kGroupMax);
+        const int item_start = start + u - cur.off;
+        const int first_cta = item_start / chunk;
+        const int last_cta = (item_start + cur.n - 1) / chunk;
+        const bool single = first_cta == last_cta;
+
+        if (PATH == kPathSimt) {
+            // this item's query rows as fp32 in shared memory (heads >= gc are zero)
+            for (int idx = tid; idx < kGroupMax * D; idx += kConsumerThreads) {
+                const int n = idx / D, d = idx - n * D;
+                const float v = (n < gc) ? __bfloat162float(a.q[(static_cast<size_t>(cur.b) * a.Hq + h0 + n) * D + d])
+                                         : 0.f;
+                qp_scratch[n * G::kQStride + d + ((d >= D / 2) ? 4 : 0)] = v;
+            }
+            named_barrier(1, kConsumerThreads);
+        }
+        st.begin_item(a, cur.b, h0, gc, qp_scratch);
+        for (int i = ((warp - u) % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < run; i += kConsumerWarps) {
+            const int uu = u + i;
+            const int s = uu % G::kStages;
+            if (!mbar_wait_bounded(&full[s], (uu / G::kStages) & 1, abort_flag)) {
+                if (lane == 0) {
+                    *abort_flag = 1;
+                    atomicOr(a.status, KV_STATUS_WAIT_TIMEOUT);
+                }
+                break;
+            }
+            const uint32_t kb = ring + s * G::kStageBytes;
+            const int valid = min(kBlockTokens, cur.ctx - (cur.off + i) * kBlockTokens);
+            st.unit(kb, kb + G::kTiles * kTileBytes, valid, a.scale_log2, qp_scratch);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&empty[s]);
+        }
+
+        // ---- merge the four warps ----
+        st.finish(acc_w, ml_w);
+        named_barrier(1, kConsumerThreads);
+        const size_t slot = static_cast<size_t>(blockIdx.x) + item;
+        for (int idx = tid; idx < gc * D; idx += kConsumerThreads) {
+            const int n = idx / D, d = idx - n * D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w)
+                M = fmaxf(M, ml_scratch[(w * kGroupMax + n) * 2]);
+            float L = 0.f, O = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float sc = exp2f(ml_scratch[(w * kGroupMax + n) * 2] - M);
+                L = fmaf(sc, ml_scratch[(w * kGroupMax + n) * 2 + 1], L);
+                O = fmaf(sc, acc_scratch[(w * kGroupMax + n) * G::kAccStride + d], O);
+            }
+            if (single) {
+                a.out[(static_cast<size_t>(cur.b) * a.Hq + h0 + n) * D + d] = __float2bfloat16(O / L);
+            } else {
+                a.part_acc[(slot * kGroupMax + n) * D + d] = O;
+                if (d == 0) {
+                    a.part_ml[(slot * kGroupMax + n) * 2] = M;
+                    a.part_ml[(slot * kGroupMax + n) * 2 + 1] = L;
+                }
+            }
+        }
+        if (!single && a.fused) {
+            __threadfence();
+            named_barrier(1, kConsumerThreads);
+            if (tid == 0) {
+                const int prev = atomicAdd(a.counters + item, 1);
+                misc[kMiscLast] = (prev == last_cta - first_cta) ? 1 : 0;
+            }
+            named_barrier(1, kConsumerThreads);
+            if (misc[kMiscLast]) {
+                __threadfence();
+                merge_pieces_global<D>(a, item, first_cta, last_cta, cur.b, h0, gc, tid, kConsumerThreads);
+                if (tid == 0)
+                    a.counters[item] = 0;
+            }
+        }
+        named_barrier(1, kConsumerThreads);
+        u += run;
+        if (u < count)
+            cursor_next_item(a, cur);
+    }
+}
+
+// Separate split-K combine: one CTA per work item.
+template <int D>
+__global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int grid_ctas)
+{
+    __shared__ int red[2][4];
+    grid_dependency_wait();
+    grid_launch_dependents();
+    const int item = blockIdx.x;
+    const int b = item / a.items_per_seq, k = item - b * a.items_per_seq;
+    int pre = 0, tot = 0;
+    for (int bb = threadIdx.x; bb < a.B; bb += 128) {
+        const int n = ctx_blocks(seq_ctx(a, bb));
+        tot += n;
+        pre += (bb < b) ? n : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tot += __shfl_xor_sync(kFull, tot, o);
+        pre += __shfl_xor_sync(kFull, pre, o);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        red[0][threadIdx.x >> 5] = tot;
+        red[1][threadIdx.x >> 5] = pre;
+    }
+    __syncthreads();
+    tot = red[0][0] + red[0][1] + red[0][2] + red[0][3];
+    pre = red[1][0] + red[1][1] + red[1][2] + red[1][3];
+    const int n = ctx_blocks(seq_ctx(a, b));
+    if (n == 0)
+        return;
+    const int total = tot * a.items_per_seq;
+    int chunk = (total + grid_ctas - 1) / grid_ctas;
+    if (chunk < a.min_chunk)
+        chunk = a.min_chunk;
+    const int item_start = pre * a.items_per_seq + k * n;
+    const int first_cta = item_start / chunk, last_cta = (item_start + n - 1) / chunk;
+    if (first_cta == last_cta)
+        return;
+    const int j = k / a.hchunks, hc = k - j * a.hchunks;
+    const int h0 = j * a.group + hc * kGroupMax;
+    const int gc = min(kGroupMax, a.group - hc * kGroupMax);
+    merge_pieces_global<D>(a, item, first_cta, last_cta, b, h0, gc, threadIdx.x, 128);
+}
+
+}  // namespace pkv
+
+// ===========================================================================
+// Host side
+// ===========================================================================
+namespace {
+
+using namespace pkv;
+
+std::atomic<int> g_opt_compute{0};
+std::atomic<int> g_opt_combine{0};
+std::atomic<int> g_opt_grid{0};
+std::atomic<int> g_opt_min_chunk{0};
+constexpr int kDefaultMinChunk = 8;
+
+constexpr int kMaxDevices = 64;
+
+int device_sm_count(int dev)
+{
+    static std::atomic<int> cache[kMaxDevices];
+    if (dev < 0 || dev >= kMaxDevices)
+        return 0;
+    int v = cache[dev].load();
+    if (v == 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return 0;
+        cache[dev].store(v);
+    }
+    return v;
+}
+
+struct Layout {
+    int items = 0, slots = 0, max_grid = 0;
+    size_t off_counters = 0, off_ml = 0, off_acc = 0, bytes = 0;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool make_layout(int B, int Hq, int Hkv, int D, int sms, Layout *L)
+{
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (D != 64 && D != 128) || sms < 1)
+        return false;
+    const int group = Hq / Hkv;
+    const long long hchunks = (group + kGroupMax - 1) / kGroupMax;
+    const long long items = static_cast<long long>(B) * Hkv * hchunks;
+    if (items > (1ll << 30))
+        return false;
+    L->items = static_cast<int>(items);
+    L->max_grid = kCtasPerSm * sms;
+    L->slots = L->max_grid + L->items;
+    L->off_counters = kStatusBytes;
+    L->off_ml = L->off_counters + round256(static_cast<size_t>(L->items) * 4);
+    L->off_acc = L->off_ml + round256(static_cast<size_t>(L->slots) * kGroupMax * 2 * 4);
+    L->bytes = L->off_acc + round256(static_cast<size_t>(L->slots) * kGroupMax * D * 4);
+    return true;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// View one cache tensor [num_blocks][16][Hkv][D] as a 4-D map (D, Hkv, 16, num_blocks)
+// with a box of 64 columns x 1 head x 16 rows x 1 block, 128-byte swizzle.
+bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv, int D)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return false;
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv), 16,
+                                static_cast<cuuint64_t>(num_blocks)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hkv) * D * 2,
+                                   static_cast<cuuint64_t>(16) * Hkv * D * 2};
+    const cuuint32_t box[4] = {64, 1, 16, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(cache), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+using DecodeFn = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
+
+template <int D, int PATH, int NH>
+struct KernelInfo {
+    static DecodeFn fn() { return decode_kernel<D, PATH, NH>; }
+    static int smem() { return Geo<D>::kSmemBytes; }
+};
+
+DecodeFn pick_kernel(int D, int path, int nh, int *smem)
+{
+#define PKV_CASE(DD, PP, NN)                          \
+    if (D == DD && path == PP && nh == NN) {          \
+        *smem = KernelInfo<DD, PP, NN>::smem();       \
+        return KernelInfo<DD, PP, NN>::fn();          \
+    }
+    PKV_CASE(64, kPathMma, 8)
+    PKV_CASE(128, kPathMma, 8)
+    PKV_CASE(64, kPathSimt, 1)
+    PKV_CASE(64, kPathSimt, 2)
+    PKV_CASE(64, kPathSimt, 4)
+    PKV_CASE(64, kPathSimt, 8)
+    PKV_CASE(128, kPathSimt, 1)
+    PKV_CASE(128, kPathSimt, 2)
+    PKV_CASE(128, kPathSimt, 4)
+    PKV_CASE(128, kPathSimt, 8)
+#undef PKV_CASE
+    return nullptr;
+}
+
+// Per (kernel, device): dynamic shared memory opted in, and resident CTAs per SM.
+int prepare_kernel(DecodeFn fn, int smem, int dev)
+{
+    struct Entry {
+        const void *fn;
+        int dev;
+        int occ;
+    };
+    static std::mutex mu;
+    static Entry table[64];
+    static int used = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (table[i].fn == reinterpret_cast<const void *>(fn) && table[i].dev == dev)
+            return table[i].occ;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 0;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, kThreads, smem) != cudaSuccess)
+        return 0;
+    if (used < 64)
+        table[used++] = Entry{reinterpret_cast<const void *>(fn), dev, occ};
+    return occ;
+}
+
+bool misaligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
+
+}  // namespace
+
+extern "C" size_t paged_attention_workspace_size(int B, int Hq, int Hkv, int D)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    Layout L;
+    if (!make_layout(B, Hq, Hkv, D, device_sm_count(dev), &L))
+        return 0;
+    return L.bytes;
+}
+
+extern "C" kv_status paged_attention_workspace_init(void *workspace, size_t workspace_bytes, kv_stream_t stream)
+{
+    if (!workspace || workspace_bytes == 0)
+        return KV_ERR_ARG;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KV_OK
+               : KV_ERR_CUDA;
+}
+
+extern "C" kv_status paged_attention_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                            const int32_t *block_tables, int max_blocks_per_seq,
+                                            const int32_t *context_lens, int B, int num_blocks, int Hq, int Hkv,
+                                            int D, float scale, int dtype, void *workspace,
+                                            size_t workspace_bytes, kv_stream_t stream)
+{
+    if (dtype != KV_DTYPE_BF16 || B < 0 || max_blocks_per_seq < 1 || num_blocks < 1 || Hq < 1 || Hkv < 1 ||
+        Hq % Hkv != 0 || (D != 64 && D != 128))
+        return KV_ERR_ARG;
+    if (B == 0)
+        return KV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !workspace)
+        return KV_ERR_ARG;
+    if (misaligned(out, 16) || misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) ||
+        misaligned(block_tables, 4) || misaligned(context_lens, 4) || misaligned(workspace, 256))
+        return KV_ERR_ARG;
+    if (static_cast<long long>(B) * max_blocks_per_seq * Hkv * ((Hq / Hkv + kGroupMax - 1) / kGroupMax) >=
+        (1ll << 31))
+        return KV_ERR_ARG;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return KV_ERR_CUDA;
+    const int sms = device_sm_count(dev);
+    Layout L;
+    if (!make_layout(B, Hq, Hkv, D, sms, &L))
+        return KV_ERR_ARG;
+    if (workspace_bytes < L.bytes)
+        return KV_ERR_ARG;
+
+    const int group = Hq / Hkv;
+    int path = g_opt_compute.load();
+    if (path == 0)
+        path = kPathMma;
+    int nh = kGroupMax;
+    if (path == kPathSimt) {
+        const int gmin = group < kGroupMax ? group : kGroupMax;
+        nh = gmin <= 1 ? 1 : gmin <= 2 ? 2 : gmin <= 4 ? 4 : 8;
+    }
+    int smem = 0;
+    DecodeFn fn = pick_kernel(D, path, nh, &smem);
+    if (!fn)
+        return KV_ERR_ARG;
+    const int occ = prepare_kernel(fn, smem, dev);
+    if (occ < 1)
+        return KV_ERR_CUDA;
+    int grid = (occ < kCtasPerSm ? occ : kCtasPerSm) * sms;
+    const int want = g_opt_grid.load();
+    if (want > 0)
+        grid = want < L.max_grid ? want : L.max_grid;
+
+    CUtensorMap tmK, tmV;
+    if (!make_cache_map(&tmK, k_cache, num_blocks, Hkv, D) || !make_cache_map(&tmV, v_cache, num_blocks, Hkv, D))
+        return KV_ERR_CUDA;
+
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    DecodeArgs a;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.part_acc = reinterpret_cast<float *>(ws + L.off_acc);
+    a.part_ml = reinterpret_cast<float *>(ws + L.off_ml);
+    a.counters = reinterpret_cast<int32_t *>(ws + L.off_counters);
+    a.status = reinterpret_cast<int32_t *>(ws);
+    a.B = B;
+    a.W = max_blocks_per_seq;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = group;
+    a.hchunks = (group + kGroupMax - 1) / kGroupMax;
+    a.items_per_seq = Hkv * a.hchunks;
+    a.num_blocks = num_blocks;
+    const int mc = g_opt_min_chunk.load();
+    a.min_chunk = mc > 0 ? mc : kDefaultMinChunk;
+    const int combine_mode = g_opt_combine.load();
+    a.fused = combine_mode == 0 ? 1 : 0;
+    a.scale_log2 = scale * 1.4426950408889634f;
+
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, fn, tmK, tmV, a) != cudaSuccess)
+        return KV_ERR_CUDA;
+
+    if (!a.fused) {
+        cudaLaunchConfig_t c2 = {};
+        c2.gridDim = dim3(L.items);
+        c2.blockDim = dim3(128);
+        c2.dynamicSmemBytes = 0;
+        c2.stream = st;
+        c2.attrs = attr;
+        c2.numAttrs = 1;
+        cudaError_t e = (D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<64>, a, grid)
+                                  : cudaLaunchKernelEx(&c2, combine_kernel<128>, a, grid);
+        if (e != cudaSuccess)
+            return KV_ERR_CUDA;
+    }
+    return KV_OK;
+}
+
+extern "C" kv_status paged_attention_read_status(const void *workspace, int32_t *status_out, int clear,
+                                                 kv_stream_t stream)
+{
+    if (!workspace || !status_out)
+        return KV_ERR_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess)
+        return KV_ERR_CUDA;
+    if (cudaMemcpy(status_out, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return KV_ERR_CUDA;
+    if (clear && cudaMemset(const_cast<void *>(workspace), 0, sizeof(int32_t)) != cudaSuccess)
+        return KV_ERR_CUDA;
+    return KV_OK;
+}
+
+extern "C" kv_status kv_decode_set_option(int key, int value)
+{
+    switch (key) {
+    case KV_OPT_COMPUTE:
+        if (value < 0 || value > 2)
+            return KV_ERR_ARG;
+        g_opt_compute.store(value);
+        return KV_OK;
+    case KV_OPT_COMBINE:
+        if (value < 0 || value > 1)
+            return KV_ERR_ARG;
+        g_opt_combine.store(value);
+        return KV_OK;
+    case KV_OPT_GRID:
+        if (value < 0)
+            return KV_ERR_ARG;
+        g_opt_grid.store(value);
+        return KV_OK;
+    case KV_OPT_MIN_CHUNK:
+        if (value < 0)
+            return KV_ERR_ARG;
+        g_opt_min_chunk.store(value);
+        return KV_OK;
+    default:
+        return KV_ERR_ARG;
+    }
+}
+
+extern "C" int kv_decode_get_option(int key)
+{
+    switch (key) {
+    case KV_OPT_COMPUTE:
+        return g_opt_compute.load();
+    case KV_OPT_COMBINE:
+        return g_opt_combine.load();
+    case KV_OPT_GRID:
+        return g_opt_grid.load();
+    case KV_OPT_MIN_CHUNK:
+        return g_opt_min_chunk.load();
+    default:
+        return -1;
+    }
+}

@@ -1,0 +1,71 @@
+"""Shared helpers for the GPU parity tests: seeded cases, and the oracle comparison.
+
+Inputs come from paged_kv_cache_470_b200.workloads (seeded, shared with the
+oracle side); expected values come only from the oracle, fed with the same
+pre-step inputs copied to the host.
+"""
+import numpy as np
+import torch
+
+from paged_kv_cache_470_b200 import workloads
+
+ATOL, RTOL = 5e-3, 1e-2   # |gpu - ref| <= ATOL + RTOL * |ref|, elementwise
+
+
+class Case:
+    """One decode step over `n_layers` layers of a workload, resident on the GPU."""
+
+    def __init__(self, cfg, device, n_layers=1, lens=None, seed=None, layout=None):
+        self.cfg = cfg
+        self.layout = layout or workloads.draw_layout(cfg, context_lens=lens, seed=seed)
+        gen = workloads.device_generator(cfg.seed if seed is None else seed, device)
+        self.k, self.v = [], []
+        for _ in range(n_layers):
+            k, v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device)
+            self.k.append(k)
+            self.v.append(v)
+        self.q, self.k_new, self.v_new = workloads.make_step_inputs(cfg, gen, device, n_layers)
+        self.tables = self.layout.block_tables.to(device)
+        self.lens = self.layout.context_lens.to(device)
+        self.slots = self.layout.slot_mapping().to(device)
+        self.n_layers = n_layers
+        self.device = device
+
+    def host_inputs(self, layer):
+        """Pre-step inputs of one layer, on the host, for the oracle."""
+        return (self.q[layer].cpu(), self.k[layer].cpu(), self.v[layer].cpu(), self.k_new[layer].cpu(),
+                self.v_new[layer].cpu())
+
+
+def oracle_step(oracle_mod, case, layer, host=None):
+    """Oracle append then oracle attention for one layer; returns (k_after, v_after, out64)."""
+    q, k, v, kn, vn = host if host is not None else case.host_inputs(layer)
+    k2, v2 = oracle_mod.kv_cache_append(k, v, kn, vn, case.layout.slot_mapping().numpy())
+    out = oracle_mod.paged_attention_decode(q, k2, v2, case.layout.block_tables.numpy(),
+                                            case.layout.context_lens.numpy(), case.cfg.scale)
+    return k2, v2, out
+
+
+def gpu_step(pkv, case, layer, workspace, out=None):
+    if out is None:
+        out = torch.empty_like(case.q[layer])
+    pkv.kv_cache_append(case.k_new[layer], case.v_new[layer], case.k[layer], case.v[layer], case.slots)
+    pkv.paged_attention_decode(out, case.q[layer], case.k[layer], case.v[layer], case.tables, case.lens,
+                               case.cfg.scale, workspace)
+    return out
+
+
+def bf16_bits_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def compare(gpu_out: torch.Tensor, ref: np.ndarray, what: str):
+    g = gpu_out.detach().float().cpu().double().numpy()
+    assert np.isfinite(g).all(), f"{what}: non-finite output"
+    err = np.abs(g - ref)
+    bad = err > ATOL + RTOL * np.abs(ref)
+    big = np.abs(ref) >= 1e-2
+    rel = (err[big] / np.abs(ref[big])).max() if big.any() else 0.0
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {bad.size} elements out of tolerance; "
+                           f"max abs err {err.max():.3e}, max rel err (|ref|>=1e-2) {rel:.3e}")
+    return float(err.max()), float(rel)

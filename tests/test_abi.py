@@ -1,0 +1,54 @@
+"""The C ABI library builds, loads without a GPU, and exports every declared symbol."""
+import ctypes
+import os
+import re
+import subprocess
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedkv.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kv_\w+|paged_attention_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("kv_cache_append", "paged_attention_decode", "paged_attention_workspace_size",
+                     "kv_pool_create", "kv_pool_alloc", "kv_pool_free", "kv_pool_incref"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(pkv):
+    lib = ctypes.CDLL(pkv.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in pagedkv.h but not exported"
+
+
+def test_binding_covers_every_declared_symbol(pkv):
+    assert set(declared_functions()) == set(pkv.EXPORTED)
+
+
+def test_only_abi_symbols_are_exported(pkv):
+    out = subprocess.run(["nm", "-D", "--defined-only", pkv.LIB_PATH], capture_output=True, text=True).stdout
+    ours = {l.split()[-1] for l in out.splitlines() if re.search(r"\b(kv_|paged_attention_)", l)}
+    assert ours == set(declared_functions())
+
+
+def test_library_is_built_for_sm100a(pkv):
+    # the build flags are the contract; check them without reading the binary
+    import runpy
+    flags = runpy.run_path(os.path.join(ROOT, "paged_kv_cache_470_b200", "build.py"))["NVCC_FLAGS"]
+    assert "arch=compute_100a,code=sm_100a" in " ".join(flags)
+
+
+def test_host_argument_checks_need_no_gpu(pkv):
+    lib = ctypes.CDLL(pkv.LIB_PATH)
+    lib.kv_cache_append.restype = ctypes.c_int
+    # D = 96 is not supported: rejected on the host before any CUDA call
+    rc = lib.kv_cache_append(None, None, None, None, None, 1, 1, 1, 96, 0, None, None)
+    assert rc == pkv.KV_ERR_ARG
+    assert pkv.set_option(pkv.KV_OPT_COMPUTE, 0) is None
+    assert lib.kv_decode_set_option(99, 0) == pkv.KV_ERR_ARG

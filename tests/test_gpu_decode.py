@@ -1,0 +1,193 @@
+"""GPU parity: append (bit-exact) and decode attention (within 5e-3 + 1e-2|ref|) against the oracle.
+
+Every call goes through the C ABI of libpagedkv.so via the ctypes binding.
+"""
+import random
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_470_b200 import workloads
+from gpu_cases import Case, bf16_bits_np, compare, gpu_step, oracle_step
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"tensor_cores": 1, "cuda_cores": 2}
+
+
+@pytest.fixture(autouse=True)
+def _default_options(pkv):
+    yield
+    for key in (pkv.KV_OPT_COMPUTE, pkv.KV_OPT_COMBINE, pkv.KV_OPT_GRID, pkv.KV_OPT_MIN_CHUNK):
+        pkv.set_option(key, 0)
+
+
+def run_and_check(pkv, oracle_mod, case, layers=None, what=""):
+    cfg = case.cfg
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    for layer in (range(case.n_layers) if layers is None else layers):
+        host = case.host_inputs(layer)
+        out = gpu_step(pkv, case, layer, ws)
+        torch.cuda.synchronize()
+        k2, v2, ref = oracle_step(oracle_mod, case, layer, host)
+        assert np.array_equal(bf16_bits_np(case.k[layer]), k2), f"{what} layer {layer}: K append not bit-exact"
+        assert np.array_equal(bf16_bits_np(case.v[layer]), v2), f"{what} layer {layer}: V append not bit-exact"
+        compare(out, ref, f"{what} layer {layer}")
+    assert pkv.read_status(ws) == 0
+
+
+# ---------------------------------------------------------------------------
+# the tiny workload, every path and combine mode
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("path", sorted(PATHS))
+@pytest.mark.parametrize("combine", [0, 1])
+def test_tiny_workload(pkv, oracle_mod, cuda_device, path, combine):
+    pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
+    pkv.set_option(pkv.KV_OPT_COMBINE, combine)
+    case = Case(workloads.CONFIGS[1], cuda_device)
+    run_and_check(pkv, oracle_mod, case, what=f"tiny/{path}/combine{combine}")
+
+
+@pytest.mark.parametrize("path", sorted(PATHS))
+@pytest.mark.parametrize("D,Hq,Hkv", [(64, 20, 4), (128, 32, 8), (128, 8, 8), (64, 16, 2), (128, 64, 8),
+                                      (128, 32, 2), (64, 12, 1)])
+def test_ragged_lengths_and_head_groups(pkv, oracle_mod, cuda_device, path, D, Hq, Hkv):
+    """Lengths at and around block edges, the table's maximum, 1 and 0; groups 1..16."""
+    pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
+    lens = [1, 15, 16, 17, 31, 32, 33, 255, 256, 0, 100, 2]
+    cfg = workloads.small_config(1, Hq=Hq, Hkv=Hkv, D=D, batch=len(lens), pool_blocks=0)
+    case = Case(cfg, cuda_device, lens=lens)
+    run_and_check(pkv, oracle_mod, case, what=f"ragged D{D} {Hq}/{Hkv} {path}")
+
+
+@pytest.mark.parametrize("cid", [2, 3])
+@pytest.mark.parametrize("grid,min_chunk", [(1, 1), (3, 1), (7, 2), (296, 1), (0, 1)])
+def test_many_split_pieces(pkv, oracle_mod, cuda_device, cid, grid, min_chunk):
+    """Items cut into many split-K pieces; few CTAs, each wrapping its stage ring many times."""
+    pkv.set_option(pkv.KV_OPT_GRID, grid)
+    pkv.set_option(pkv.KV_OPT_MIN_CHUNK, min_chunk)
+    cfg = workloads.small_config(cid, batch=6, ctx_lo=1, ctx_hi=1500, W=96, n_layers=1)
+    case = Case(cfg, cuda_device)
+    run_and_check(pkv, oracle_mod, case, what=f"config {cid} shape, grid {grid} min_chunk {min_chunk}")
+
+
+# ---------------------------------------------------------------------------
+# exact special cases and invariances
+# ---------------------------------------------------------------------------
+def test_single_token_context_returns_v_exactly(pkv, oracle_mod, cuda_device):
+    cfg = workloads.small_config(1, batch=8)
+    case = Case(cfg, cuda_device, lens=[1] * 8)
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    out = gpu_step(pkv, case, 0, ws)
+    g = cfg.Hq // cfg.Hkv
+    expect = case.v_new[0].repeat_interleave(g, dim=1)   # the only token is the appended one
+    assert torch.equal(out, expect)
+
+
+def test_empty_context_gives_zeros(pkv, cuda_device):
+    cfg = workloads.small_config(1, batch=3)
+    case = Case(cfg, cuda_device, lens=[0, 5, 0])
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    out = torch.full_like(case.q[0], 7.0)
+    gpu_step(pkv, case, 0, ws, out)
+    torch.cuda.synchronize()
+    assert (out[0] == 0).all() and (out[2] == 0).all() and torch.isfinite(out[1].float()).all()
+
+
+def test_physical_permutation_is_bit_identical(pkv, cuda_device):
+    cfg = workloads.small_config(2, batch=16, n_layers=1)
+    case = Case(cfg, cuda_device)
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    out1 = gpu_step(pkv, case, 0, ws).clone()
+    nb = case.layout.num_blocks
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(3)).to(cuda_device)
+    k2, v2 = torch.empty_like(case.k[0]), torch.empty_like(case.v[0])
+    k2[perm], v2[perm] = case.k[0], case.v[0]
+    tables2 = torch.where(case.tables >= 0, perm[case.tables.clamp(min=0).long()].int(), case.tables)
+    out2 = torch.empty_like(out1)
+    pkv.paged_attention_decode(out2, case.q[0], k2, v2, tables2, case.lens, cfg.scale, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+
+
+def test_repeat_is_bit_identical(pkv, cuda_device):
+    cfg = workloads.small_config(3, batch=8, n_layers=1)
+    case = Case(cfg, cuda_device)
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    out1 = gpu_step(pkv, case, 0, ws).clone()
+    out2 = torch.empty_like(out1)
+    for _ in range(3):
+        pkv.paged_attention_decode(out2, case.q[0], case.k[0], case.v[0], case.tables, case.lens, cfg.scale, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(out1, out2)
+
+
+def test_bad_block_id_and_length_are_flagged_not_faulted(pkv, cuda_device):
+    cfg = workloads.small_config(1, batch=4)
+    case = Case(cfg, cuda_device, lens=[40, 40, 40, 40])
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    out = torch.empty_like(case.q[0])
+    tables = case.tables.clone()
+    tables[1, 1] = case.layout.num_blocks + 1000
+    pkv.paged_attention_decode(out, case.q[0], case.k[0], case.v[0], tables, case.lens, cfg.scale, ws)
+    assert pkv.read_status(ws) & pkv.KV_STATUS_BAD_BLOCK_ID
+    lens = case.lens.clone()
+    lens[2] = cfg.W * 16 + 5
+    pkv.paged_attention_decode(out, case.q[0], case.k[0], case.v[0], case.tables, lens, cfg.scale, ws)
+    assert pkv.read_status(ws) & pkv.KV_STATUS_BAD_CONTEXT
+    # a clean call afterwards is clean
+    pkv.paged_attention_decode(out, case.q[0], case.k[0], case.v[0], case.tables, case.lens, cfg.scale, ws)
+    assert pkv.read_status(ws) == 0
+
+
+def test_append_bit_exact_with_padding_and_bad_slots(pkv, oracle_mod, cuda_device):
+    g = torch.Generator(device=cuda_device).manual_seed(5)
+    nb, Hkv, D, T = 37, 8, 128, 50
+    kc = torch.randn(nb, 16, Hkv, D, generator=g, device=cuda_device).to(torch.bfloat16)
+    vc = torch.randn(nb, 16, Hkv, D, generator=g, device=cuda_device).to(torch.bfloat16)
+    kn = torch.randn(T, Hkv, D, generator=g, device=cuda_device).to(torch.bfloat16)
+    vn = torch.randn(T, Hkv, D, generator=g, device=cuda_device).to(torch.bfloat16)
+    slots = torch.randperm(nb * 16, generator=torch.Generator().manual_seed(1))[:T].to(torch.int64)
+    slots[::7] = -1
+    k_host, v_host = kc.cpu(), vc.cpu()
+    ek, ev = oracle_mod.kv_cache_append(k_host, v_host, kn.cpu(), vn.cpu(), slots.numpy())
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    pkv.kv_cache_append(kn, vn, kc, vc, slots.to(cuda_device), flag)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits_np(kc), ek) and np.array_equal(bf16_bits_np(vc), ev)
+    assert int(flag) == 0
+    bad = slots.clone()
+    bad[3] = nb * 16          # one past the pool: skipped and flagged
+    before_k, before_v = kc.clone(), vc.clone()
+    pkv.kv_cache_append(kn, vn, kc, vc, bad.to(cuda_device), flag)
+    torch.cuda.synchronize()
+    assert int(flag) & pkv.KV_STATUS_BAD_SLOT
+    # the other rows were rewritten with the same bytes; nothing else changed
+    assert torch.equal(kc, before_k) and torch.equal(vc, before_v)
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the bench times
+# ---------------------------------------------------------------------------
+def _full_size(pkv, oracle_mod, cuda_device, cid, n_alloc):
+    cfg = workloads.CONFIGS[cid]
+    case = Case(cfg, cuda_device, n_layers=n_alloc)
+    layers = sorted({0, n_alloc - 1, random.Random(cid).randrange(n_alloc)})
+    run_and_check(pkv, oracle_mod, case, layers=layers, what=f"config {cid}")
+
+
+def test_full_size_05b_gqa(pkv, oracle_mod, cuda_device):
+    _full_size(pkv, oracle_mod, cuda_device, 2, 24)
+
+
+def test_full_size_llama3_8b_shape(pkv, oracle_mod, cuda_device):
+    _full_size(pkv, oracle_mod, cuda_device, 3, 3)
+
+
+def test_full_size_llama2_7b_mha(pkv, oracle_mod, cuda_device):
+    _full_size(pkv, oracle_mod, cuda_device, 4, 2)
+
+
+def test_full_size_70b_mix_with_shared_prefix(pkv, oracle_mod, cuda_device):
+    _full_size(pkv, oracle_mod, cuda_device, 5, 2)
