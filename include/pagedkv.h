@@ -161,6 +161,33 @@ KV_API kv_status paged_attention_read_status(const void *workspace, int32_t *sta
                                       int clear, kv_stream_t stream);
 
 /*
+ * The same decode as paged_attention_decode, for callers that cannot allocate
+ * device memory (for example a plugin inside a host program that owns every
+ * device allocation, or code that must not trigger cudaMalloc's implicit
+ * device synchronisation). The pages have no counterpart: it changes where
+ * the split-K scratch lives, not what is computed.
+ *
+ * The scratch is one fixed array of KV_NOALLOC_SCRATCH_BYTES (16 MiB) inside
+ * the library, present on every GPU that loads it until the process exits.
+ * The caller still passes inputs and outputs; nothing is allocated or freed.
+ * Sizes whose scratch (paged_attention_workspace_size) exceeds the array are
+ * rejected with KV_ERR_ARG. The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current); make that
+ * first call before any stream capture. Each call clears the array's status
+ * word and counters on `stream` before the kernel. All calls share the one
+ * array: calls that can overlap on the GPU (other streams, other threads)
+ * race and give wrong results; serialise them. Device data errors are
+ * guarded as in paged_attention_decode but cannot be read back here.
+ */
+#define KV_NOALLOC_SCRATCH_BYTES (16u << 20)
+KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
+                                                const void *k_cache, const void *v_cache,
+                                                const int32_t *block_tables, int max_blocks_per_seq,
+                                                const int32_t *context_lens, int B,
+                                                int num_blocks, int Hq, int Hkv, int D,
+                                                float scale, int dtype, kv_stream_t stream);
+
+/*
  * Process-wide tuning switches (defaults are the tuned choices).
  *   KV_OPT_COMPUTE:   0 auto, 1 tensor cores (mma.sync bf16), 2 CUDA cores
  *   KV_OPT_COMBINE:   0 split-K merge fused into the last CTA of each work

@@ -35,6 +35,8 @@ _sig = {
     "paged_attention_workspace_init": (_I, [_P, _SZ, _P]),
     "paged_attention_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _SZ,
                                     _P]),
+    "paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                                            _P]),
     "paged_attention_read_status": (_I, [_P, _P, _I, _P]),
     "kv_decode_set_option": (_I, [_I, _I]),
     "kv_decode_get_option": (_I, [_I]),

@@ -1041,6 +1041,60 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
     return KV_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Decode without caller-provided workspace.
+//
+// For callers that cannot allocate device memory themselves: a plugin running
+// inside a host program that owns every device allocation, or a code path
+// where the implicit device synchronisation of cudaMalloc is not allowed. The
+// split-K scratch lives in one fixed array in this library's device image
+// instead, held by every GPU that loads the library until the process exits.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr size_t kNoAllocScratchBytes = KV_NOALLOC_SCRATCH_BYTES;
+}
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+extern "C" kv_status paged_attention_decode_noalloc(void *out, const void *q, const void *k_cache,
+                                                    const void *v_cache, const int32_t *block_tables,
+                                                    int max_blocks_per_seq, const int32_t *context_lens, int B,
+                                                    int num_blocks, int Hq, int Hkv, int D, float scale, int dtype,
+                                                    kv_stream_t stream)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return KV_ERR_CUDA;
+    // In host code the array's name is not a device address: look the address
+    // up once per device, with that device current.
+    static std::atomic<void *> scratch[kMaxDevices];
+    static std::mutex setup_mu;
+    void *ws = scratch[dev].load();
+    if (!ws) {
+        std::lock_guard<std::mutex> lock(setup_mu);
+        ws = scratch[dev].load();
+        if (!ws) {
+            void *p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+                return KV_ERR_CUDA;
+            scratch[dev].store(p);
+            ws = p;
+        }
+    }
+    Layout L;
+    if (!make_layout(B, Hq, Hkv, D, device_sm_count(dev), &L))
+        return KV_ERR_ARG;
+    if (L.bytes > kNoAllocScratchBytes)
+        return KV_ERR_ARG;  // more split-K scratch than the fixed array holds
+    if (B == 0)
+        return KV_OK;
+    // The array keeps the previous call's contents: the status word and the
+    // per-item counters must start at zero.
+    if (cudaMemsetAsync(ws, 0, L.off_ml, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return KV_ERR_CUDA;
+    return paged_attention_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, B,
+                                  num_blocks, Hq, Hkv, D, scale, dtype, ws, kNoAllocScratchBytes, stream);
+}
+
 extern "C" kv_status paged_attention_read_status(const void *workspace, int32_t *status_out, int clear,
                                                  kv_stream_t stream)
 {
