@@ -331,12 +331,28 @@ class OracleSampler:
         return done_bytes, time.perf_counter() - t0, done_layers * self.cfg.batch
 
 
+def run_profile_step(args, cfg, device):
+    """Only the step's graph replays (for ncu): no e2e, no per-kernel timing, no CPU baseline."""
+    import paged_kv_cache_470_b200 as pkv
+    wl = Workload(cfg, device)
+    graph = capture(wl.step)
+    for _ in range(args.warmup + args.steps):
+        graph.replay()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_step": cfg.name, "layers": cfg.n_layers, "replays": args.warmup + args.steps,
+                      "status": pkv.read_status(wl.ws)}), flush=True)
+
+
 def run_ours(args, world, rank, local):
     import paged_kv_cache_470_b200 as pkv
     cfg = workloads.CONFIGS[args.config]
+    if args.layers:
+        cfg = workloads.small_config(args.config, n_layers=args.layers)
     device = torch.device("cuda", local if world > 1 else 0)
     if args.compute:
         pkv.set_option(pkv.KV_OPT_COMPUTE, {"tensor": 1, "cuda": 2}[args.compute])
+    if args.profile_step:
+        return run_profile_step(args, cfg, device)
     wl = Workload(cfg, device, rank)
     lens = [int(c) for c in wl.layout.context_lens]
     share = wl.layout.shares_prefix.tolist()
@@ -459,6 +475,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--reference-budget", type=float, default=120.0)
+    ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling a smaller case)")
+    ap.add_argument("--profile-step", action="store_true", help="only replay the step graph (for ncu)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -194,13 +194,17 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
  *                     item, 1 separate combine kernel
  *   KV_OPT_GRID:      0 auto (CTAs resident on all SMs), n > 0 launch n CTAs
  *                     (n is capped by what the workspace was sized for)
- *   KV_OPT_MIN_CHUNK: 0 auto, n > 0 minimum KV blocks per CTA
+ *   KV_OPT_MIN_CHUNK: 0 auto, n > 0 minimum work units (KV blocks of one
+ *                     kv-head group) per CTA
+ *   KV_OPT_PRODUCER_LANES: 0 auto, 1/2/4/8 lanes of the producer warp that
+ *                     issue tile loads
  * Returns KV_ERR_ARG for an unknown key or value.
  */
 #define KV_OPT_COMPUTE 1
 #define KV_OPT_COMBINE 2
 #define KV_OPT_GRID 3
 #define KV_OPT_MIN_CHUNK 4
+#define KV_OPT_PRODUCER_LANES 5
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

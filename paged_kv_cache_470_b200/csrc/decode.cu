@@ -7,28 +7,34 @@
 //     out[b][h] = sum_t softmax_t(scale * <q[b][h], K_t>) V_t,   t < c,
 // where token t lives in physical block block_tables[b][t / 16], row t % 16.
 //
-// Work decomposition. A work item is (sequence b, kv head j, chunk of at most
-// 8 query heads of j's group); its work units are the ceil(c/16) KV blocks of
-// the sequence. All units of all items are laid end to end and cut into
-// equal contiguous ranges, one per CTA (the grid is sized to be resident on
-// every SM at once). A CTA therefore handles whole items and at most two
-// partial items; an item cut between CTAs is a split-K item: each piece
-// produces (running max, running sum, unnormalised accumulator) in fp32 and a
-// log-sum-exp merge joins them. The merge runs in the last CTA to finish a
-// piece of that item (an atomic counter, no spinning), or, as an option, in a
-// separate combine kernel.
+// Work decomposition. The kv heads are taken in groups of HG (4 when Hkv is a
+// multiple of 4, else 2 or 1). A work item is (sequence b, kv-head group,
+// chunk of at most 8 query heads per kv head); its work units are the
+// ceil(c/16) KV blocks of the sequence, each unit being the group's HG heads of
+// one block: one TMA box of 16 rows x HG heads x 64 columns (8 KB when HG=4)
+// per 64 columns of K and of V. A box costs about as much to issue as one four
+// times larger, so HG heads travel together.
 //
-// Inside a CTA: warp 4 is the producer. It reads block ids from the table and
-// issues TMA tile loads of the item's 16 K rows and 16 V rows (one 128-byte
-// swizzled box per 64 columns) into a ring of shared-memory stages guarded by
-// mbarriers. Warps 0-3 consume units round robin, each keeping an fp32 online
-// softmax (running max and sum per query head) and its own accumulator; at the
-// end of an item the four warps are merged through shared memory.
+// All units of all items are laid end to end and cut into equal contiguous
+// ranges, one per CTA (one resident CTA per SM). A CTA handles whole items
+// and at most two partial ones; an item cut between CTAs is a split-K item:
+// each piece leaves (running max, running sum, unnormalised accumulator) in
+// fp32 and a log-sum-exp merge joins them, in the last CTA to finish a piece
+// of that item (an atomic counter, no spinning) or in a separate combine
+// kernel.
+//
+// Inside a CTA, warp 8 is the producer: it reads block ids from the table and
+// issues the TMA loads into a ring of shared-memory stages guarded by
+// mbarriers. Warps 0-7 are consumers arranged as 8/HG streams of HG warps:
+// stream s takes units s, s + 8/HG, ...; within a stream, warp hh handles kv
+// head hh of the group. Each warp keeps an fp32 online softmax (running max
+// and sum per query head) and its accumulator in registers; at the end of an
+// item the streams are merged pairwise through shared memory.
 //
 // Two consumer arithmetic paths:
 //  * tensor cores: S^T[16 tokens x 8 heads] = K_blk * Q^T with
 //    mma.sync.m16n8k16 (bf16 in, fp32 accumulate; the 16 tokens of a block are
-//    the M dimension, the group's query heads the N dimension), then
+//    the M dimension, the kv head's query heads the N dimension), then
 //    O^T[D x 8] += V_blk^T * P^T, with the probabilities split into a bf16
 //    high part and a bf16 residual so that P keeps ~16 significant bits.
 //  * CUDA cores: fp32 FMAs on values unpacked from bf16.
@@ -42,38 +48,38 @@
 
 namespace pkv {
 
-constexpr int kThreads = 160;
-constexpr int kConsumerWarps = 4;
+constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
-constexpr int kProducerWarp = 4;
-constexpr int kGroupMax = 8;             // query heads per work item
-constexpr int kTileBytes = 16 * 128;     // one TMA box: 16 rows x 64 bf16, 128B-swizzled
-constexpr int kCtasPerSm = 2;
+constexpr int kProducerWarp = kConsumerWarps;
+constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kGroupMax = 8;            // query heads per kv head per work item
+constexpr int kMaxHG = 4;               // kv heads per work unit
+constexpr int kHeadTileBytes = 2048;    // one kv head: 16 rows x 64 bf16, 128B-swizzled
+constexpr int kMergeSlots = 4;          // warps that hand their state over per merge round
+constexpr int kCtasPerSm = 1;
 constexpr int kStatusBytes = 256;
 constexpr unsigned kFull = 0xffffffffu;
 
 enum ComputePath { kPathMma = 1, kPathSimt = 2 };
 
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
 template <int D>
 struct Geo {
     static_assert(D == 64 || D == 128, "head dim");
-    static constexpr int kTiles = D / 64;
-    static constexpr int kStageBytes = 2 * kTiles * kTileBytes;   // K and V of one block
-    // A multiple of the consumer-warp count, so stage s is always consumed by
-    // warp s % 4, in order: a warp never waits on round r+1 of a stage whose
-    // round r another warp has not consumed yet (the parity wait could not
-    // tell those two rounds apart).
-    static constexpr int kStages = ((80 * 1024) / kStageBytes) / kConsumerWarps * kConsumerWarps;  // 20 or 8
-    static_assert(kStages % kConsumerWarps == 0, "stage ownership must be fixed per warp");
-    static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kAccStride = D + 4;                      // padded: conflict-free scratch writes
-    static constexpr int kQStride = D + 8;                        // second half shifted by 4 floats
-    static constexpr int kOffAcc = kRingBytes;
-    static constexpr int kOffMl = kOffAcc + kConsumerWarps * kGroupMax * kAccStride * 4;
-    static constexpr int kOffQ = kOffMl + kConsumerWarps * kGroupMax * 2 * 4;
-    static constexpr int kOffP = kOffQ + kGroupMax * kQStride * 4;
-    static constexpr int kOffBar = kOffP + kConsumerWarps * 16 * kGroupMax * 4;
-    static constexpr int kOffMisc = kOffBar + 2 * kStages * 8;
+    static constexpr int kTiles = D / 64;                       // 64-column boxes per K (and per V)
+    static constexpr int kRingBytes = 192 * 1024;
+    static constexpr int kMaxStages = kRingBytes / (2 * kTiles * kHeadTileBytes);  // HG = 1
+    static constexpr int kMmaRegs = (D / 16) * 4 + 4;
+    static constexpr int kSimtRegs = kGroupMax * (D / 32) + 2 * kGroupMax;
+    static constexpr int kMergeBytes = kMergeSlots * cmax(kMmaRegs, kSimtRegs) * 32 * 4;
+    static constexpr int kQStride = D + 8;                      // second half shifted by 4 floats
+    static constexpr int kQBytes = kMaxHG * kGroupMax * kQStride * 4;
+    static constexpr int kPBytes = kConsumerWarps * 16 * kGroupMax * 4;
+    static constexpr int kScratchBytes = cmax(kMergeBytes, kQBytes + kPBytes);
+    static constexpr int kOffScratch = kRingBytes;
+    static constexpr int kOffBar = kOffScratch + kScratchBytes;
+    static constexpr int kOffMisc = kOffBar + 2 * kMaxStages * 8;
     static constexpr int kMiscInts = 16;
     static constexpr int kSmemBytes = kOffMisc + kMiscInts * 4 + 1024;  // + room to align the base
 };
@@ -83,18 +89,24 @@ struct DecodeArgs {
     const __nv_bfloat16 *q;
     const int32_t *block_tables;
     const int32_t *context_lens;
-    float *part_acc;     // [slots][8][D]
-    float *part_ml;      // [slots][8][2]  (max in log2 units, sum)
+    float *part_acc;     // [slots][kMaxHG][8][D]
+    float *part_ml;      // [slots][kMaxHG][8][2]  (max in log2 units, sum)
     int32_t *counters;   // [items]
     int32_t *status;
-    int B, W, Hq, Hkv, group, hchunks, items_per_seq, num_blocks;
+    int B, W, Hq, Hkv, group, num_blocks;
+    int hg;              // kv heads per unit (HG)
+    int streams;         // consumer streams = 8 / HG
+    int hchunks;         // query-head chunks per kv head = ceil(group / 8)
+    int items_per_seq;   // (Hkv / HG) * hchunks
+    int stages, stage_bytes, tile_stride;  // ring geometry; tile_stride = HG * 2048
+    int prod_lanes;      // producer lanes issuing TMA
     int min_chunk;
     int fused;
     float scale_log2;    // scale * log2(e)
 };
 
 // misc ints in shared memory
-enum { kMiscAbort = 0, kMiscLocB = 1, kMiscLocR = 2, kMiscLast = 3, kMiscZero = 4, kMiscWarpSums = 8 };
+enum { kMiscAbort = 0, kMiscLocB = 1, kMiscLocR = 2, kMiscLast = 3, kMiscZero = 4, kMiscWarpSums = 6 };
 
 __device__ __forceinline__ int clamp_ctx(int c, int W)
 {
@@ -103,7 +115,7 @@ __device__ __forceinline__ int clamp_ctx(int c, int W)
 __device__ __forceinline__ int seq_ctx(const DecodeArgs &a, int b) { return clamp_ctx(__ldg(a.context_lens + b), a.W); }
 __device__ __forceinline__ int ctx_blocks(int c) { return (c + kBlockTokens - 1) / kBlockTokens; }
 
-// Inclusive scan over the 160 threads; *total receives the sum of all values.
+// Inclusive scan over all kThreads threads; *total receives the sum.
 __device__ __forceinline__ int block_scan_incl(int v, volatile int *warp_sums, int *total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -131,7 +143,7 @@ __device__ __forceinline__ int block_scan_incl(int v, volatile int *warp_sums, i
 
 struct Cursor {
     int b;     // sequence
-    int k;     // item within the sequence: j * hchunks + head chunk
+    int k;     // item within the sequence: head group * hchunks + query-head chunk
     int off;   // block offset within the sequence
     int ctx;   // tokens of sequence b (clamped)
     int n;     // blocks of sequence b
@@ -173,34 +185,69 @@ __device__ __forceinline__ void sts128_zero(uint32_t addr)
     asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(addr), "r"(0) : "memory");
 }
 
-// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128B-swizzled box.
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside one head's 128B-swizzled tile.
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
+// exp2(x - m) for merging states whose maxima may both be -inf (empty states).
+__device__ __forceinline__ float rescale(float x, float m) { return m == -INFINITY ? 0.f : exp2f(x - m); }
+
+// Where an item's outputs go.
+struct ItemOut {
+    int b, h0, gc;   // sequence, first query head of this warp's kv head, valid query heads (<= 8)
+    size_t slot;     // split-K piece slot (only for partial items)
+    int hh;          // kv head within the group
+};
+
+__device__ __forceinline__ ItemOut item_out(const DecodeArgs &a, const Cursor &cur, int hh)
+{
+    const int hg = cur.k / a.hchunks, hc = cur.k - hg * a.hchunks;
+    ItemOut o;
+    o.b = cur.b;
+    o.hh = hh;
+    o.h0 = (hg * a.hg + hh) * a.group + hc * kGroupMax;
+    o.gc = min(kGroupMax, a.group - hc * kGroupMax);
+    o.slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(cur.b) * a.items_per_seq + cur.k;
+    return o;
+}
+
 // ---------------------------------------------------------------------------
-// Per-warp consumer state and arithmetic.
+// Per-warp consumer state and arithmetic (one kv head of each unit).
 // ---------------------------------------------------------------------------
 template <int D, int PATH, int NH>
 struct Consumer;
 
 // Tensor-core path. Lane (r = lane/4, c = lane%4) holds scores of tokens r and
-// r+8 for heads 2c and 2c+1, and the accumulator O^T rows d = 16*mt + r (+8)
-// for the same two heads.
+// r+8 for query heads 2c and 2c+1, and the accumulator O^T rows d = 16*mt + r
+// (+8) for the same two heads.
 template <int D, int NH>
 struct Consumer<D, kPathMma, NH> {
     static constexpr int kTiles = D / 64;
     static constexpr int kMt = D / 16;
-    uint32_t qf[kMt][2];
+    static constexpr int kRegs = kMt * 4 + 4;
+    uint32_t qf[kMt][2];   // this item's query fragments (B operand of S^T = K Q^T)
+    uint32_t qn[kMt][2];   // the next item's, loaded one item ahead
     float acc[kMt][4];
     float m0, m1, l0, l1;
 
-    __device__ __forceinline__ void begin_item(const DecodeArgs &a, int b, int h0, int gc, float *)
+    // Issue the loads of an item's query fragments into qn (used at its begin_item).
+    __device__ __forceinline__ void prefetch_q(const DecodeArgs &a, const ItemOut &o)
     {
         const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
-        const uint32_t *qrow = reinterpret_cast<const uint32_t *>(a.q + (static_cast<size_t>(b) * a.Hq + h0 + r) * D);
+        const uint32_t *qrow =
+            reinterpret_cast<const uint32_t *>(a.q + (static_cast<size_t>(o.b) * a.Hq + o.h0 + r) * D);
 #pragma unroll
         for (int kk = 0; kk < kMt; ++kk) {
-            qf[kk][0] = (r < gc) ? __ldg(qrow + kk * 8 + c) : 0u;
-            qf[kk][1] = (r < gc) ? __ldg(qrow + kk * 8 + 4 + c) : 0u;
+            qn[kk][0] = (r < o.gc) ? __ldg(qrow + kk * 8 + c) : 0u;
+            qn[kk][1] = (r < o.gc) ? __ldg(qrow + kk * 8 + 4 + c) : 0u;
+        }
+    }
+
+    __device__ __forceinline__ void begin_item(const DecodeArgs &, const ItemOut &, const float *)
+    {
+#pragma unroll
+        for (int kk = 0; kk < kMt; ++kk) {
+            qf[kk][0] = qn[kk][0];
+            qf[kk][1] = qn[kk][1];
         }
 #pragma unroll
         for (int mt = 0; mt < kMt; ++mt)
@@ -209,7 +256,8 @@ struct Consumer<D, kPathMma, NH> {
         l0 = l1 = 0.f;
     }
 
-    __device__ __forceinline__ void unit(uint32_t kbase, uint32_t vbase, int valid, float sl2, float *)
+    __device__ __forceinline__ void unit(uint32_t kbase, uint32_t vbase, int tile_stride, int valid, float sl2,
+                                         const float *, float *)
     {
         const int lane = threadIdx.x & 31, r = lane >> 2, mi = lane >> 3, rr = lane & 7;
         if (valid < 16) {
@@ -219,7 +267,7 @@ struct Consumer<D, kPathMma, NH> {
                 const int t = idx / (8 * kTiles);
                 const int rem = idx - t * 8 * kTiles;
                 const int tile = rem >> 3, ch = rem & 7;
-                sts128_zero(vbase + tile * kTileBytes + (valid + t) * 128 + ch * 16);
+                sts128_zero(vbase + tile * tile_stride + (valid + t) * 128 + ch * 16);
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
@@ -232,7 +280,7 @@ struct Consumer<D, kPathMma, NH> {
             for (int kk = 0; kk < kMt; ++kk) {
                 const int tile = kk >> 2, kc = kk & 3;
                 uint32_t af[4];
-                ldmatrix_x4(af, kbase + tile * kTileBytes + swz(row, (kc << 1) + (mi >> 1)));
+                ldmatrix_x4(af, kbase + tile * tile_stride + swz(row, (kc << 1) + (mi >> 1)));
                 mma_bf16_16816(s, af, qf[kk][0], qf[kk][1]);
             }
         }
@@ -271,49 +319,125 @@ struct Consumer<D, kPathMma, NH> {
             acc[mt][3] *= al1;
             const int tile = mt >> 2, kc = mt & 3;
             uint32_t af[4];
-            ldmatrix_x4_trans(af, vbase + tile * kTileBytes + swz(vrow, (kc << 1) + (mi & 1)));
+            ldmatrix_x4_trans(af, vbase + tile * tile_stride + swz(vrow, (kc << 1) + (mi & 1)));
             mma_bf16_16816(acc[mt], af, bh0, bh1);
             mma_bf16_16816(acc[mt], af, bl0, bl1);
         }
     }
 
-    // Write this warp's (m, l, acc) for heads 0..7 into the merge scratch.
-    __device__ __forceinline__ void finish(float *acc_w, float *ml_w)
+    // Sum the running sums over the lanes that share a query head.
+    __device__ __forceinline__ void finish()
     {
-        const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
 #pragma unroll
         for (int o = 4; o < 32; o <<= 1) {
             l0 += __shfl_xor_sync(kFull, l0, o);
             l1 += __shfl_xor_sync(kFull, l1, o);
         }
-        constexpr int AS = Geo<D>::kAccStride;
+    }
+
+    // Hand this warp's state to a partner warp (same kv head, same lane layout).
+    __device__ __forceinline__ void save(float *slot) const
+    {
+        const int lane = threadIdx.x & 31;
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                slot[(mt * 4 + i) * 32 + lane] = acc[mt][i];
+        slot[(kMt * 4 + 0) * 32 + lane] = m0;
+        slot[(kMt * 4 + 1) * 32 + lane] = m1;
+        slot[(kMt * 4 + 2) * 32 + lane] = l0;
+        slot[(kMt * 4 + 3) * 32 + lane] = l1;
+    }
+
+    __device__ __forceinline__ void merge(const float *slot)
+    {
+        const int lane = threadIdx.x & 31;
+        const float pm0 = slot[(kMt * 4 + 0) * 32 + lane], pm1 = slot[(kMt * 4 + 1) * 32 + lane];
+        const float pl0 = slot[(kMt * 4 + 2) * 32 + lane], pl1 = slot[(kMt * 4 + 3) * 32 + lane];
+        const float M0 = fmaxf(m0, pm0), M1 = fmaxf(m1, pm1);
+        const float a0 = rescale(m0, M0), b0 = rescale(pm0, M0);
+        const float a1 = rescale(m1, M1), b1 = rescale(pm1, M1);
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt) {
+            acc[mt][0] = acc[mt][0] * a0 + slot[(mt * 4 + 0) * 32 + lane] * b0;
+            acc[mt][1] = acc[mt][1] * a1 + slot[(mt * 4 + 1) * 32 + lane] * b1;
+            acc[mt][2] = acc[mt][2] * a0 + slot[(mt * 4 + 2) * 32 + lane] * b0;
+            acc[mt][3] = acc[mt][3] * a1 + slot[(mt * 4 + 3) * 32 + lane] * b1;
+        }
+        l0 = l0 * a0 + pl0 * b0;
+        l1 = l1 * a1 + pl1 * b1;
+        m0 = M0;
+        m1 = M1;
+    }
+
+    __device__ __forceinline__ void store_final(const DecodeArgs &a, const ItemOut &o) const
+    {
+        const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+        const int n0 = 2 * c, n1 = 2 * c + 1;
+        const float i0 = 1.f / l0, i1 = 1.f / l1;
+        __nv_bfloat16 *o0 = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n0) * D;
+        __nv_bfloat16 *o1 = o0 + D;
 #pragma unroll
         for (int mt = 0; mt < kMt; ++mt) {
             const int d = mt * 16 + r;
-            acc_w[(2 * c) * AS + d] = acc[mt][0];
-            acc_w[(2 * c + 1) * AS + d] = acc[mt][1];
-            acc_w[(2 * c) * AS + d + 8] = acc[mt][2];
-            acc_w[(2 * c + 1) * AS + d + 8] = acc[mt][3];
+            if (n0 < o.gc) {
+                o0[d] = __float2bfloat16(acc[mt][0] * i0);
+                o0[d + 8] = __float2bfloat16(acc[mt][2] * i0);
+            }
+            if (n1 < o.gc) {
+                o1[d] = __float2bfloat16(acc[mt][1] * i1);
+                o1[d + 8] = __float2bfloat16(acc[mt][3] * i1);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void store_partial(const DecodeArgs &a, const ItemOut &o) const
+    {
+        const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+        const int n0 = 2 * c, n1 = 2 * c + 1;
+        const size_t head0 = (o.slot * kMaxHG + o.hh) * kGroupMax;
+        float *p0 = a.part_acc + (head0 + n0) * D;
+        float *p1 = a.part_acc + (head0 + n1) * D;
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt) {
+            const int d = mt * 16 + r;
+            if (n0 < o.gc) {
+                p0[d] = acc[mt][0];
+                p0[d + 8] = acc[mt][2];
+            }
+            if (n1 < o.gc) {
+                p1[d] = acc[mt][1];
+                p1[d + 8] = acc[mt][3];
+            }
         }
         if (r == 0) {
-            ml_w[(2 * c) * 2] = m0;
-            ml_w[(2 * c) * 2 + 1] = l0;
-            ml_w[(2 * c + 1) * 2] = m1;
-            ml_w[(2 * c + 1) * 2 + 1] = l1;
+            if (n0 < o.gc) {
+                a.part_ml[(head0 + n0) * 2] = m0;
+                a.part_ml[(head0 + n0) * 2 + 1] = l0;
+            }
+            if (n1 < o.gc) {
+                a.part_ml[(head0 + n1) * 2] = m1;
+                a.part_ml[(head0 + n1) * 2 + 1] = l1;
+            }
         }
     }
 };
 
 // CUDA-core path. QK: lane (t = lane/2, half = lane%2) dots token t's half row
-// with every head; PV: lane owns D/32 output columns for every head.
+// with every query head; PV: lane owns D/32 output columns for every head.
 template <int D, int NH>
 struct Consumer<D, kPathSimt, NH> {
     static constexpr int E = D / 32;
     static constexpr int CPH = D / 16;
+    static constexpr int kRegs = NH * E + 2 * NH;
     float acc[NH][E];
     float m[NH], l[NH];
 
-    __device__ __forceinline__ void begin_item(const DecodeArgs &, int, int, int, float *)
+    // The CUDA-core path stages the whole item's q in shared memory instead.
+    __device__ __forceinline__ void prefetch_q(const DecodeArgs &, const ItemOut &) {}
+
+    __device__ __forceinline__ void begin_item(const DecodeArgs &, const ItemOut &, const float *)
     {
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
@@ -325,12 +449,11 @@ struct Consumer<D, kPathSimt, NH> {
         }
     }
 
-    // q_s: [8][kQStride] fp32 (filled by the CTA), p_s: this warp's [16][8] fp32
-    __device__ __forceinline__ void unit(uint32_t kbase, uint32_t vbase, int valid, float sl2, float *qp)
+    // q_s: this kv head's [8][kQStride] fp32 rows; p_s: this warp's [16][8] fp32
+    __device__ __forceinline__ void unit(uint32_t kbase, uint32_t vbase, int tile_stride, int valid, float sl2,
+                                         const float *q_s, float *p_s)
     {
         constexpr int QS = Geo<D>::kQStride;
-        const float *q_s = qp;
-        float *p_s = qp + kGroupMax * QS + (threadIdx.x >> 5) * 16 * kGroupMax;
         const int lane = threadIdx.x & 31, t = lane >> 1, half = lane & 1;
         float dot[NH];
 #pragma unroll
@@ -339,7 +462,7 @@ struct Consumer<D, kPathSimt, NH> {
 #pragma unroll
         for (int cc = 0; cc < CPH; ++cc) {
             const int dcol = half * (D / 2) + cc * 8;
-            const uint4 kv = lds128(kbase + (dcol >> 6) * kTileBytes + swz(t, (dcol & 63) >> 3));
+            const uint4 kv = lds128(kbase + (dcol >> 6) * tile_stride + swz(t, (dcol & 63) >> 3));
             const float k0 = bf16lo_to_f32(kv.x), k1 = bf16hi_to_f32(kv.x), k2 = bf16lo_to_f32(kv.y),
                         k3 = bf16hi_to_f32(kv.y), k4 = bf16lo_to_f32(kv.z), k5 = bf16hi_to_f32(kv.z),
                         k6 = bf16lo_to_f32(kv.w), k7 = bf16hi_to_f32(kv.w);
@@ -379,7 +502,7 @@ struct Consumer<D, kPathSimt, NH> {
         }
         __syncwarp();
         const int d0 = lane * E;
-        const uint32_t vcol = (d0 >> 6) * kTileBytes;
+        const uint32_t vcol = (d0 >> 6) * tile_stride;
         const int chunk = (d0 & 63) >> 3, within = d0 & 7;
 #pragma unroll
         for (int n = 0; n < NH; ++n)
@@ -412,50 +535,202 @@ struct Consumer<D, kPathSimt, NH> {
         __syncwarp();
     }
 
-    __device__ __forceinline__ void finish(float *acc_w, float *ml_w)
+    __device__ __forceinline__ void finish()
+    {
+#pragma unroll
+        for (int n = 0; n < NH; ++n)
+#pragma unroll
+            for (int o = 2; o < 32; o <<= 1)
+                l[n] += __shfl_xor_sync(kFull, l[n], o);
+    }
+
+    __device__ __forceinline__ void save(float *slot) const
     {
         const int lane = threadIdx.x & 31;
-        constexpr int AS = Geo<D>::kAccStride;
 #pragma unroll
-        for (int n = 0; n < kGroupMax; ++n) {
-            float ln = 0.f, mn = -INFINITY;
-            if (n < NH) {
-                ln = l[n];
-#pragma unroll
-                for (int o = 2; o < 32; o <<= 1)
-                    ln += __shfl_xor_sync(kFull, ln, o);
-                mn = m[n];
-            }
+        for (int n = 0; n < NH; ++n) {
 #pragma unroll
             for (int e = 0; e < E; ++e)
-                acc_w[n * AS + lane * E + e] = (n < NH) ? acc[n < NH ? n : 0][e] : 0.f;
-            if (lane == 0) {
-                ml_w[n * 2] = mn;
-                ml_w[n * 2 + 1] = ln;
+                slot[(n * E + e) * 32 + lane] = acc[n][e];
+            slot[(NH * E + n) * 32 + lane] = m[n];
+            slot[(NH * E + NH + n) * 32 + lane] = l[n];
+        }
+    }
+
+    __device__ __forceinline__ void merge(const float *slot)
+    {
+        const int lane = threadIdx.x & 31;
+#pragma unroll
+        for (int n = 0; n < NH; ++n) {
+            const float pm = slot[(NH * E + n) * 32 + lane], pl = slot[(NH * E + NH + n) * 32 + lane];
+            const float M = fmaxf(m[n], pm);
+            const float a = rescale(m[n], M), b = rescale(pm, M);
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                acc[n][e] = acc[n][e] * a + slot[(n * E + e) * 32 + lane] * b;
+            l[n] = l[n] * a + pl * b;
+            m[n] = M;
+        }
+    }
+
+    __device__ __forceinline__ void store_final(const DecodeArgs &a, const ItemOut &o) const
+    {
+        const int lane = threadIdx.x & 31;
+#pragma unroll
+        for (int n = 0; n < NH; ++n) {
+            if (n < o.gc) {
+                const float inv = 1.f / l[n];
+                __nv_bfloat16 *dst = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n) * D + lane * E;
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    dst[e] = __float2bfloat16(acc[n][e] * inv);
+            }
+        }
+    }
+
+    __device__ __forceinline__ void store_partial(const DecodeArgs &a, const ItemOut &o) const
+    {
+        const int lane = threadIdx.x & 31;
+        const size_t head0 = (o.slot * kMaxHG + o.hh) * kGroupMax;
+#pragma unroll
+        for (int n = 0; n < NH; ++n) {
+            if (n < o.gc) {
+                float *dst = a.part_acc + (head0 + n) * D + lane * E;
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    dst[e] = acc[n][e];
+                if (lane == 0) {
+                    a.part_ml[(head0 + n) * 2] = m[n];
+                    a.part_ml[(head0 + n) * 2 + 1] = l[n];
+                }
             }
         }
     }
 };
 
-// Log-sum-exp merge of split-K pieces of one item, read from global memory.
+// Log-sum-exp merge of the split-K pieces of one item, read from global memory.
+// The item's pieces sit in slots first_cta + item .. last_cta + item. Each
+// thread merges two groups of four output columns at a time, and all loads
+// for up to four pieces are issued before any is used, so a merge costs
+// about one memory round trip per four pieces.
+constexpr int kMergeBatch = 4;
+
 template <int D>
 __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int item, int first_cta, int last_cta,
-                                                    int b, int h0, int gc, int tid, int nthreads)
+                                                    int b, int k, int tid, int nthreads)
 {
-    for (int idx = tid; idx < gc * D; idx += nthreads) {
-        const int n = idx / D, d = idx - n * D;
-        float M = -INFINITY;
-        for (int c = first_cta; c <= last_cta; ++c)
-            M = fmaxf(M, __ldcg(a.part_ml + ((static_cast<size_t>(c) + item) * kGroupMax + n) * 2));
-        float L = 0.f, O = 0.f;
-        for (int c = first_cta; c <= last_cta; ++c) {
-            const size_t slot = static_cast<size_t>(c) + item;
-            const float sc = exp2f(__ldcg(a.part_ml + (slot * kGroupMax + n) * 2) - M);
-            L = fmaf(sc, __ldcg(a.part_ml + (slot * kGroupMax + n) * 2 + 1), L);
-            O = fmaf(sc, __ldcg(a.part_acc + (slot * kGroupMax + n) * D + d), O);
+    constexpr int D4 = D / 4;
+    const int hg = k / a.hchunks, hc = k - hg * a.hchunks;
+    const int gc = min(kGroupMax, a.group - hc * kGroupMax);
+    const int per_head = gc * D4;
+    const int total = a.hg * per_head;
+    for (int base = tid; base < total; base += 2 * nthreads) {
+        size_t head[2];
+        int col[2];
+        bool ok[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int idx = base + e * nthreads;
+            ok[e] = idx < total;
+            const int i2 = ok[e] ? idx : base;
+            const int hh = i2 / per_head;
+            const int rem = i2 - hh * per_head;
+            const int n = rem / D4;
+            col[e] = (rem - n * D4) * 4;
+            head[e] = static_cast<size_t>(hh) * kGroupMax + n;  // within a slot
         }
-        a.out[(static_cast<size_t>(b) * a.Hq + h0 + n) * D + d] = __float2bfloat16(O / L);
+        float M[2] = {-INFINITY, -INFINITY}, L[2] = {0.f, 0.f};
+        float4 O[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+        for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
+            float mv[2][kMergeBatch], lv[2][kMergeBatch];
+            float4 ov[2][kMergeBatch];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+#pragma unroll
+                for (int j = 0; j < kMergeBatch; ++j) {
+                    const int c = c0 + j;
+                    if (c <= last_cta) {
+                        const size_t h = (static_cast<size_t>(c) + item) * (kMaxHG * kGroupMax) + head[e];
+                        mv[e][j] = __ldcg(a.part_ml + h * 2);
+                        lv[e][j] = __ldcg(a.part_ml + h * 2 + 1);
+                        ov[e][j] = __ldcg(reinterpret_cast<const float4 *>(a.part_acc + h * D + col[e]));
+                    } else {
+                        mv[e][j] = -INFINITY;
+                        lv[e][j] = 0.f;
+                        ov[e][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float Mb = M[e];
+#pragma unroll
+                for (int j = 0; j < kMergeBatch; ++j)
+                    Mb = fmaxf(Mb, mv[e][j]);
+                const float sc = rescale(M[e], Mb);
+                L[e] *= sc;
+                O[e].x *= sc;
+                O[e].y *= sc;
+                O[e].z *= sc;
+                O[e].w *= sc;
+#pragma unroll
+                for (int j = 0; j < kMergeBatch; ++j) {
+                    const float w = rescale(mv[e][j], Mb);
+                    L[e] = fmaf(w, lv[e][j], L[e]);
+                    O[e].x = fmaf(w, ov[e][j].x, O[e].x);
+                    O[e].y = fmaf(w, ov[e][j].y, O[e].y);
+                    O[e].z = fmaf(w, ov[e][j].z, O[e].z);
+                    O[e].w = fmaf(w, ov[e][j].w, O[e].w);
+                }
+                M[e] = Mb;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            if (!ok[e])
+                continue;
+            const int hh = static_cast<int>(head[e] / kGroupMax), n = static_cast<int>(head[e] % kGroupMax);
+            const int h = (hg * a.hg + hh) * a.group + hc * kGroupMax + n;
+            const float inv = 1.f / L[e];
+            __nv_bfloat162 lo = __floats2bfloat162_rn(O[e].x * inv, O[e].y * inv);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(O[e].z * inv, O[e].w * inv);
+            uint2 packed;
+            packed.x = *reinterpret_cast<uint32_t *>(&lo);
+            packed.y = *reinterpret_cast<uint32_t *>(&hi);
+            *reinterpret_cast<uint2 *>(a.out + (static_cast<size_t>(b) * a.Hq + h) * D + col[e]) = packed;
+        }
     }
+}
+
+// Outputs of empty sequences are zero; also flag out-of-range lengths. Run by CTA 0.
+template <int D>
+__device__ __forceinline__ void zero_empty_outputs(const DecodeArgs &a, int tid, int nthreads)
+{
+    for (int b = tid; b < a.B; b += nthreads) {
+        const int c = __ldg(a.context_lens + b);
+        if (c < 0 || c > a.W * kBlockTokens)
+            atomicOr(a.status, KV_STATUS_BAD_CONTEXT);
+        if (clamp_ctx(c, a.W) == 0) {
+            __nv_bfloat16 *o = a.out + static_cast<size_t>(b) * a.Hq * D;
+            for (int i = 0; i < a.Hq * D; ++i)
+                o[i] = __float2bfloat16(0.f);
+        }
+    }
+}
+
+// Lane i (< m) reads the block id of unit cur.off + i of sequence cur.b; ids
+// outside the pool are flagged and replaced by block 0 (never read out of bounds).
+__device__ __forceinline__ int load_block_ids(const DecodeArgs &a, const Cursor &cur, int m, int lane)
+{
+    int blk = 0;
+    if (lane < m) {
+        blk = __ldg(a.block_tables + static_cast<size_t>(cur.b) * a.W + cur.off + lane);
+        if (blk < 0 || blk >= a.num_blocks) {
+            atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
+            blk = 0;
+        }
+    }
+    return blk;
 }
 
 template <int D, int PATH, int NH>
@@ -469,18 +744,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const uint32_t base_s = (raw_s + 1023u) & ~1023u;
     unsigned char *base = smem_raw + (base_s - raw_s);
     uint64_t *full = reinterpret_cast<uint64_t *>(base + G::kOffBar);
-    uint64_t *empty = full + G::kStages;
+    uint64_t *empty = full + G::kMaxStages;
     volatile int *misc = reinterpret_cast<volatile int *>(base + G::kOffMisc);
-    float *acc_scratch = reinterpret_cast<float *>(base + G::kOffAcc);
-    float *ml_scratch = reinterpret_cast<float *>(base + G::kOffMl);
-    float *qp_scratch = reinterpret_cast<float *>(base + G::kOffQ);
+    float *scratch = reinterpret_cast<float *>(base + G::kOffScratch);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int S = a.stages;
 
     if (tid == 0) {
-        for (int s = 0; s < G::kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], a.hg);  // the HG warps of the consuming stream
         }
         mbar_fence_init();
         misc[kMiscAbort] = 0;
@@ -527,25 +801,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
     }
 
-    // Everything below may touch what the previous kernel in the stream writes.
-    grid_dependency_wait();
-    grid_launch_dependents();
-
-    if (blockIdx.x == 0) {
-        // outputs of empty sequences, and the length check
-        for (int b = tid; b < a.B; b += kThreads) {
-            const int c = __ldg(a.context_lens + b);
-            if (c < 0 || c > a.W * kBlockTokens)
-                atomicOr(a.status, KV_STATUS_BAD_CONTEXT);
-            if (clamp_ctx(c, a.W) == 0) {
-                __nv_bfloat16 *o = a.out + static_cast<size_t>(b) * a.Hq * D;
-                for (int i = 0; i < a.Hq * D; ++i)
-                    o[i] = __float2bfloat16(0.f);
-            }
-        }
-    }
-    if (count <= 0)
+    if (count <= 0) {
+        grid_dependency_wait();
+        grid_launch_dependents();
+        if (blockIdx.x == 0)
+            zero_empty_outputs<D>(a, tid, kThreads);
         return;
+    }
 
     Cursor cur0;
     cur0.b = misc[kMiscLocB];
@@ -561,52 +823,59 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
     if (warp == kProducerWarp) {
         // ---------------- producer: block ids -> TMA loads ----------------
+        // The first batch of block ids is read before waiting on the previous
+        // grid (no kernel of this library writes the tables); the cache itself
+        // is only touched after the wait.
+        int blk_first = load_block_ids(a, cur0, min(32, min(cur0.n - cur0.off, count)), lane);
+        grid_dependency_wait();
+        grid_launch_dependents();
         const uint64_t policy = l2_policy_evict_first();
+        const int NL = a.prod_lanes;
         Cursor cur = cur0;
         int u = 0, issued = 0;
-        bool stop = false;
+        bool stop = false, first_batch = true;
         while (u < count && !stop) {
             const int run = min(cur.n - cur.off, count - u);
-            const int j = cur.k / a.hchunks;
-            const int32_t *row = a.block_tables + static_cast<size_t>(cur.b) * a.W + cur.off;
+            const int head0 = (cur.k / a.hchunks) * a.hg;
             for (int bi = 0; bi < run && !stop; bi += 32) {
                 const int m = min(32, run - bi);
-                int blk = 0;
-                if (lane < m) {
-                    blk = __ldg(row + bi + lane);
-                    if (blk < 0 || blk >= a.num_blocks) {
-                        atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
-                        blk = 0;
-                    }
+                int blk;
+                if (first_batch) {
+                    blk = blk_first;
+                    first_batch = false;
+                } else {
+                    Cursor at = cur;
+                    at.off = cur.off + bi;
+                    blk = load_block_ids(a, at, m, lane);
                 }
-                for (int i = 0; i < m; ++i) {
-                    const int phys = __shfl_sync(kFull, blk, i);
-                    const int uu = u + bi + i;
-                    const int s = uu % G::kStages;
+                for (int i0 = 0; i0 < m; i0 += NL) {
+                    const int i = i0 + lane;
+                    const int phys = __shfl_sync(kFull, blk, i & 31);
                     int ok = 1;
-                    if (lane == 0) {
-                        ok = mbar_wait_bounded(&empty[s], ((uu / G::kStages) & 1) ^ 1, abort_flag);
+                    if (lane < NL && i < m) {
+                        const int uu = u + bi + i;
+                        const int s = uu % S;
+                        ok = mbar_wait_bounded(&empty[s], ((uu / S) & 1) ^ 1, abort_flag);
                         if (ok) {
-                            mbar_arrive_expect_tx(&full[s], G::kStageBytes);
-                            const uint32_t dst = ring + s * G::kStageBytes;
+                            mbar_arrive_expect_tx(&full[s], a.stage_bytes);
+                            const uint32_t dst = ring + s * a.stage_bytes;
 #pragma unroll
                             for (int t = 0; t < G::kTiles; ++t)
-                                tma_load_4d(dst + t * kTileBytes, &tmK, t * 64, j, 0, phys, &full[s], policy);
+                                tma_load_4d(dst + t * a.tile_stride, &tmK, t * 64, 0, head0, phys, &full[s], policy);
 #pragma unroll
                             for (int t = 0; t < G::kTiles; ++t)
-                                tma_load_4d(dst + (G::kTiles + t) * kTileBytes, &tmV, t * 64, j, 0, phys, &full[s],
-                                            policy);
+                                tma_load_4d(dst + (G::kTiles + t) * a.tile_stride, &tmV, t * 64, 0, head0, phys,
+                                            &full[s], policy);
                         } else {
                             *abort_flag = 1;
                             atomicOr(a.status, KV_STATUS_WAIT_TIMEOUT);
                         }
                     }
-                    ok = __shfl_sync(kFull, ok, 0);
-                    if (!ok) {
+                    if (!__all_sync(kFull, ok)) {
                         stop = true;
                         break;
                     }
-                    issued = uu + 1;
+                    issued = u + bi + min(i0 + NL, m);
                 }
             }
             u += run;
@@ -614,25 +883,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 cursor_next_item(a, cur);
         }
         // No load may land after this CTA exits: wait (bounded) for the last ones.
-        if (lane == 0) {
-            for (int v = max(0, issued - G::kStages); v < issued; ++v)
-                mbar_wait_bounded(&full[v % G::kStages], (v / G::kStages) & 1, misc + kMiscZero);
+        if (lane < NL) {
+            for (int v = max(0, issued - S); v < issued; ++v)
+                if (v % NL == lane)
+                    mbar_wait_bounded(&full[v % S], (v / S) & 1, misc + kMiscZero);
         }
         return;
     }
 
-    // -------------------- consumers: warps 0..3 --------------------
+    // -------------------- consumers: warps 0..7 --------------------
+    const int hh = warp % a.hg;          // kv head within the group
+    const int stream = warp / a.hg;      // which units: u % streams == stream
+    const int NS = a.streams;
     Consumer<D, PATH, NH> st;
+    float *q_s = scratch + hh * kGroupMax * G::kQStride;                         // CUDA-core path only
+    float *p_s = scratch + kMaxHG * kGroupMax * G::kQStride + warp * 16 * kGroupMax;
+    st.prefetch_q(a, item_out(a, cur0, hh));  // q is never written by this library: no wait needed
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if (blockIdx.x == 0)
+        zero_empty_outputs<D>(a, tid, kConsumerThreads);
     Cursor cur = cur0;
     int u = 0;
-    float *acc_w = acc_scratch + warp * kGroupMax * G::kAccStride;
-    float *ml_w = ml_scratch + warp * kGroupMax * 2;
     while (u < count) {
         const int run = min(cur.n - cur.off, count - u);
         const int item = cur.b * a.items_per_seq + cur.k;
-        const int j = cur.k / a.hchunks, hc = cur.k - (cur.k / a.hchunks) * a.hchunks;
-        const int h0 = j * a.group + hc * kGroupMax;
-        const int gc = min(kGroupMax, a.group - hc * kGroupMax);
+        const int hg = cur.k / a.hchunks, hc = cur.k - hg * a.hchunks;
+        const ItemOut o = item_out(a, cur, hh);
         const int item_start = start + u - cur.off;
         const int first_cta = item_start / chunk;
         const int last_cta = (item_start + cur.n - 1) / chunk;
@@ -640,62 +917,68 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
         if (PATH == kPathSimt) {
             // this item's query rows as fp32 in shared memory (heads >= gc are zero)
-            for (int idx = tid; idx < kGroupMax * D; idx += kConsumerThreads) {
-                const int n = idx / D, d = idx - n * D;
-                const float v = (n < gc) ? __bfloat162float(a.q[(static_cast<size_t>(cur.b) * a.Hq + h0 + n) * D + d])
-                                         : 0.f;
-                qp_scratch[n * G::kQStride + d + ((d >= D / 2) ? 4 : 0)] = v;
+            const int per = kGroupMax * D;
+            for (int idx = tid; idx < a.hg * per; idx += kConsumerThreads) {
+                const int h2 = idx / per;
+                const int rem = idx - h2 * per;
+                const int n = rem / D, d = rem - n * D;
+                const int h = (hg * a.hg + h2) * a.group + hc * kGroupMax + n;
+                const float v = (n < o.gc) ? __bfloat162float(a.q[(static_cast<size_t>(cur.b) * a.Hq + h) * D + d])
+                                           : 0.f;
+                scratch[(h2 * kGroupMax + n) * G::kQStride + d + ((d >= D / 2) ? 4 : 0)] = v;
             }
             named_barrier(1, kConsumerThreads);
         }
-        st.begin_item(a, cur.b, h0, gc, qp_scratch);
-        for (int i = ((warp - u) % kConsumerWarps + kConsumerWarps) % kConsumerWarps; i < run; i += kConsumerWarps) {
+        st.begin_item(a, o, q_s);
+        if (u + run < count) {
+            Cursor next = cur;
+            cursor_next_item(a, next);
+            st.prefetch_q(a, item_out(a, next, hh));
+        }
+        for (int i = ((stream - u) % NS + NS) % NS; i < run; i += NS) {
             const int uu = u + i;
-            const int s = uu % G::kStages;
-            if (!mbar_wait_bounded(&full[s], (uu / G::kStages) & 1, abort_flag)) {
+            const int s = uu % S;
+            if (!mbar_wait_bounded(&full[s], (uu / S) & 1, abort_flag)) {
                 if (lane == 0) {
                     *abort_flag = 1;
                     atomicOr(a.status, KV_STATUS_WAIT_TIMEOUT);
                 }
                 break;
             }
-            const uint32_t kb = ring + s * G::kStageBytes;
+            const uint32_t kb = ring + s * a.stage_bytes + hh * kHeadTileBytes;
             const int valid = min(kBlockTokens, cur.ctx - (cur.off + i) * kBlockTokens);
-            st.unit(kb, kb + G::kTiles * kTileBytes, valid, a.scale_log2, qp_scratch);
+            st.unit(kb, kb + G::kTiles * a.tile_stride, a.tile_stride, valid, a.scale_log2, q_s, p_s);
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&empty[s]);
         }
+        st.finish();
 
-        // ---- merge the four warps ----
-        st.finish(acc_w, ml_w);
-        named_barrier(1, kConsumerThreads);
-        const size_t slot = static_cast<size_t>(blockIdx.x) + item;
-        for (int idx = tid; idx < gc * D; idx += kConsumerThreads) {
-            const int n = idx / D, d = idx - n * D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w)
-                M = fmaxf(M, ml_scratch[(w * kGroupMax + n) * 2]);
-            float L = 0.f, O = 0.f;
-#pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) {
-                const float sc = exp2f(ml_scratch[(w * kGroupMax + n) * 2] - M);
-                L = fmaf(sc, ml_scratch[(w * kGroupMax + n) * 2 + 1], L);
-                O = fmaf(sc, acc_scratch[(w * kGroupMax + n) * G::kAccStride + d], O);
-            }
-            if (single) {
-                a.out[(static_cast<size_t>(cur.b) * a.Hq + h0 + n) * D + d] = __float2bfloat16(O / L);
-            } else {
-                a.part_acc[(slot * kGroupMax + n) * D + d] = O;
-                if (d == 0) {
-                    a.part_ml[(slot * kGroupMax + n) * 2] = M;
-                    a.part_ml[(slot * kGroupMax + n) * 2 + 1] = L;
-                }
-            }
+        // ---- merge the streams pairwise: stream s + step hands over to stream s ----
+        if (PATH == kPathSimt)
+            named_barrier(1, kConsumerThreads);  // the scratch also holds q_s / p_s
+        for (int step = 1; step < NS; step <<= 1) {
+            const bool giver = (stream % (2 * step)) == step;
+            const bool taker = (stream % (2 * step)) == 0 && stream + step < NS;
+            const int slot_giver = (stream / (2 * step)) * a.hg + hh;
+            const int slot_taker = ((stream + step) / (2 * step)) * a.hg + hh;
+            if (giver)
+                st.save(scratch + slot_giver * Consumer<D, PATH, NH>::kRegs * 32);
+            named_barrier(1, kConsumerThreads);
+            if (taker)
+                st.merge(scratch + slot_taker * Consumer<D, PATH, NH>::kRegs * 32);
+            named_barrier(1, kConsumerThreads);
+        }
+
+        if (stream == 0) {
+            if (single)
+                st.store_final(a, o);
+            else
+                st.store_partial(a, o);
         }
         if (!single && a.fused) {
-            __threadfence();
+            if (stream == 0)
+                __threadfence();  // this warp's partial is visible before the counter moves
             named_barrier(1, kConsumerThreads);
             if (tid == 0) {
                 const int prev = atomicAdd(a.counters + item, 1);
@@ -704,7 +987,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             named_barrier(1, kConsumerThreads);
             if (misc[kMiscLast]) {
                 __threadfence();
-                merge_pieces_global<D>(a, item, first_cta, last_cta, cur.b, h0, gc, tid, kConsumerThreads);
+                merge_pieces_global<D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads);
                 if (tid == 0)
                     a.counters[item] = 0;
             }
@@ -754,10 +1037,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int gr
     const int first_cta = item_start / chunk, last_cta = (item_start + n - 1) / chunk;
     if (first_cta == last_cta)
         return;
-    const int j = k / a.hchunks, hc = k - j * a.hchunks;
-    const int h0 = j * a.group + hc * kGroupMax;
-    const int gc = min(kGroupMax, a.group - hc * kGroupMax);
-    merge_pieces_global<D>(a, item, first_cta, last_cta, b, h0, gc, threadIdx.x, 128);
+    merge_pieces_global<D>(a, item, first_cta, last_cta, b, k, threadIdx.x, 128);
 }
 
 }  // namespace pkv
@@ -773,7 +1053,8 @@ std::atomic<int> g_opt_compute{0};
 std::atomic<int> g_opt_combine{0};
 std::atomic<int> g_opt_grid{0};
 std::atomic<int> g_opt_min_chunk{0};
-constexpr int kDefaultMinChunk = 8;
+std::atomic<int> g_opt_prod_lanes{0};
+constexpr int kDefaultMinChunk = 4;
 
 constexpr int kMaxDevices = 64;
 
@@ -791,6 +1072,9 @@ int device_sm_count(int dev)
     return v;
 }
 
+// kv heads per work unit: 4 when Hkv is a multiple of 4, else 2 or 1
+int heads_per_unit(int Hkv) { return Hkv % 4 == 0 ? 4 : (Hkv % 2 == 0 ? 2 : 1); }
+
 struct Layout {
     int items = 0, slots = 0, max_grid = 0;
     size_t off_counters = 0, off_ml = 0, off_acc = 0, bytes = 0;
@@ -804,7 +1088,7 @@ bool make_layout(int B, int Hq, int Hkv, int D, int sms, Layout *L)
         return false;
     const int group = Hq / Hkv;
     const long long hchunks = (group + kGroupMax - 1) / kGroupMax;
-    const long long items = static_cast<long long>(B) * Hkv * hchunks;
+    const long long items = static_cast<long long>(B) * (Hkv / heads_per_unit(Hkv)) * hchunks;
     if (items > (1ll << 30))
         return false;
     L->items = static_cast<int>(items);
@@ -812,8 +1096,8 @@ bool make_layout(int B, int Hq, int Hkv, int D, int sms, Layout *L)
     L->slots = L->max_grid + L->items;
     L->off_counters = kStatusBytes;
     L->off_ml = L->off_counters + round256(static_cast<size_t>(L->items) * 4);
-    L->off_acc = L->off_ml + round256(static_cast<size_t>(L->slots) * kGroupMax * 2 * 4);
-    L->bytes = L->off_acc + round256(static_cast<size_t>(L->slots) * kGroupMax * D * 4);
+    L->off_acc = L->off_ml + round256(static_cast<size_t>(L->slots) * kMaxHG * kGroupMax * 2 * 4);
+    L->bytes = L->off_acc + round256(static_cast<size_t>(L->slots) * kMaxHG * kGroupMax * D * 4);
     return true;
 }
 
@@ -835,18 +1119,20 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
-// View one cache tensor [num_blocks][16][Hkv][D] as a 4-D map (D, Hkv, 16, num_blocks)
-// with a box of 64 columns x 1 head x 16 rows x 1 block, 128-byte swizzle.
-bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv, int D)
+// View one cache tensor [num_blocks][16][Hkv][D] as a 4-D map whose dimensions
+// are (column, row, kv head, block) -- rows inside heads, so each head's 16
+// rows land as one contiguous 128B-swizzled 2 KB tile -- with a box of
+// 64 columns x 16 rows x HG heads x 1 block.
+bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv, int D, int hg)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc)
         return false;
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(Hkv), 16,
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), 16, static_cast<cuuint64_t>(Hkv),
                                 static_cast<cuuint64_t>(num_blocks)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(Hkv) * D * 2,
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Hkv) * D * 2, static_cast<cuuint64_t>(D) * 2,
                                    static_cast<cuuint64_t>(16) * Hkv * D * 2};
-    const cuuint32_t box[4] = {64, 1, 16, 1};
+    const cuuint32_t box[4] = {64, 16, static_cast<cuuint32_t>(hg), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(cache), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -947,8 +1233,10 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
     if (misaligned(out, 16) || misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) ||
         misaligned(block_tables, 4) || misaligned(context_lens, 4) || misaligned(workspace, 256))
         return KV_ERR_ARG;
-    if (static_cast<long long>(B) * max_blocks_per_seq * Hkv * ((Hq / Hkv + kGroupMax - 1) / kGroupMax) >=
-        (1ll << 31))
+    const int group = Hq / Hkv;
+    const int hg = heads_per_unit(Hkv);
+    const int hchunks = (group + kGroupMax - 1) / kGroupMax;
+    if (static_cast<long long>(B) * max_blocks_per_seq * (Hkv / hg) * hchunks >= (1ll << 31))
         return KV_ERR_ARG;
 
     int dev = 0;
@@ -961,7 +1249,6 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
     if (workspace_bytes < L.bytes)
         return KV_ERR_ARG;
 
-    const int group = Hq / Hkv;
     int path = g_opt_compute.load();
     if (path == 0)
         path = kPathMma;
@@ -982,8 +1269,25 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
     if (want > 0)
         grid = want < L.max_grid ? want : L.max_grid;
 
+    // ring geometry: stages a multiple of the consumer streams and of the producer lanes
+    const int tiles = D / 64;
+    const int streams = kConsumerWarps / hg;
+    int lanes = g_opt_prod_lanes.load();
+    if (lanes <= 0)
+        lanes = hg >= 4 ? 1 : (hg == 2 ? 2 : 4);
+    const int stage_bytes = 2 * tiles * hg * kHeadTileBytes;
+    const int unit_of = streams > lanes ? streams : lanes;
+    const int ring = D == 64 ? Geo<64>::kRingBytes : Geo<128>::kRingBytes;
+    const int max_stages = D == 64 ? Geo<64>::kMaxStages : Geo<128>::kMaxStages;
+    int stages = (ring / stage_bytes) / unit_of * unit_of;
+    if (stages > max_stages)
+        stages = max_stages / unit_of * unit_of;
+    if (stages < unit_of)
+        return KV_ERR_ARG;
+
     CUtensorMap tmK, tmV;
-    if (!make_cache_map(&tmK, k_cache, num_blocks, Hkv, D) || !make_cache_map(&tmV, v_cache, num_blocks, Hkv, D))
+    if (!make_cache_map(&tmK, k_cache, num_blocks, Hkv, D, hg) ||
+        !make_cache_map(&tmV, v_cache, num_blocks, Hkv, D, hg))
         return KV_ERR_CUDA;
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
@@ -1001,9 +1305,15 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
     a.Hq = Hq;
     a.Hkv = Hkv;
     a.group = group;
-    a.hchunks = (group + kGroupMax - 1) / kGroupMax;
-    a.items_per_seq = Hkv * a.hchunks;
     a.num_blocks = num_blocks;
+    a.hg = hg;
+    a.streams = streams;
+    a.hchunks = hchunks;
+    a.items_per_seq = (Hkv / hg) * hchunks;
+    a.stages = stages;
+    a.stage_bytes = stage_bytes;
+    a.tile_stride = hg * kHeadTileBytes;
+    a.prod_lanes = lanes;
     const int mc = g_opt_min_chunk.load();
     a.min_chunk = mc > 0 ? mc : kDefaultMinChunk;
     const int combine_mode = g_opt_combine.load();
@@ -1133,6 +1443,11 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_min_chunk.store(value);
         return KV_OK;
+    case KV_OPT_PRODUCER_LANES:
+        if (value < 0 || value > 8 || (value & (value - 1)) != 0)
+            return KV_ERR_ARG;
+        g_opt_prod_lanes.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -1149,6 +1464,8 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_grid.load();
     case KV_OPT_MIN_CHUNK:
         return g_opt_min_chunk.load();
+    case KV_OPT_PRODUCER_LANES:
+        return g_opt_prod_lanes.load();
     default:
         return -1;
     }

@@ -19,7 +19,8 @@ PATHS = {"tensor_cores": 1, "cuda_cores": 2}
 @pytest.fixture(autouse=True)
 def _default_options(pkv):
     yield
-    for key in (pkv.KV_OPT_COMPUTE, pkv.KV_OPT_COMBINE, pkv.KV_OPT_GRID, pkv.KV_OPT_MIN_CHUNK):
+    for key in (pkv.KV_OPT_COMPUTE, pkv.KV_OPT_COMBINE, pkv.KV_OPT_GRID, pkv.KV_OPT_MIN_CHUNK,
+                pkv.KV_OPT_PRODUCER_LANES):
         pkv.set_option(key, 0)
 
 
@@ -51,7 +52,7 @@ def test_tiny_workload(pkv, oracle_mod, cuda_device, path, combine):
 
 @pytest.mark.parametrize("path", sorted(PATHS))
 @pytest.mark.parametrize("D,Hq,Hkv", [(64, 20, 4), (128, 32, 8), (128, 8, 8), (64, 16, 2), (128, 64, 8),
-                                      (128, 32, 2), (64, 12, 1)])
+                                      (128, 32, 2), (64, 12, 1), (64, 18, 6), (128, 7, 7), (128, 32, 32)])
 def test_ragged_lengths_and_head_groups(pkv, oracle_mod, cuda_device, path, D, Hq, Hkv):
     """Lengths at and around block edges, the table's maximum, 1 and 0; groups 1..16."""
     pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
@@ -70,6 +71,16 @@ def test_many_split_pieces(pkv, oracle_mod, cuda_device, cid, grid, min_chunk):
     cfg = workloads.small_config(cid, batch=6, ctx_lo=1, ctx_hi=1500, W=96, n_layers=1)
     case = Case(cfg, cuda_device)
     run_and_check(pkv, oracle_mod, case, what=f"config {cid} shape, grid {grid} min_chunk {min_chunk}")
+
+
+@pytest.mark.parametrize("lanes", [1, 2, 4, 8])
+@pytest.mark.parametrize("Hkv", [1, 4])
+def test_producer_lanes(pkv, oracle_mod, cuda_device, lanes, Hkv):
+    """Tile loads issued from 1..8 producer lanes (units of 1 or 4 kv heads)."""
+    pkv.set_option(pkv.KV_OPT_PRODUCER_LANES, lanes)
+    cfg = workloads.small_config(2, Hq=4 * Hkv, Hkv=Hkv, batch=5, ctx_lo=1, ctx_hi=900, W=64, n_layers=1)
+    case = Case(cfg, cuda_device)
+    run_and_check(pkv, oracle_mod, case, what=f"{lanes} producer lanes, Hkv {Hkv}")
 
 
 # ---------------------------------------------------------------------------
