@@ -209,6 +209,10 @@ class Workload:
         self.pkv = pkv
         self.cfg = cfg
         self.layout = workloads.draw_layout(cfg)
+        if cfg.redraw_fraction > 0:
+            # the batch is re-formed every step through the block pool (shared-prefix refcounts)
+            from paged_kv_cache_470_b200.batch import ContinuousBatch
+            self.layout = ContinuousBatch(cfg, int(self.layout.num_blocks * 1.25), seed=cfg.seed + 1000 * rank)
         gen = workloads.device_generator(cfg.seed + 1000 * rank, device)
         self.k, self.v = [], []
         for _ in range(cfg.n_layers):
@@ -221,14 +225,28 @@ class Workload:
         self.slots = self.layout.slot_mapping().to(device)
         self.out = torch.empty_like(self.q)
         self.ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D, device)
+        self.fused = True
+
+    def redraw(self):
+        """Re-form the batch (host bookkeeping) and upload the new tables; not timed."""
+        self.layout.redraw()
+        self.tables.copy_(self.layout.block_tables)
+        self.lens.copy_(self.layout.context_lens)
+        self.slots.copy_(self.layout.slot_mapping())
 
     def step(self, stream=None):
+        """Every layer: append this step's token and attend (one fused launch, or two kernels)."""
         pkv, cfg = self.pkv, self.cfg
         for layer in range(cfg.n_layers):
-            pkv.kv_cache_append(self.k_new[layer], self.v_new[layer], self.k[layer], self.v[layer], self.slots,
-                                stream=stream)
-            pkv.paged_attention_decode(self.out[layer], self.q[layer], self.k[layer], self.v[layer], self.tables,
-                                       self.lens, cfg.scale, self.ws, stream=stream)
+            if self.fused:
+                pkv.paged_attention_decode_append(self.out[layer], self.q[layer], self.k_new[layer],
+                                                  self.v_new[layer], self.k[layer], self.v[layer], self.slots,
+                                                  self.tables, self.lens, cfg.scale, self.ws, stream=stream)
+            else:
+                pkv.kv_cache_append(self.k_new[layer], self.v_new[layer], self.k[layer], self.v[layer], self.slots,
+                                    stream=stream)
+                pkv.paged_attention_decode(self.out[layer], self.q[layer], self.k[layer], self.v[layer],
+                                           self.tables, self.lens, cfg.scale, self.ws, stream=stream)
 
 
 def capture(fn):
@@ -258,8 +276,32 @@ def time_replays(graph, steps, world):
     return start.elapsed_time(end) / steps
 
 
+def time_replays_redraw(graph, wl, steps, world):
+    """Per-step device time of the graph, with an untimed batch re-draw before each step.
+
+    Returns (mean ms per step, total algorithmic bytes over the timed steps).
+    """
+    cfg = wl.cfg
+    total_ms, total_bytes = 0.0, 0
+    dist_barrier(world)
+    for _ in range(steps):
+        wl.redraw()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        graph.replay()
+        end.record()
+        torch.cuda.synchronize()
+        total_ms += start.elapsed_time(end)
+        lens = [int(c) for c in wl.layout.context_lens]
+        total_bytes += layer_bytes(cfg, lens, wl.layout.shares_prefix.tolist(), unique_prefix=True)["total"] * cfg.n_layers
+    dist_barrier(world)
+    return total_ms / steps, total_bytes
+
+
 def decode_kernel_duration_ms(wl, reps=5):
-    """Average duration of one paged_attention_decode launch, by CUDA events on its stream, cycling layers."""
+    """Average duration of one decode launch (with the fused append when the step uses it), by CUDA events on
+    its stream, cycling through the layers."""
     pkv, cfg = wl.pkv, wl.cfg
     stream = torch.cuda.current_stream()
     evs = []
@@ -267,8 +309,13 @@ def decode_kernel_duration_ms(wl, reps=5):
         for layer in range(cfg.n_layers):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            pkv.paged_attention_decode(wl.out[layer], wl.q[layer], wl.k[layer], wl.v[layer], wl.tables, wl.lens,
-                                       cfg.scale, wl.ws, stream=stream)
+            if wl.fused:  # rewriting this step's token is idempotent
+                pkv.paged_attention_decode_append(wl.out[layer], wl.q[layer], wl.k_new[layer], wl.v_new[layer],
+                                                  wl.k[layer], wl.v[layer], wl.slots, wl.tables, wl.lens,
+                                                  cfg.scale, wl.ws, stream=stream)
+            else:
+                pkv.paged_attention_decode(wl.out[layer], wl.q[layer], wl.k[layer], wl.v[layer], wl.tables,
+                                           wl.lens, cfg.scale, wl.ws, stream=stream)
             b.record(stream)
             evs.append((a, b))
     torch.cuda.synchronize()
@@ -335,6 +382,7 @@ def run_profile_step(args, cfg, device):
     """Only the step's graph replays (for ncu): no e2e, no per-kernel timing, no CPU baseline."""
     import paged_kv_cache_470_b200 as pkv
     wl = Workload(cfg, device)
+    wl.fused = not args.separate_append
     graph = capture(wl.step)
     for _ in range(args.warmup + args.steps):
         graph.replay()
@@ -354,6 +402,7 @@ def run_ours(args, world, rank, local):
     if args.profile_step:
         return run_profile_step(args, cfg, device)
     wl = Workload(cfg, device, rank)
+    wl.fused = not args.separate_append
     lens = [int(c) for c in wl.layout.context_lens]
     share = wl.layout.shares_prefix.tolist()
     lb_logical = layer_bytes(cfg, lens, share, unique_prefix=False)
@@ -364,16 +413,24 @@ def run_ours(args, world, rank, local):
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
+    redraw = cfg.redraw_fraction > 0
     with ClockSampler(device.index or 0) as clk:
-        ms = time_replays(graph, args.steps, world)
+        if redraw:
+            ms, timed_bytes = time_replays_redraw(graph, wl, args.steps, world)
+            step_bytes = timed_bytes // args.steps
+        else:
+            ms = time_replays(graph, args.steps, world)
     ms = dist_max(ms, world)
     status = pkv.read_status(wl.ws)
 
-    # the decode kernel alone, for the roofline
+    # the decode kernel alone, for the roofline (on the batch as it stands now)
+    lens = [int(c) for c in wl.layout.context_lens]
+    lb_unique = layer_bytes(cfg, lens, wl.layout.shares_prefix.tolist(), unique_prefix=True)
+    lb_logical = layer_bytes(cfg, lens, wl.layout.shares_prefix.tolist(), unique_prefix=False)
     kern_ms, n_launch = decode_kernel_duration_ms(wl)
     kern_ms = dist_max(kern_ms, world)
     peak, peak_kind = measured_peak()
-    kern_bytes = lb_unique["decode_kernel"]
+    kern_bytes = lb_unique["decode_kernel"] + (lb_unique["append"] if wl.fused else 0)
     achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
     traffic = profiled_traffic()
 
@@ -414,7 +471,9 @@ def run_ours(args, world, rank, local):
                    "algorithmic_bytes_per_step": step_bytes,
                    "l2": "inputs larger than L2: every step reads all layers' distinct caches "
                          f"({lb_unique['kv'] * cfg.n_layers / 1e9:.2f} GB of KV vs 126 MB L2)",
-                   "timing": "CUDA-graph replay of the whole step, CUDA events, max over ranks",
+                   "timing": "CUDA-graph replay of the whole step, CUDA events, max over ranks"
+                             + ("; 10% of the batch re-drawn through the block pool before each step (untimed)"
+                                if redraw else ""),
                    "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -423,8 +482,10 @@ def run_ours(args, world, rank, local):
                      "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)},
         "e2e": {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": "kv_cache_append + paged_attention_decode per layer, captured in a CUDA graph with the copies"},
-        "gpu_launches": (2 if pkv.get_option(pkv.KV_OPT_COMBINE) == 0 else 3) * cfg.n_layers * args.steps,
+                "api": ("paged_attention_decode_append" if wl.fused else "kv_cache_append + paged_attention_decode")
+                       + " per layer, captured in a CUDA graph with the copies"},
+        "gpu_launches": ((1 if wl.fused else 2) + (pkv.get_option(pkv.KV_OPT_COMBINE) == 1))
+                        * cfg.n_layers * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
         "cpu_baseline": cpu,
@@ -477,6 +538,8 @@ def main(argv=None):
     ap.add_argument("--reference-budget", type=float, default=120.0)
     ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling a smaller case)")
     ap.add_argument("--profile-step", action="store_true", help="only replay the step graph (for ncu)")
+    ap.add_argument("--separate-append", action="store_true",
+                    help="append with kv_cache_append, then paged_attention_decode (two launches per layer)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -161,6 +161,30 @@ KV_API kv_status paged_attention_read_status(const void *workspace, int32_t *sta
                                       int clear, kv_stream_t stream);
 
 /*
+ * Append fused into decode: the same result as kv_cache_append(k_new, v_new,
+ * k_cache, v_cache, slot_mapping, T = B, ...) followed by
+ * paged_attention_decode(...), in one kernel launch. k_new/v_new are
+ * [B][Hkv][D] bf16 (16-byte aligned), slot_mapping [B] int64 (device).
+ * Sequence b's new token must be its last cached token: slot_mapping[b] ==
+ * block_tables[b][(c-1)/16] * 16 + (c-1) % 16 with c = context_lens[b], and
+ * its block must not be read by any other sequence of the batch (true for
+ * blocks from kv_pool_append_slots). A negative slot appends nothing; any
+ * other slot is not written, KV_STATUS_BAD_SLOT is recorded in the workspace
+ * status word and that sequence's output is unspecified. ("Module 23:
+ * Serving", section 23.4: a block fills as its sequence grows.)
+ */
+KV_API kv_status paged_attention_decode_append(void *out, const void *q,
+                                               const void *k_new, const void *v_new,
+                                               void *k_cache, void *v_cache,
+                                               const int64_t *slot_mapping,
+                                               const int32_t *block_tables, int max_blocks_per_seq,
+                                               const int32_t *context_lens, int B,
+                                               int num_blocks, int Hq, int Hkv, int D,
+                                               float scale, int dtype,
+                                               void *workspace, size_t workspace_bytes,
+                                               kv_stream_t stream);
+
+/*
  * The same decode as paged_attention_decode, for callers that cannot allocate
  * device memory (for example a plugin inside a host program that owns every
  * device allocation, or code that must not trigger cudaMalloc's implicit

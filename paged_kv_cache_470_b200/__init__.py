@@ -35,6 +35,8 @@ _sig = {
     "paged_attention_workspace_init": (_I, [_P, _SZ, _P]),
     "paged_attention_decode": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P, _SZ,
                                     _P]),
+    "paged_attention_decode_append": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float,
+                                           _I, _P, _SZ, _P]),
     "paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
                                             _P]),
     "paged_attention_read_status": (_I, [_P, _P, _I, _P]),
@@ -128,6 +130,26 @@ def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Te
     _check("paged_attention_decode", _lib.paged_attention_decode(
         _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
         _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), KV_DTYPE_BF16,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
+    return out
+
+
+def paged_attention_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                                  k_cache: torch.Tensor, v_cache: torch.Tensor, slot_mapping: torch.Tensor,
+                                  block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                                  workspace: torch.Tensor, stream=None) -> torch.Tensor:
+    """kv_cache_append of this step's token (the last of each sequence) fused into the decode."""
+    B, Hq, D = q.shape
+    num_blocks, _, Hkv, Dk = k_cache.shape
+    if Dk != D or tuple(out.shape) != (B, Hq, D) or tuple(k_new.shape) != (B, Hkv, D):
+        raise ValueError("shape mismatch")
+    _check("paged_attention_decode_append", _lib.paged_attention_decode_append(
+        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
+        _dev(k_new, "k_new", torch.bfloat16), _dev(v_new, "v_new", torch.bfloat16),
+        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(slot_mapping, "slot_mapping", torch.int64),
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), KV_DTYPE_BF16,
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))

@@ -103,6 +103,12 @@ struct DecodeArgs {
     int min_chunk;
     int fused;
     float scale_log2;    // scale * log2(e)
+    // fused append (append != 0): this step's token of sequence b is k_new/v_new[b],
+    // at slot slots[b], which must be position context_lens[b] - 1 of sequence b
+    int append;
+    const uint4 *k_new, *v_new;   // [B][Hkv][D] bf16, as 16-byte chunks
+    uint4 *k_cache, *v_cache;     // [num_blocks][16][Hkv][D] bf16, as 16-byte chunks
+    const int64_t *slots;         // [B]
 };
 
 // misc ints in shared memory
@@ -190,6 +196,14 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 +
 
 // exp2(x - m) for merging states whose maxima may both be -inf (empty states).
 __device__ __forceinline__ float rescale(float x, float m) { return m == -INFINITY ? 0.f : exp2f(x - m); }
+
+// The new token of one kv head of an item, for the fused append: lane l < D/8
+// holds 16-byte chunk l of the K row, lane D/8 <= l < D/4 chunk l - D/8 of the
+// V row. `slot` is where it goes (-1: nothing to append, or a bad slot).
+struct AppendRow {
+    uint4 chunk;
+    long long slot;
+};
 
 // Where an item's outputs go.
 struct ItemOut {
@@ -702,6 +716,64 @@ __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int ite
     }
 }
 
+// Load the new token row of kv head `j` of sequence b (fused append). The slot
+// must be the sequence's last position; otherwise nothing is appended for it and
+// KV_STATUS_BAD_SLOT is raised (by the first kv head's warp).
+template <int D>
+__device__ __forceinline__ AppendRow load_append_row(const DecodeArgs &a, const Cursor &cur, int j, bool report)
+{
+    AppendRow r;
+    r.slot = -1;
+    r.chunk = make_uint4(0u, 0u, 0u, 0u);
+    if (!a.append || cur.ctx == 0)
+        return r;
+    const int lane = threadIdx.x & 31;
+    const long long slot = __ldg(a.slots + cur.b);
+    if (slot < 0)
+        return r;
+    const int last = cur.ctx - 1;
+    const int blk = __ldg(a.block_tables + static_cast<size_t>(cur.b) * a.W + last / kBlockTokens);
+    const long long expect = static_cast<long long>(blk) * kBlockTokens + last % kBlockTokens;
+    if (slot != expect || blk < 0 || blk >= a.num_blocks) {
+        if (report && lane == 0)
+            atomicOr(a.status, KV_STATUS_BAD_SLOT);
+        return r;
+    }
+    r.slot = slot;
+    constexpr int C = D / 8;  // 16-byte chunks per head row
+    const size_t row = (static_cast<size_t>(cur.b) * a.Hkv + j) * C;
+    if (lane < C)
+        r.chunk = __ldg(a.k_new + row + lane);
+    else if (lane < 2 * C)
+        r.chunk = __ldg(a.v_new + row + lane - C);
+    return r;
+}
+
+// Put the new token into this warp's tiles of the stage (row (c-1) % 16) and,
+// if `write`, into the cache in global memory.
+template <int D>
+__device__ __forceinline__ void apply_append_row(const DecodeArgs &a, const AppendRow &r, int j, int row,
+                                                 uint32_t kbase, uint32_t vbase, int tile_stride, bool write)
+{
+    constexpr int C = D / 8;
+    const int lane = threadIdx.x & 31;
+    if (r.slot >= 0 && lane < 2 * C) {
+        const bool is_v = lane >= C;
+        const int ch = is_v ? lane - C : lane;
+        const uint32_t addr = (is_v ? vbase : kbase) + (ch >> 3) * tile_stride + swz(row, ch & 7);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r.chunk.x), "r"(r.chunk.y),
+                     "r"(r.chunk.z), "r"(r.chunk.w)
+                     : "memory");
+        if (write) {
+            uint4 *dst = (is_v ? a.v_cache : a.k_cache) + (static_cast<size_t>(r.slot) * a.Hkv + j) * C + ch;
+            *dst = r.chunk;
+        }
+        // the stage is refilled by TMA later: order these writes before that
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncwarp();
+}
+
 // Outputs of empty sequences are zero; also flag out-of-range lengths. Run by CTA 0.
 template <int D>
 __device__ __forceinline__ void zero_empty_outputs(const DecodeArgs &a, int tid, int nthreads)
@@ -901,6 +973,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     st.prefetch_q(a, item_out(a, cur0, hh));  // q is never written by this library: no wait needed
     grid_dependency_wait();
     grid_launch_dependents();
+    // the new token rows (fused append) are loaded after the wait: the caller may
+    // have produced them in the previous kernel
+    AppendRow ar_next = load_append_row<D>(a, cur0, (cur0.k / a.hchunks) * a.hg + hh,
+                                           hh == 0 && (cur0.k % a.hchunks) == 0);
     if (blockIdx.x == 0)
         zero_empty_outputs<D>(a, tid, kConsumerThreads);
     Cursor cur = cur0;
@@ -930,10 +1006,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             named_barrier(1, kConsumerThreads);
         }
         st.begin_item(a, o, q_s);
+        const AppendRow ar = ar_next;
+        const int j_head = hg * a.hg + hh;
         if (u + run < count) {
             Cursor next = cur;
             cursor_next_item(a, next);
             st.prefetch_q(a, item_out(a, next, hh));
+            ar_next = load_append_row<D>(a, next, (next.k / a.hchunks) * a.hg + hh,
+                                         hh == 0 && (next.k % a.hchunks) == 0);
         }
         for (int i = ((stream - u) % NS + NS) % NS; i < run; i += NS) {
             const int uu = u + i;
@@ -947,6 +1027,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             const uint32_t kb = ring + s * a.stage_bytes + hh * kHeadTileBytes;
             const int valid = min(kBlockTokens, cur.ctx - (cur.off + i) * kBlockTokens);
+            if (cur.off + i == cur.n - 1)  // the block holding this step's token
+                apply_append_row<D>(a, ar, j_head, valid - 1, kb, kb + G::kTiles * a.tile_stride, a.tile_stride,
+                                    hc == 0);
             st.unit(kb, kb + G::kTiles * a.tile_stride, a.tile_stride, valid, a.scale_log2, q_s, p_s);
             __syncwarp();
             if (lane == 0)
@@ -1217,11 +1300,13 @@ extern "C" kv_status paged_attention_workspace_init(void *workspace, size_t work
                : KV_ERR_CUDA;
 }
 
-extern "C" kv_status paged_attention_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
-                                            const int32_t *block_tables, int max_blocks_per_seq,
-                                            const int32_t *context_lens, int B, int num_blocks, int Hq, int Hkv,
-                                            int D, float scale, int dtype, void *workspace,
-                                            size_t workspace_bytes, kv_stream_t stream)
+// Shared by paged_attention_decode (k_new == nullptr) and the fused
+// append + decode entry point.
+static kv_status decode_impl(void *out, const void *q, const void *k_new, const void *v_new, const void *k_cache,
+                             const void *v_cache, const int64_t *slot_mapping, const int32_t *block_tables,
+                             int max_blocks_per_seq, const int32_t *context_lens, int B, int num_blocks, int Hq,
+                             int Hkv, int D, float scale, int dtype, void *workspace, size_t workspace_bytes,
+                             kv_stream_t stream)
 {
     if (dtype != KV_DTYPE_BF16 || B < 0 || max_blocks_per_seq < 1 || num_blocks < 1 || Hq < 1 || Hkv < 1 ||
         Hq % Hkv != 0 || (D != 64 && D != 128))
@@ -1319,6 +1404,12 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
     const int combine_mode = g_opt_combine.load();
     a.fused = combine_mode == 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;
+    a.append = k_new != nullptr ? 1 : 0;
+    a.k_new = static_cast<const uint4 *>(k_new);
+    a.v_new = static_cast<const uint4 *>(v_new);
+    a.k_cache = static_cast<uint4 *>(const_cast<void *>(k_cache));
+    a.v_cache = static_cast<uint4 *>(const_cast<void *>(v_cache));
+    a.slots = slot_mapping;
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
@@ -1349,6 +1440,30 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
             return KV_ERR_CUDA;
     }
     return KV_OK;
+}
+
+extern "C" kv_status paged_attention_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                            const int32_t *block_tables, int max_blocks_per_seq,
+                                            const int32_t *context_lens, int B, int num_blocks, int Hq, int Hkv,
+                                            int D, float scale, int dtype, void *workspace,
+                                            size_t workspace_bytes, kv_stream_t stream)
+{
+    return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, block_tables, max_blocks_per_seq,
+                       context_lens, B, num_blocks, Hq, Hkv, D, scale, dtype, workspace, workspace_bytes, stream);
+}
+
+extern "C" kv_status paged_attention_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
+                                                   void *k_cache, void *v_cache, const int64_t *slot_mapping,
+                                                   const int32_t *block_tables, int max_blocks_per_seq,
+                                                   const int32_t *context_lens, int B, int num_blocks, int Hq,
+                                                   int Hkv, int D, float scale, int dtype, void *workspace,
+                                                   size_t workspace_bytes, kv_stream_t stream)
+{
+    if (!k_new || !v_new || !slot_mapping || misaligned(k_new, 16) || misaligned(v_new, 16) ||
+        misaligned(slot_mapping, 8))
+        return KV_ERR_ARG;
+    return decode_impl(out, q, k_new, v_new, k_cache, v_cache, slot_mapping, block_tables, max_blocks_per_seq,
+                       context_lens, B, num_blocks, Hq, Hkv, D, scale, dtype, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -17,7 +17,7 @@ class Case:
 
     def __init__(self, cfg, device, n_layers=1, lens=None, seed=None, layout=None):
         self.cfg = cfg
-        self.layout = layout or workloads.draw_layout(cfg, context_lens=lens, seed=seed)
+        self.layout = layout if layout is not None else workloads.draw_layout(cfg, context_lens=lens, seed=seed)
         gen = workloads.device_generator(cfg.seed if seed is None else seed, device)
         self.k, self.v = [], []
         for _ in range(n_layers):
@@ -46,12 +46,18 @@ def oracle_step(oracle_mod, case, layer, host=None):
     return k2, v2, out
 
 
-def gpu_step(pkv, case, layer, workspace, out=None):
+def gpu_step(pkv, case, layer, workspace, out=None, fused=False):
+    """Append this step's token and attend: two kernels, or one with the append fused in."""
     if out is None:
         out = torch.empty_like(case.q[layer])
-    pkv.kv_cache_append(case.k_new[layer], case.v_new[layer], case.k[layer], case.v[layer], case.slots)
-    pkv.paged_attention_decode(out, case.q[layer], case.k[layer], case.v[layer], case.tables, case.lens,
-                               case.cfg.scale, workspace)
+    if fused:
+        pkv.paged_attention_decode_append(out, case.q[layer], case.k_new[layer], case.v_new[layer], case.k[layer],
+                                          case.v[layer], case.slots, case.tables, case.lens, case.cfg.scale,
+                                          workspace)
+    else:
+        pkv.kv_cache_append(case.k_new[layer], case.v_new[layer], case.k[layer], case.v[layer], case.slots)
+        pkv.paged_attention_decode(out, case.q[layer], case.k[layer], case.v[layer], case.tables, case.lens,
+                                   case.cfg.scale, workspace)
     return out
 
 

@@ -24,30 +24,33 @@ def _default_options(pkv):
         pkv.set_option(key, 0)
 
 
-def run_and_check(pkv, oracle_mod, case, layers=None, what=""):
+def run_and_check(pkv, oracle_mod, case, layers=None, what="", fused=None):
+    """Every listed layer against the oracle; `fused` None alternates separate and fused append."""
     cfg = case.cfg
     ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
-    for layer in (range(case.n_layers) if layers is None else layers):
+    for n, layer in enumerate(range(case.n_layers) if layers is None else layers):
         host = case.host_inputs(layer)
-        out = gpu_step(pkv, case, layer, ws)
+        f = (n % 2 == 1) if fused is None else fused
+        out = gpu_step(pkv, case, layer, ws, fused=f)
         torch.cuda.synchronize()
         k2, v2, ref = oracle_step(oracle_mod, case, layer, host)
         assert np.array_equal(bf16_bits_np(case.k[layer]), k2), f"{what} layer {layer}: K append not bit-exact"
         assert np.array_equal(bf16_bits_np(case.v[layer]), v2), f"{what} layer {layer}: V append not bit-exact"
-        compare(out, ref, f"{what} layer {layer}")
+        compare(out, ref, f"{what} layer {layer}{' (fused append)' if f else ''}")
     assert pkv.read_status(ws) == 0
 
 
 # ---------------------------------------------------------------------------
 # the tiny workload, every path and combine mode
 # ---------------------------------------------------------------------------
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("path", sorted(PATHS))
 @pytest.mark.parametrize("combine", [0, 1])
-def test_tiny_workload(pkv, oracle_mod, cuda_device, path, combine):
+def test_tiny_workload(pkv, oracle_mod, cuda_device, path, combine, fused):
     pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
     pkv.set_option(pkv.KV_OPT_COMBINE, combine)
     case = Case(workloads.CONFIGS[1], cuda_device)
-    run_and_check(pkv, oracle_mod, case, what=f"tiny/{path}/combine{combine}")
+    run_and_check(pkv, oracle_mod, case, what=f"tiny/{path}/combine{combine}", fused=fused)
 
 
 @pytest.mark.parametrize("path", sorted(PATHS))
@@ -57,8 +60,8 @@ def test_ragged_lengths_and_head_groups(pkv, oracle_mod, cuda_device, path, D, H
     """Lengths at and around block edges, the table's maximum, 1 and 0; groups 1..16."""
     pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
     lens = [1, 15, 16, 17, 31, 32, 33, 255, 256, 0, 100, 2]
-    cfg = workloads.small_config(1, Hq=Hq, Hkv=Hkv, D=D, batch=len(lens), pool_blocks=0)
-    case = Case(cfg, cuda_device, lens=lens)
+    cfg = workloads.small_config(1, Hq=Hq, Hkv=Hkv, D=D, batch=len(lens), pool_blocks=0, n_layers=2)
+    case = Case(cfg, cuda_device, lens=lens, n_layers=2)
     run_and_check(pkv, oracle_mod, case, what=f"ragged D{D} {Hq}/{Hkv} {path}")
 
 
@@ -202,3 +205,39 @@ def test_full_size_llama2_7b_mha(pkv, oracle_mod, cuda_device):
 
 def test_full_size_70b_mix_with_shared_prefix(pkv, oracle_mod, cuda_device):
     _full_size(pkv, oracle_mod, cuda_device, 5, 2)
+
+
+def test_full_size_70b_mix_after_redraws(pkv, oracle_mod, cuda_device):
+    """The 70B-style mix after two steps of re-drawing 10% of the batch through the block pool."""
+    from paged_kv_cache_470_b200.batch import ContinuousBatch
+    cfg = workloads.CONFIGS[5]
+    cb = ContinuousBatch(cfg, int(workloads.draw_layout(cfg).num_blocks * 1.25))
+    cb.redraw()
+    cb.redraw()
+    cb.check()
+    case = Case(cfg, cuda_device, n_layers=2, layout=cb)
+    run_and_check(pkv, oracle_mod, case, what="70B mix after re-draws")
+
+
+def test_fused_append_rejects_a_slot_that_is_not_the_last_token(pkv, oracle_mod, cuda_device):
+    cfg = workloads.small_config(1, batch=4)
+    case = Case(cfg, cuda_device, lens=[40, 17, 1, 33])
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    bad = case.slots.clone()
+    bad[1] -= 1                              # one row before sequence 1's last token
+    before_k, before_v = case.k[0].clone(), case.v[0].clone()
+    out = torch.empty_like(case.q[0])
+    pkv.paged_attention_decode_append(out, case.q[0], case.k_new[0], case.v_new[0], case.k[0], case.v[0], bad,
+                                      case.tables, case.lens, cfg.scale, ws)
+    assert pkv.read_status(ws) & pkv.KV_STATUS_BAD_SLOT
+    # sequences 0, 2, 3 were appended exactly; sequence 1's rows are untouched
+    host_k, host_v = before_k.cpu(), before_v.cpu()
+    slots = bad.clone()
+    slots[1] = -1
+    ek, ev = oracle_mod.kv_cache_append(host_k, host_v, case.k_new[0].cpu(), case.v_new[0].cpu(), slots.cpu().numpy())
+    assert np.array_equal(bf16_bits_np(case.k[0]), ek) and np.array_equal(bf16_bits_np(case.v[0]), ev)
+    # a negative slot appends nothing and is not an error
+    slots_none = torch.full_like(case.slots, -1)
+    pkv.paged_attention_decode_append(out, case.q[0], case.k_new[0], case.v_new[0], case.k[0], case.v[0],
+                                      slots_none, case.tables, case.lens, cfg.scale, ws)
+    assert pkv.read_status(ws) == 0

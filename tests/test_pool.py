@@ -197,3 +197,28 @@ def test_reservation_admits_four_paging_admits_eight(pkv):
             done[b] = int(lens[b]) >= final[b]
     assert lens.tolist() == final
     assert 96 - p.num_free() == sum(-(-c // 16) for c in final)
+
+
+def test_continuous_batch_redraw_keeps_refcounts(pkv):
+    """The 70B-style mix: half the sequences share a 64-block prefix; 10% are re-drawn each step."""
+    from paged_kv_cache_470_b200 import workloads
+    from paged_kv_cache_470_b200.batch import ContinuousBatch
+    cfg = workloads.small_config(5, batch=40)
+    layout = workloads.draw_layout(cfg)
+    cb = ContinuousBatch(cfg, int(layout.num_blocks * 1.3))
+    cb.check()
+    assert len(cb.prefix) == 64
+    assert all(cb.pool.refcount(i) == 1 + int(cb.shares.sum()) for i in cb.prefix)
+    for _ in range(10):
+        rows = cb.redraw()
+        assert len(rows) == 4
+        cb.check()
+        for b in range(cfg.batch):
+            c = int(cb.context_lens[b])
+            assert 1 <= c <= cfg.W * 16
+            if cb.shares[b]:
+                assert c >= 1025 and cb.block_tables[b, :64].tolist() == cb.prefix
+        slots = cb.slot_mapping()
+        assert len(set(slots.tolist())) == cfg.batch        # every new token has its own slot
+        for b in range(cfg.batch):                          # ... in a block no other sequence uses
+            assert cb.pool.refcount(int(slots[b]) // 16) == 1
