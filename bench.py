@@ -399,6 +399,10 @@ def run_ours(args, world, rank, local):
     device = torch.device("cuda", local if world > 1 else 0)
     if args.compute:
         pkv.set_option(pkv.KV_OPT_COMPUTE, {"tensor": 1, "cuda": 2}[args.compute])
+    if args.grid:
+        pkv.set_option(pkv.KV_OPT_GRID, args.grid)
+    if args.combine_kernel:
+        pkv.set_option(pkv.KV_OPT_COMBINE, 1)
     if args.profile_step:
         return run_profile_step(args, cfg, device)
     wl = Workload(cfg, device, rank)
@@ -538,6 +542,8 @@ def main(argv=None):
     ap.add_argument("--reference-budget", type=float, default=120.0)
     ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling a smaller case)")
     ap.add_argument("--profile-step", action="store_true", help="only replay the step graph (for ncu)")
+    ap.add_argument("--grid", type=int, default=0, help="decode CTAs per launch (0: one per SM)")
+    ap.add_argument("--combine-kernel", action="store_true", help="split-K merge in a separate kernel")
     ap.add_argument("--separate-append", action="store_true",
                     help="append with kv_cache_append, then paged_attention_decode (two launches per layer)")
     args = ap.parse_args(argv)

@@ -51,7 +51,9 @@ namespace pkv {
 constexpr int kConsumerWarps = 8;
 constexpr int kConsumerThreads = kConsumerWarps * 32;
 constexpr int kProducerWarp = kConsumerWarps;
-constexpr int kThreads = kConsumerThreads + 32;
+constexpr int kHelperWarp = kConsumerWarps + 1;   // counts finished split pieces off the consumers' path
+constexpr int kThreads = kConsumerThreads + 64;
+constexpr int kPieceQueue = 4;                    // consumer -> helper queue of finished split pieces
 constexpr int kGroupMax = 8;            // query heads per kv head per work item
 constexpr int kMaxHG = 4;               // kv heads per work unit
 constexpr int kHeadTileBytes = 2048;    // one kv head: 16 rows x 64 bf16, 128B-swizzled
@@ -61,6 +63,7 @@ constexpr int kStatusBytes = 256;
 constexpr unsigned kFull = 0xffffffffu;
 
 enum ComputePath { kPathMma = 1, kPathSimt = 2 };
+constexpr int kMergeBatch = 4;          // split-K pieces whose loads are in flight together
 
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
@@ -79,8 +82,9 @@ struct Geo {
     static constexpr int kScratchBytes = cmax(kMergeBytes, kQBytes + kPBytes);
     static constexpr int kOffScratch = kRingBytes;
     static constexpr int kOffBar = kOffScratch + kScratchBytes;
-    static constexpr int kOffMisc = kOffBar + 2 * kMaxStages * 8;
-    static constexpr int kMiscInts = 16;
+    static constexpr int kOffQBar = kOffBar + 2 * kMaxStages * 8;    // piece queue: full[4], empty[4]
+    static constexpr int kOffMisc = kOffQBar + 2 * kPieceQueue * 8;
+    static constexpr int kMiscInts = 48;
     static constexpr int kSmemBytes = kOffMisc + kMiscInts * 4 + 1024;  // + room to align the base
 };
 
@@ -112,7 +116,16 @@ struct DecodeArgs {
 };
 
 // misc ints in shared memory
-enum { kMiscAbort = 0, kMiscLocB = 1, kMiscLocR = 2, kMiscLast = 3, kMiscZero = 4, kMiscWarpSums = 6 };
+enum {
+    kMiscAbort = 0,
+    kMiscLocB = 1,
+    kMiscLocR = 2,
+    kMiscSolo = 3,      // this piece's item has all its other pieces finished
+    kMiscZero = 4,
+    kMiscLast = 5,      // the CTA's final piece completed its item: merge it
+    kMiscWarpSums = 6,  // 10 ints
+    kMiscQueue = 16,    // kPieceQueue descriptors of 5 ints: item, first cta, last cta, b, k
+};
 
 __device__ __forceinline__ int clamp_ctx(int c, int W)
 {
@@ -193,6 +206,25 @@ __device__ __forceinline__ void sts128_zero(uint32_t addr)
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside one head's 128B-swizzled tile.
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+// Split-K counters. A finished piece releases its partial with a release
+// atomic (the writes of the other threads are ordered before it by a bar.sync);
+// a CTA that observes a count (relaxed load or the atomic's result) and then
+// merges issues an acquire fence first. Neither the relaxed load nor the
+// release atomic makes the issuing thread wait for the round trip.
+__device__ __forceinline__ int ld_relaxed_gpu(const int32_t *p)
+{
+    int v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ int atom_add_release_gpu(int32_t *p, int v)
+{
+    int prev;
+    asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(prev) : "l"(p), "r"(v) : "memory");
+    return prev;
+}
+__device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 // exp2(x - m) for merging states whose maxima may both be -inf (empty states).
 __device__ __forceinline__ float rescale(float x, float m) { return m == -INFINITY ? 0.f : exp2f(x - m); }
@@ -383,6 +415,102 @@ struct Consumer<D, kPathMma, NH> {
         l1 = l1 * a1 + pl1 * b1;
         m0 = M0;
         m1 = M1;
+    }
+
+    // All other pieces of this split item are finished: merge them with this
+    // warp's state, in the same order and arithmetic as merge_pieces_global, so
+    // the result does not depend on which CTA merges.
+    __device__ __forceinline__ void merge_solo(const DecodeArgs &a, const ItemOut &o, int item, int first_cta,
+                                               int last_cta)
+    {
+        const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+        const int self = static_cast<int>(blockIdx.x);
+        const size_t hbase = static_cast<size_t>(o.hh) * kGroupMax;
+        const int n0 = 2 * c, n1 = 2 * c + 1;
+        float M0 = -INFINITY, M1 = -INFINITY, L0 = 0.f, L1 = 0.f;
+        float O[kMt][4];
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt)
+            O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f;
+        for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
+            float mv0[kMergeBatch], mv1[kMergeBatch], lv0[kMergeBatch], lv1[kMergeBatch];
+#pragma unroll
+            for (int j = 0; j < kMergeBatch; ++j) {
+                const int cc = c0 + j;
+                if (cc > last_cta) {
+                    mv0[j] = mv1[j] = -INFINITY;
+                    lv0[j] = lv1[j] = 0.f;
+                } else if (cc == self) {
+                    mv0[j] = m0;
+                    mv1[j] = m1;
+                    lv0[j] = l0;
+                    lv1[j] = l1;
+                } else {
+                    const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase;
+                    mv0[j] = __ldcg(a.part_ml + (h + n0) * 2);
+                    lv0[j] = __ldcg(a.part_ml + (h + n0) * 2 + 1);
+                    mv1[j] = __ldcg(a.part_ml + (h + n1) * 2);
+                    lv1[j] = __ldcg(a.part_ml + (h + n1) * 2 + 1);
+                }
+            }
+            float Mb0 = M0, Mb1 = M1;
+#pragma unroll
+            for (int j = 0; j < kMergeBatch; ++j) {
+                Mb0 = fmaxf(Mb0, mv0[j]);
+                Mb1 = fmaxf(Mb1, mv1[j]);
+            }
+            const float sc0 = rescale(M0, Mb0), sc1 = rescale(M1, Mb1);
+            L0 *= sc0;
+            L1 *= sc1;
+#pragma unroll
+            for (int mt = 0; mt < kMt; ++mt) {
+                O[mt][0] *= sc0;
+                O[mt][1] *= sc1;
+                O[mt][2] *= sc0;
+                O[mt][3] *= sc1;
+            }
+#pragma unroll
+            for (int j = 0; j < kMergeBatch; ++j) {
+                const int cc = c0 + j;
+                const float w0 = rescale(mv0[j], Mb0), w1 = rescale(mv1[j], Mb1);
+                L0 = fmaf(w0, lv0[j], L0);
+                L1 = fmaf(w1, lv1[j], L1);
+                if (cc > last_cta)
+                    continue;  // a padding piece adds exact zeros
+                if (cc == self) {
+#pragma unroll
+                    for (int mt = 0; mt < kMt; ++mt) {
+                        O[mt][0] = fmaf(w0, acc[mt][0], O[mt][0]);
+                        O[mt][1] = fmaf(w1, acc[mt][1], O[mt][1]);
+                        O[mt][2] = fmaf(w0, acc[mt][2], O[mt][2]);
+                        O[mt][3] = fmaf(w1, acc[mt][3], O[mt][3]);
+                    }
+                } else {
+                    const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase;
+                    const float *p0 = a.part_acc + (h + n0) * D;
+                    const float *p1 = a.part_acc + (h + n1) * D;
+#pragma unroll
+                    for (int mt = 0; mt < kMt; ++mt) {
+                        const int d = mt * 16 + r;
+                        O[mt][0] = fmaf(w0, __ldcg(p0 + d), O[mt][0]);
+                        O[mt][1] = fmaf(w1, __ldcg(p1 + d), O[mt][1]);
+                        O[mt][2] = fmaf(w0, __ldcg(p0 + d + 8), O[mt][2]);
+                        O[mt][3] = fmaf(w1, __ldcg(p1 + d + 8), O[mt][3]);
+                    }
+                }
+            }
+            M0 = Mb0;
+            M1 = Mb1;
+        }
+#pragma unroll
+        for (int mt = 0; mt < kMt; ++mt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc[mt][i] = O[mt][i];
+        m0 = M0;
+        m1 = M1;
+        l0 = L0;
+        l1 = L1;
     }
 
     __device__ __forceinline__ void store_final(const DecodeArgs &a, const ItemOut &o) const
@@ -587,6 +715,74 @@ struct Consumer<D, kPathSimt, NH> {
         }
     }
 
+    // As Consumer<D, kPathMma>::merge_solo: same order and arithmetic as merge_pieces_global.
+    __device__ __forceinline__ void merge_solo(const DecodeArgs &a, const ItemOut &o, int item, int first_cta,
+                                               int last_cta)
+    {
+        const int lane = threadIdx.x & 31;
+        const int self = static_cast<int>(blockIdx.x);
+        const size_t hbase = static_cast<size_t>(o.hh) * kGroupMax;
+#pragma unroll
+        for (int n = 0; n < NH; ++n) {
+            float M = -INFINITY, L = 0.f;
+            float O[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                O[e] = 0.f;
+            for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
+                float mv[kMergeBatch], lv[kMergeBatch];
+#pragma unroll
+                for (int j = 0; j < kMergeBatch; ++j) {
+                    const int cc = c0 + j;
+                    if (cc > last_cta) {
+                        mv[j] = -INFINITY;
+                        lv[j] = 0.f;
+                    } else if (cc == self) {
+                        mv[j] = m[n];
+                        lv[j] = l[n];
+                    } else {
+                        const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase + n;
+                        mv[j] = __ldcg(a.part_ml + h * 2);
+                        lv[j] = __ldcg(a.part_ml + h * 2 + 1);
+                    }
+                }
+                float Mb = M;
+#pragma unroll
+                for (int j = 0; j < kMergeBatch; ++j)
+                    Mb = fmaxf(Mb, mv[j]);
+                const float sc = rescale(M, Mb);
+                L *= sc;
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    O[e] *= sc;
+#pragma unroll
+                for (int j = 0; j < kMergeBatch; ++j) {
+                    const int cc = c0 + j;
+                    const float w = rescale(mv[j], Mb);
+                    L = fmaf(w, lv[j], L);
+                    if (cc > last_cta)
+                        continue;
+                    if (cc == self) {
+#pragma unroll
+                        for (int e = 0; e < E; ++e)
+                            O[e] = fmaf(w, acc[n][e], O[e]);
+                    } else {
+                        const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase + n;
+#pragma unroll
+                        for (int e = 0; e < E; ++e)
+                            O[e] = fmaf(w, __ldcg(a.part_acc + h * D + lane * E + e), O[e]);
+                    }
+                }
+                M = Mb;
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e)
+                acc[n][e] = O[e];
+            m[n] = M;
+            l[n] = L;
+        }
+    }
+
     __device__ __forceinline__ void store_final(const DecodeArgs &a, const ItemOut &o) const
     {
         const int lane = threadIdx.x & 31;
@@ -627,8 +823,6 @@ struct Consumer<D, kPathSimt, NH> {
 // thread merges two groups of four output columns at a time, and all loads
 // for up to four pieces are issued before any is used, so a merge costs
 // about one memory round trip per four pieces.
-constexpr int kMergeBatch = 4;
-
 template <int D>
 __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int item, int first_cta, int last_cta,
                                                     int b, int k, int tid, int nthreads)
@@ -819,6 +1013,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     uint64_t *empty = full + G::kMaxStages;
     volatile int *misc = reinterpret_cast<volatile int *>(base + G::kOffMisc);
     float *scratch = reinterpret_cast<float *>(base + G::kOffScratch);
+    uint64_t *qbar = reinterpret_cast<uint64_t *>(base + G::kOffQBar);  // [0,4): full, [4,8): empty
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int S = a.stages;
@@ -828,6 +1023,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], a.hg);  // the HG warps of the consuming stream
         }
+        for (int q = 0; q < 2 * kPieceQueue; ++q)
+            mbar_init(qbar + q, 1);
         mbar_fence_init();
         misc[kMiscAbort] = 0;
         misc[kMiscLocB] = -1;
@@ -963,6 +1160,43 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         return;
     }
 
+    if (warp == kHelperWarp) {
+        // ------------- helper: count finished split pieces in -------------
+        // For each split piece the consumers finished (other than their last),
+        // release its partial and count it in; if that completes the item, merge
+        // the item here. Waiting for the release is this warp's job, not theirs.
+        grid_dependency_wait();
+        grid_launch_dependents();
+        if (!a.fused)
+            return;
+        for (int k = 0;; ++k) {
+            const int q = k % kPieceQueue;
+            if (!mbar_wait_bounded(qbar + q, (k / kPieceQueue) & 1, abort_flag))
+                break;
+            const volatile int *desc = misc + kMiscQueue + 5 * q;
+            const int item = desc[0], first_cta = desc[1], last_cta = desc[2], b = desc[3], kk = desc[4];
+            if (item < 0)
+                break;
+            int last = 0;
+            if (lane == 0) {
+                last = atom_add_release_gpu(a.counters + item, 1) == last_cta - first_cta;
+                if (last)
+                    fence_acquire_gpu();
+            }
+            last = __shfl_sync(kFull, last, 0);
+            if (last) {
+                merge_pieces_global<D>(a, item, first_cta, last_cta, b, kk, lane, 32);
+                __syncwarp();
+                if (lane == 0)
+                    a.counters[item] = 0;
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(qbar + kPieceQueue + q);
+        }
+        return;
+    }
+
     // -------------------- consumers: warps 0..7 --------------------
     const int hh = warp % a.hg;          // kv head within the group
     const int stream = warp / a.hg;      // which units: u % streams == stream
@@ -981,6 +1215,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         zero_empty_outputs<D>(a, tid, kConsumerThreads);
     Cursor cur = cur0;
     int u = 0;
+    int pushed = 0;  // split pieces handed to the helper (thread 0's count)
     while (u < count) {
         const int run = min(cur.n - cur.off, count - u);
         const int item = cur.b * a.items_per_seq + cur.k;
@@ -990,6 +1225,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int first_cta = item_start / chunk;
         const int last_cta = (item_start + cur.n - 1) / chunk;
         const bool single = first_cta == last_cta;
+        // pieces of this item already finished elsewhere: read by thread 0 when it
+        // starts its last unit of the piece, used at the epilogue
+        int seen = -1;
 
         if (PATH == kPathSimt) {
             // this item's query rows as fp32 in shared memory (heads >= gc are zero)
@@ -1025,6 +1263,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 }
                 break;
             }
+            if (tid == 0 && !single && a.fused && i + NS >= run)
+                seen = ld_relaxed_gpu(a.counters + item);
             const uint32_t kb = ring + s * a.stage_bytes + hh * kHeadTileBytes;
             const int valid = min(kBlockTokens, cur.ctx - (cur.off + i) * kBlockTokens);
             if (cur.off + i == cur.n - 1)  // the block holding this step's token
@@ -1036,9 +1276,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 mbar_arrive(&empty[s]);
         }
         st.finish();
+        const bool final_piece = u + run == count;
+        if (tid == 0) {
+            bool solo_now = false;
+            if (!single && a.fused) {
+                solo_now = seen == last_cta - first_cta;
+                if (solo_now)
+                    fence_acquire_gpu();  // the other pieces' partials, before anyone reads them
+            }
+            misc[kMiscSolo] = solo_now ? 1 : 0;
+        }
 
         // ---- merge the streams pairwise: stream s + step hands over to stream s ----
-        if (PATH == kPathSimt)
+        if (PATH == kPathSimt || NS == 1)
             named_barrier(1, kConsumerThreads);  // the scratch also holds q_s / p_s
         for (int step = 1; step < NS; step <<= 1) {
             const bool giver = (stream % (2 * step)) == step;
@@ -1053,32 +1303,73 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             named_barrier(1, kConsumerThreads);
         }
 
+        // Split items: if every other piece was already done when this one started,
+        // this CTA merges them now (no partial, no counter traffic). Otherwise it
+        // stores its partial and counts itself in; the CTA that completes the count
+        // merges from global memory -- checked at that CTA's next epilogue.
+        const bool solo = misc[kMiscSolo] != 0;
         if (stream == 0) {
-            if (single)
+            if (single) {
                 st.store_final(a, o);
-            else
+            } else if (solo) {
+                st.merge_solo(a, o, item, first_cta, last_cta);
+                st.store_final(a, o);
+            } else {
                 st.store_partial(a, o);
-        }
-        if (!single && a.fused) {
-            if (stream == 0)
-                __threadfence();  // this warp's partial is visible before the counter moves
-            named_barrier(1, kConsumerThreads);
-            if (tid == 0) {
-                const int prev = atomicAdd(a.counters + item, 1);
-                misc[kMiscLast] = (prev == last_cta - first_cta) ? 1 : 0;
-            }
-            named_barrier(1, kConsumerThreads);
-            if (misc[kMiscLast]) {
-                __threadfence();
-                merge_pieces_global<D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads);
-                if (tid == 0)
-                    a.counters[item] = 0;
             }
         }
-        named_barrier(1, kConsumerThreads);
+        if (!single && a.fused && solo && tid == 0)
+            a.counters[item] = 0;
+        named_barrier(1, kConsumerThreads);  // this piece's partial is written; the scratch is free
+        if (!single && a.fused && !solo) {
+            if (!final_piece) {
+                // hand the count to the helper warp and go on streaming
+                if (tid == 0) {
+                    const int q = pushed % kPieceQueue;
+                    if (mbar_wait_bounded(qbar + kPieceQueue + q, ((pushed / kPieceQueue) & 1) ^ 1, abort_flag)) {
+                        volatile int *desc = misc + kMiscQueue + 5 * q;
+                        desc[0] = item;
+                        desc[1] = first_cta;
+                        desc[2] = last_cta;
+                        desc[3] = cur.b;
+                        desc[4] = cur.k;
+                        mbar_arrive(qbar + q);
+                        ++pushed;
+                    } else {
+                        *abort_flag = 1;
+                        atomicOr(a.status, KV_STATUS_WAIT_TIMEOUT);
+                    }
+                }
+            } else {
+                // the CTA's last piece: count it in and merge here if it completed the item
+                if (tid == 0) {
+                    const bool last = atom_add_release_gpu(a.counters + item, 1) == last_cta - first_cta;
+                    if (last)
+                        fence_acquire_gpu();
+                    misc[kMiscLast] = last ? 1 : 0;
+                }
+                named_barrier(1, kConsumerThreads);
+                if (misc[kMiscLast]) {
+                    merge_pieces_global<D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads);
+                    if (tid == 0)
+                        a.counters[item] = 0;
+                }
+            }
+        }
         u += run;
         if (u < count)
             cursor_next_item(a, cur);
+    }
+    // tell the helper there is nothing more
+    if (tid == 0 && a.fused) {
+        const int q = pushed % kPieceQueue;
+        if (mbar_wait_bounded(qbar + kPieceQueue + q, ((pushed / kPieceQueue) & 1) ^ 1, abort_flag)) {
+            misc[kMiscQueue + 5 * q] = -1;
+            mbar_arrive(qbar + q);
+        } else {
+            *abort_flag = 1;
+            atomicOr(a.status, KV_STATUS_WAIT_TIMEOUT);
+        }
     }
 }
 
