@@ -222,6 +222,9 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
  *                     kv-head group) per CTA
  *   KV_OPT_PRODUCER_LANES: 0 auto, 1/2/4/8 lanes of the producer warp that
  *                     issue tile loads
+ *   KV_OPT_HEAD_GROUP: 0 auto (4 if it divides Hkv, else 2 or 1), or 1/2/4 kv
+ *                     heads per work unit when it divides Hkv. It changes
+ *                     paged_attention_workspace_size: set it before sizing.
  * Returns KV_ERR_ARG for an unknown key or value.
  */
 #define KV_OPT_COMPUTE 1
@@ -229,6 +232,7 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
 #define KV_OPT_GRID 3
 #define KV_OPT_MIN_CHUNK 4
 #define KV_OPT_PRODUCER_LANES 5
+#define KV_OPT_HEAD_GROUP 6
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

@@ -1428,6 +1428,7 @@ std::atomic<int> g_opt_combine{0};
 std::atomic<int> g_opt_grid{0};
 std::atomic<int> g_opt_min_chunk{0};
 std::atomic<int> g_opt_prod_lanes{0};
+std::atomic<int> g_opt_head_group{0};
 constexpr int kDefaultMinChunk = 4;
 
 constexpr int kMaxDevices = 64;
@@ -1446,8 +1447,15 @@ int device_sm_count(int dev)
     return v;
 }
 
-// kv heads per work unit: 4 when Hkv is a multiple of 4, else 2 or 1
-int heads_per_unit(int Hkv) { return Hkv % 4 == 0 ? 4 : (Hkv % 2 == 0 ? 2 : 1); }
+// kv heads per work unit: 4 when Hkv is a multiple of 4, else 2 or 1 (or the
+// KV_OPT_HEAD_GROUP setting when it divides Hkv)
+int heads_per_unit(int Hkv)
+{
+    const int want = g_opt_head_group.load();
+    if (want > 0 && Hkv % want == 0)
+        return want;
+    return Hkv % 4 == 0 ? 4 : (Hkv % 2 == 0 ? 2 : 1);
+}
 
 struct Layout {
     int items = 0, slots = 0, max_grid = 0;
@@ -1854,6 +1862,11 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_prod_lanes.store(value);
         return KV_OK;
+    case KV_OPT_HEAD_GROUP:
+        if (value != 0 && value != 1 && value != 2 && value != 4)
+            return KV_ERR_ARG;
+        g_opt_head_group.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -1872,6 +1885,8 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_min_chunk.load();
     case KV_OPT_PRODUCER_LANES:
         return g_opt_prod_lanes.load();
+    case KV_OPT_HEAD_GROUP:
+        return g_opt_head_group.load();
     default:
         return -1;
     }

@@ -20,7 +20,7 @@ PATHS = {"tensor_cores": 1, "cuda_cores": 2}
 def _default_options(pkv):
     yield
     for key in (pkv.KV_OPT_COMPUTE, pkv.KV_OPT_COMBINE, pkv.KV_OPT_GRID, pkv.KV_OPT_MIN_CHUNK,
-                pkv.KV_OPT_PRODUCER_LANES):
+                pkv.KV_OPT_PRODUCER_LANES, pkv.KV_OPT_HEAD_GROUP):
         pkv.set_option(key, 0)
 
 
@@ -74,6 +74,15 @@ def test_many_split_pieces(pkv, oracle_mod, cuda_device, cid, grid, min_chunk):
     cfg = workloads.small_config(cid, batch=6, ctx_lo=1, ctx_hi=1500, W=96, n_layers=1)
     case = Case(cfg, cuda_device)
     run_and_check(pkv, oracle_mod, case, what=f"config {cid} shape, grid {grid} min_chunk {min_chunk}")
+
+
+@pytest.mark.parametrize("hg", [1, 2, 4])
+def test_forced_head_groups(pkv, oracle_mod, cuda_device, hg):
+    """Work units of 1, 2 or 4 kv heads give the same answers."""
+    pkv.set_option(pkv.KV_OPT_HEAD_GROUP, hg)
+    cfg = workloads.small_config(2, batch=9, ctx_lo=1, ctx_hi=900, W=64, n_layers=2)
+    case = Case(cfg, cuda_device, n_layers=2)
+    run_and_check(pkv, oracle_mod, case, what=f"{hg} kv heads per unit")
 
 
 @pytest.mark.parametrize("lanes", [1, 2, 4, 8])
