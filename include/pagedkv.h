@@ -75,6 +75,7 @@ typedef int kv_status;
 #define KV_ERR_CUDA (-4)   /* a CUDA runtime call failed                           */
 
 #define KV_DTYPE_BF16 0
+#define KV_DTYPE_FP16 1
 #define KV_BLOCK_TOKENS 16
 
 /* Bits of the device status word kept in the attention workspace. */
@@ -279,6 +280,73 @@ KV_API int kv_pool_refcount(const void *pool, int32_t id);
 KV_API kv_status kv_pool_append_slots(void *pool, int32_t *block_tables, int W,
                                int32_t *context_lens, int B,
                                int64_t *slot_mapping_out);
+
+/*
+ * Fork: child_row[i] = parent_row[i] for i < n_blocks, each block gaining one
+ * reference (a child sequence starts on its parent's blocks, e.g. several
+ * samples of one prompt). Host arrays; child_row may equal parent_row.
+ * KV_ERR_STATE (nothing changed) if any id is out of range or free.
+ */
+KV_API kv_status kv_pool_fork(void *pool, const int32_t *parent_row, int n_blocks, int32_t *child_row);
+
+/*
+ * Copy-on-write variant of kv_pool_append_slots: when a sequence's new token
+ * would land in a partly filled block that other sequences also reference,
+ * the sequence gets a fresh block instead, the shared block loses that
+ * reference, and the pair (shared block, fresh block) is written to
+ * copy_src_out / copy_dst_out (host arrays of B entries; *n_copies_out is set).
+ * Before this step's append, the caller copies every pair in every layer's K
+ * and V cache (kv_cache_copy_blocks). If all sequences referencing a shared
+ * block append to it in the same step, the last of them keeps the block.
+ * ("Designing an LLM serving system", section "Paged attention": when
+ * sequences sharing a block diverge, the block is copied on write.)
+ * All or nothing: KV_ERR_OOM / KV_ERR_ARG / KV_ERR_STATE as kv_pool_append_slots.
+ */
+KV_API kv_status kv_pool_append_slots_cow(void *pool, int32_t *block_tables, int W,
+                                          int32_t *context_lens, int B,
+                                          int64_t *slot_mapping_out,
+                                          int32_t *copy_src_out, int32_t *copy_dst_out,
+                                          int *n_copies_out);
+
+/* ------------------------------------------------------------------------ */
+/* Whole-block moves over a list of cache tensors                            */
+/* ------------------------------------------------------------------------ */
+/*
+ * caches is a HOST array of n_caches device pointers (1 <= n_caches <= 128;
+ * n_caches == 0 or n == 0 is a no-op), each a cache tensor [num_blocks][16]
+ * [Hkv][D] of element type dtype (KV_DTYPE_BF16 or KV_DTYPE_FP16; bytes are
+ * moved as they are), typically every layer's K and V cache, so that one launch
+ * serves a whole step. Block ids are device int32 arrays of n entries; an id
+ * outside [0, num_blocks) is skipped and KV_STATUS_BAD_BLOCK_ID OR-ed into
+ * *error_flag (device int32, may be NULL). All device pointers 16-byte aligned
+ * (else KV_ERR_ARG); D a multiple of 8. Asynchronous on stream; nothing is
+ * allocated.
+ */
+/*
+ * Copy-on-write: caches[c][dst_ids[i]] = caches[c][src_ids[i]] for every c and
+ * i < n. Destinations must be distinct and no block may be both a source and a
+ * destination in one call (copies run in parallel). ("Designing an LLM serving
+ * system", section "Paged attention": when sequences sharing a block diverge,
+ * the block is copied on write.)
+ */
+KV_API kv_status kv_cache_copy_blocks(void *const *caches, int n_caches, const int32_t *src_ids,
+                                      const int32_t *dst_ids, int n, int num_blocks, int Hkv, int D,
+                                      int dtype, int32_t *error_flag, kv_stream_t stream);
+/*
+ * Swap-out staging: out[c][i] = caches[c][block_ids[i]], out a contiguous
+ * device buffer [n_caches][n][16][Hkv][D] (then one device-to-host copy).
+ * ("Designing an LLM serving system", section "Scheduling: when prefill meets
+ * decode": under memory pressure a preempted sequence's cache blocks are
+ * swapped out, and back in when it resumes.)
+ */
+KV_API kv_status kv_cache_gather_blocks(void *out, void *const *caches, int n_caches,
+                                        const int32_t *block_ids, int n, int num_blocks, int Hkv,
+                                        int D, int dtype, int32_t *error_flag, kv_stream_t stream);
+/* Swap-in: caches[c][block_ids[i]] = in[c][i], in laid out as gather's out.
+ * Ids must be distinct. */
+KV_API kv_status kv_cache_scatter_blocks(void *const *caches, int n_caches, const void *in,
+                                         const int32_t *block_ids, int n, int num_blocks, int Hkv,
+                                         int D, int dtype, int32_t *error_flag, kv_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,6 +19,13 @@ Contents, each citing the passage it follows:
 * :func:`kv_cache_append` -- the byte-exact scatter of new tokens into their
   block slots, slot = block * 16 + offset ("Module 23: Serving", section 23.4:
   blocks are allocated as the sequence grows).
+* :func:`sequence_tokens` -- the logical token rows of one sequence, read
+  through its block table (step 1 of the attention definition above).
+* :func:`copy_blocks`, :func:`gather_blocks`, :func:`scatter_blocks` --
+  whole-block moves: the copy of a shared block when sequences diverge
+  ("Designing an LLM serving system", section "Paged attention": copy on
+  write) and swapping a preempted sequence's blocks out and back in (same
+  page, section "Scheduling: when prefill meets decode").
 * :class:`RefBlockPool` -- a dictionary model of block allocation with
   reference counts for shared prefixes ("Designing an LLM serving system",
   section "Paged attention": blocks can be shared; "Module 23: Serving",
@@ -162,6 +169,45 @@ def kv_cache_append(k_cache, v_cache, k_new, v_new, slot_mapping):
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (status {rc})")
     return kc, vc
+
+
+# ---------------------------------------------------------------------------
+# Reading a sequence through its table, and whole-block moves (numpy).
+# ---------------------------------------------------------------------------
+def sequence_tokens(cache: np.ndarray, table_row, context_len: int) -> np.ndarray:
+    """Rows [c, ...] of one sequence: token t is cache[table_row[t // 16]][t % 16].
+
+    "Designing an LLM serving system", section "Paged attention": logical
+    positions map to physical blocks through the sequence's page table.
+    """
+    out = np.empty((context_len,) + cache.shape[2:], dtype=cache.dtype)
+    for t in range(context_len):
+        out[t] = cache[int(table_row[t // BLOCK_TOKENS])][t % BLOCK_TOKENS]
+    return out
+
+
+def copy_blocks(cache: np.ndarray, src_ids, dst_ids) -> np.ndarray:
+    """A new cache with block dst_ids[i] replaced by block src_ids[i] (all read before any write)."""
+    src_ids, dst_ids = list(src_ids), list(dst_ids)
+    if len(src_ids) != len(dst_ids):
+        raise ValueError("src_ids and dst_ids differ in length")
+    out = cache.copy()
+    for s, d in zip(src_ids, dst_ids):
+        out[d] = cache[s]
+    return out
+
+
+def gather_blocks(cache: np.ndarray, ids) -> np.ndarray:
+    """Blocks ids[0], ids[1], ... stacked in that order (swap-out staging)."""
+    return np.stack([cache[i] for i in ids]) if len(ids) else np.empty((0,) + cache.shape[1:], cache.dtype)
+
+
+def scatter_blocks(cache: np.ndarray, data: np.ndarray, ids) -> np.ndarray:
+    """A new cache with block ids[i] replaced by data[i] (swap-in)."""
+    out = cache.copy()
+    for i, b in enumerate(ids):
+        out[b] = data[i]
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -22,7 +22,7 @@ if not os.path.exists(LIB_PATH):
 _lib = ctypes.CDLL(LIB_PATH)
 
 KV_OK, KV_ERR_ARG, KV_ERR_OOM, KV_ERR_STATE, KV_ERR_CUDA = 0, -1, -2, -3, -4
-KV_DTYPE_BF16 = 0
+KV_DTYPE_BF16, KV_DTYPE_FP16 = 0, 1
 BLOCK_TOKENS = 16
 KV_STATUS_BAD_BLOCK_ID, KV_STATUS_BAD_CONTEXT, KV_STATUS_WAIT_TIMEOUT, KV_STATUS_BAD_SLOT = 1, 2, 4, 8
 KV_OPT_COMPUTE, KV_OPT_COMBINE, KV_OPT_GRID, KV_OPT_MIN_CHUNK, KV_OPT_PRODUCER_LANES, KV_OPT_HEAD_GROUP = (
@@ -52,6 +52,11 @@ _sig = {
     "kv_pool_num_blocks": (_I, [_P]),
     "kv_pool_refcount": (_I, [_P, ctypes.c_int32]),
     "kv_pool_append_slots": (_I, [_P, _P, _I, _P, _I, _P]),
+    "kv_pool_fork": (_I, [_P, _P, _I, _P]),
+    "kv_pool_append_slots_cow": (_I, [_P, _P, _I, _P, _I, _P, _P, _P, ctypes.POINTER(ctypes.c_int)]),
+    "kv_cache_copy_blocks": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "kv_cache_gather_blocks": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "kv_cache_scatter_blocks": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
 }
 for _name, (_res, _args) in _sig.items():
     _f = getattr(_lib, _name)
@@ -157,6 +162,73 @@ def paged_attention_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: tor
     return out
 
 
+def _cache_dtype(cache: torch.Tensor) -> int:
+    if cache.dtype == torch.bfloat16:
+        return KV_DTYPE_BF16
+    if cache.dtype == torch.float16:
+        return KV_DTYPE_FP16
+    raise ValueError(f"cache must be bfloat16 or float16, got {cache.dtype}")
+
+
+def _cache_list(caches) -> tuple[ctypes.Array, int, tuple]:
+    """Host pointer array for a list of same-shape, same-dtype cache tensors [num_blocks,16,Hkv,D]."""
+    caches = list(caches)
+    if not caches:
+        raise ValueError("no caches given")
+    shape, dtype = tuple(caches[0].shape), caches[0].dtype
+    if len(shape) != 4 or shape[1] != BLOCK_TOKENS:
+        raise ValueError("caches must be [num_blocks,16,Hkv,D]")
+    for i, c in enumerate(caches):
+        if tuple(c.shape) != shape or c.dtype != dtype:
+            raise ValueError("caches must share shape and dtype")
+        _dev(c, f"caches[{i}]")
+    ptrs = (ctypes.c_void_p * len(caches))(*[c.data_ptr() for c in caches])
+    return ptrs, len(caches), shape
+
+
+def kv_cache_copy_blocks(caches, src_ids: torch.Tensor, dst_ids: torch.Tensor,
+                         error_flag: torch.Tensor | None = None, stream=None) -> None:
+    """caches[c][dst_ids[i]] = caches[c][src_ids[i]] for whole blocks of every cache (copy-on-write).
+
+    ``caches`` is a list of cache tensors (e.g. every layer's K and V); ids are int32 on the device.
+    """
+    ptrs, nc, (num_blocks, _, Hkv, D) = _cache_list(caches)
+    n = src_ids.numel()
+    if dst_ids.numel() != n:
+        raise ValueError("shape mismatch")
+    ef = _dev(error_flag, "error_flag", torch.int32) if error_flag is not None else None
+    _check("kv_cache_copy_blocks", _lib.kv_cache_copy_blocks(
+        ptrs, nc, _dev(src_ids, "src_ids", torch.int32), _dev(dst_ids, "dst_ids", torch.int32), n,
+        num_blocks, Hkv, D, _cache_dtype(caches[0]), ef, _stream_handle(stream)))
+
+
+def kv_cache_gather_blocks(out: torch.Tensor, caches, block_ids: torch.Tensor,
+                           error_flag: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[c,i] = caches[c][block_ids[i]]; out is [len(caches),n,16,Hkv,D] (swap-out staging)."""
+    ptrs, nc, (num_blocks, bt, Hkv, D) = _cache_list(caches)
+    n = block_ids.numel()
+    if tuple(out.shape) != (nc, n, bt, Hkv, D) or out.dtype != caches[0].dtype:
+        raise ValueError("shape mismatch")
+    ef = _dev(error_flag, "error_flag", torch.int32) if error_flag is not None else None
+    _check("kv_cache_gather_blocks", _lib.kv_cache_gather_blocks(
+        _dev(out, "out"), ptrs, nc, _dev(block_ids, "block_ids", torch.int32), n, num_blocks, Hkv, D,
+        _cache_dtype(caches[0]), ef, _stream_handle(stream)))
+    return out
+
+
+def kv_cache_scatter_blocks(caches, inp: torch.Tensor, block_ids: torch.Tensor,
+                            error_flag: torch.Tensor | None = None, stream=None) -> None:
+    """caches[c][block_ids[i]] = inp[c,i]; inp is [len(caches),n,16,Hkv,D] (swap-in)."""
+    ptrs, nc, (num_blocks, bt, Hkv, D) = _cache_list(caches)
+    n = block_ids.numel()
+    if tuple(inp.shape) != (nc, n, bt, Hkv, D) or inp.dtype != caches[0].dtype:
+        raise ValueError("shape mismatch")
+    ef = _dev(error_flag, "error_flag", torch.int32) if error_flag is not None else None
+    _check("kv_cache_scatter_blocks", _lib.kv_cache_scatter_blocks(
+        ptrs, nc, _dev(inp, "inp"), _dev(block_ids, "block_ids", torch.int32), n, num_blocks, Hkv, D,
+        _cache_dtype(caches[0]), ef, _stream_handle(stream)))
+
+
 def read_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
     """Synchronise the stream and return (optionally clearing) the device status word."""
     v = ctypes.c_int32(0)
@@ -234,3 +306,29 @@ class BlockPool:
         B, W = block_tables.shape
         _check("kv_pool_append_slots", _lib.kv_pool_append_slots(
             self._h, block_tables.data_ptr(), W, context_lens.data_ptr(), B, slot_mapping.data_ptr()))
+
+    def fork(self, parent_ids) -> list[int]:
+        """A child's block ids: the parent's, each with one more reference."""
+        ids = list(parent_ids)
+        child = (ctypes.c_int32 * max(len(ids), 1))()
+        _check("kv_pool_fork", _lib.kv_pool_fork(self._h, _i32(ids), len(ids), child))
+        return list(child[:len(ids)])
+
+    def append_slots_cow(self, block_tables: torch.Tensor, context_lens: torch.Tensor,
+                         slot_mapping: torch.Tensor) -> tuple[list[int], list[int]]:
+        """append_slots that copies a shared partly filled tail block instead of refusing it.
+
+        Returns (src, dst): the blocks to copy, in every layer's caches, before this step's append.
+        """
+        for t, name, dt in ((block_tables, "block_tables", torch.int32), (context_lens, "context_lens", torch.int32),
+                            (slot_mapping, "slot_mapping", torch.int64)):
+            if t.is_cuda or not t.is_contiguous() or t.dtype != dt:
+                raise ValueError(f"{name} must be a contiguous host {dt} tensor")
+        B, W = block_tables.shape
+        src = (ctypes.c_int32 * max(B, 1))()
+        dst = (ctypes.c_int32 * max(B, 1))()
+        n = ctypes.c_int(0)
+        _check("kv_pool_append_slots_cow", _lib.kv_pool_append_slots_cow(
+            self._h, block_tables.data_ptr(), W, context_lens.data_ptr(), B, slot_mapping.data_ptr(), src, dst,
+            ctypes.byref(n)))
+        return list(src[:n.value]), list(dst[:n.value])

@@ -176,3 +176,88 @@ extern "C" kv_status kv_pool_append_slots(void *pool, int32_t *block_tables, int
     }
     return KV_OK;
 }
+
+extern "C" kv_status kv_pool_fork(void *pool, const int32_t *parent_row, int n_blocks, int32_t *child_row)
+{
+    if (!pool || n_blocks < 0 || (n_blocks > 0 && (!parent_row || !child_row)))
+        return KV_ERR_ARG;
+    BlockPool *p = as_pool(pool);
+    std::lock_guard<std::mutex> lock(p->mu);
+    const int64_t nb = static_cast<int64_t>(p->refcount.size());
+    for (int i = 0; i < n_blocks; ++i)
+        if (parent_row[i] < 0 || parent_row[i] >= nb || p->refcount[static_cast<size_t>(parent_row[i])] <= 0)
+            return KV_ERR_STATE;
+    for (int i = 0; i < n_blocks; ++i) {
+        ++p->refcount[static_cast<size_t>(parent_row[i])];
+        child_row[i] = parent_row[i];
+    }
+    return KV_OK;
+}
+
+extern "C" kv_status kv_pool_append_slots_cow(void *pool, int32_t *block_tables, int W, int32_t *context_lens, int B,
+                                              int64_t *slot_mapping_out, int32_t *copy_src_out,
+                                              int32_t *copy_dst_out, int *n_copies_out)
+{
+    if (!pool || B < 0 || W < 1 || !n_copies_out ||
+        (B > 0 && (!block_tables || !context_lens || !slot_mapping_out || !copy_src_out || !copy_dst_out)))
+        return KV_ERR_ARG;
+    BlockPool *p = as_pool(pool);
+    std::lock_guard<std::mutex> lock(p->mu);
+    const int64_t nb = static_cast<int64_t>(p->refcount.size());
+    // validate the whole step first; count fresh blocks and copies
+    size_t need = 0;
+    std::unordered_map<int32_t, int> drops;  // references the copies will give up, per shared block
+    for (int b = 0; b < B; ++b) {
+        const int c = context_lens[b];
+        if (c < 0 || c / KV_BLOCK_TOKENS >= W)
+            return KV_ERR_ARG;
+        if (c % KV_BLOCK_TOKENS == 0) {
+            ++need;
+            continue;
+        }
+        const int32_t tail = block_tables[static_cast<size_t>(b) * W + c / KV_BLOCK_TOKENS];
+        if (tail < 0 || tail >= nb || p->refcount[static_cast<size_t>(tail)] <= 0)
+            return KV_ERR_STATE;
+        if (p->refcount[static_cast<size_t>(tail)] > 1)
+            ++drops[tail];
+    }
+    // A block whose every reference appends this step would be copied for all of
+    // them and then freed; the last of them keeps it instead (it is then private).
+    for (auto &kv : drops) {
+        if (kv.second >= p->refcount[static_cast<size_t>(kv.first)])
+            kv.second = p->refcount[static_cast<size_t>(kv.first)] - 1;
+        need += static_cast<size_t>(kv.second);
+    }
+    if (need > p->free_ids.size())
+        return KV_ERR_OOM;
+    int copies = 0;
+    for (int b = 0; b < B; ++b) {
+        const int c = context_lens[b];
+        int32_t *row = block_tables + static_cast<size_t>(b) * W;
+        if (c % KV_BLOCK_TOKENS == 0) {
+            const int32_t id = p->free_ids.back();
+            p->free_ids.pop_back();
+            p->refcount[static_cast<size_t>(id)] = 1;
+            row[c / KV_BLOCK_TOKENS] = id;
+        } else {
+            const int32_t tail = row[c / KV_BLOCK_TOKENS];
+            auto it = drops.find(tail);
+            if (it != drops.end() && it->second > 0) {
+                --it->second;
+                const int32_t id = p->free_ids.back();
+                p->free_ids.pop_back();
+                p->refcount[static_cast<size_t>(id)] = 1;
+                --p->refcount[static_cast<size_t>(tail)];
+                row[c / KV_BLOCK_TOKENS] = id;
+                copy_src_out[copies] = tail;
+                copy_dst_out[copies] = id;
+                ++copies;
+            }
+        }
+        slot_mapping_out[b] =
+            static_cast<int64_t>(row[c / KV_BLOCK_TOKENS]) * KV_BLOCK_TOKENS + c % KV_BLOCK_TOKENS;
+        context_lens[b] = c + 1;
+    }
+    *n_copies_out = copies;
+    return KV_OK;
+}

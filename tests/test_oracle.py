@@ -306,6 +306,45 @@ def test_ref_pool_semantics(oracle_mod):
 
 
 # ---------------------------------------------------------------------------
+# reading through the table, and whole-block moves
+# ---------------------------------------------------------------------------
+def test_sequence_tokens_recovers_the_dense_sequence(oracle_mod):
+    """paginate() places each dense sequence in shuffled blocks with its own loop; reading
+    back through the table gives the dense rows, and never a filler row."""
+    lens = [1, 15, 16, 17, 40]
+    q, K, V = make_dense_case(5, lens, 4, 2, 8)
+    kp, vp, tab = paginate(K, V, lens, 2, 8, 20, 3, 6)
+    for b, c in enumerate(lens):
+        np.testing.assert_array_equal(oracle_mod.sequence_tokens(kp, tab[b], c), bits(K[b]))
+        np.testing.assert_array_equal(oracle_mod.sequence_tokens(vp, tab[b], c), bits(V[b]))
+
+
+def test_block_moves(oracle_mod):
+    rng = np.random.default_rng(7)
+    cache = rng.integers(0, 2 ** 16, size=(12, 16, 2, 8), dtype=np.uint16)
+    src, dst = [3, 3, 9], [0, 5, 11]
+    out = oracle_mod.copy_blocks(cache, src, dst)
+    for s_, d_ in zip(src, dst):
+        np.testing.assert_array_equal(out[d_], cache[s_])
+    untouched = [i for i in range(12) if i not in dst]
+    np.testing.assert_array_equal(out[untouched], cache[untouched])
+    # a swap: every source read before any write
+    sw = oracle_mod.copy_blocks(cache, [1, 2], [2, 1])
+    np.testing.assert_array_equal(sw[1], cache[2])
+    np.testing.assert_array_equal(sw[2], cache[1])
+    # gather then scatter into other blocks moves the rows; gathering those gives them back
+    ids, new_ids = [7, 2, 10], [4, 8, 6]
+    packed = oracle_mod.gather_blocks(cache, ids)
+    assert packed.shape == (3, 16, 2, 8)
+    for k, i in enumerate(ids):
+        assert int(packed[k].astype(np.uint64).sum()) == int(cache[i].astype(np.uint64).sum())
+    back = oracle_mod.scatter_blocks(np.zeros_like(cache), packed, new_ids)
+    np.testing.assert_array_equal(oracle_mod.gather_blocks(back, new_ids), packed)
+    assert not back[[i for i in range(12) if i not in new_ids]].any()
+    assert oracle_mod.gather_blocks(cache, []).shape == (0, 16, 2, 8)
+
+
+# ---------------------------------------------------------------------------
 # the pins catch planted mistakes
 # ---------------------------------------------------------------------------
 MUTANTS = {

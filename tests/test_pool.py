@@ -222,3 +222,74 @@ def test_continuous_batch_redraw_keeps_refcounts(pkv):
         assert len(set(slots.tolist())) == cfg.batch        # every new token has its own slot
         for b in range(cfg.batch):                          # ... in a block no other sequence uses
             assert cb.pool.refcount(int(slots[b]) // 16) == 1
+
+
+# ---------------------------------------------------------------------------
+# fork and copy-on-write ("Designing an LLM serving system", section "Paged attention")
+# ---------------------------------------------------------------------------
+def test_fork_shares_every_block(pkv):
+    p = pkv.BlockPool(6)
+    parent = p.alloc(3)
+    child = p.fork(parent)
+    assert child == parent and all(p.refcount(i) == 2 for i in parent)
+    free_id = next(i for i in range(6) if p.refcount(i) == 0)
+    with pytest.raises(pkv.KVError) as e:
+        p.fork([parent[0], free_id])               # a free block cannot be forked
+    assert e.value.status == pkv.KV_ERR_STATE
+    assert all(p.refcount(i) == 2 for i in parent)
+    assert p.fork([]) == []
+
+
+def test_copy_on_write_keeps_every_sequence_view(pkv, oracle_mod):
+    from cow_cases import ForkScenario, OracleBackend
+    for seed in (0, 1, 2):
+        sc = ForkScenario(pkv, seed=seed)
+        sc.run(oracle_mod, OracleBackend(oracle_mod, sc), n_random_steps=60)
+        assert sc.copies_total >= 3
+
+
+def test_copy_on_write_without_sharing_matches_append_slots(pkv):
+    """With no shared tail, the copy-on-write variant does exactly what append_slots does."""
+    a, b = pkv.BlockPool(40), pkv.BlockPool(40)
+    B, W = 4, 8
+    ta, tb = torch.full((B, W), -1, dtype=torch.int32), torch.full((B, W), -1, dtype=torch.int32)
+    la, lb = torch.zeros(B, dtype=torch.int32), torch.zeros(B, dtype=torch.int32)
+    sa, sb = torch.zeros(B, dtype=torch.int64), torch.zeros(B, dtype=torch.int64)
+    for _ in range(70):
+        a.append_slots(ta, la, sa)
+        src, dst = b.append_slots_cow(tb, lb, sb)
+        assert src == [] and dst == []
+        assert torch.equal(ta, tb) and torch.equal(la, lb) and torch.equal(sa, sb)
+
+
+def test_copy_on_write_errors_leave_state_unchanged(pkv):
+    p = pkv.BlockPool(3)
+    tables = torch.full((3, 2), -1, dtype=torch.int32)
+    blk = p.alloc(1)[0]
+    p.fork([blk])
+    p.fork([blk])                                  # three sequences on one 5-token block
+    tables[:, 0] = blk
+    p.alloc(1)                                     # one block left free
+    lens = torch.tensor([5, 5, 5], dtype=torch.int32)
+    slots = torch.zeros(3, dtype=torch.int64)
+    t0, l0 = tables.clone(), lens.clone()
+    with pytest.raises(pkv.KVError) as e:          # all three append: two copies, one free block
+        p.append_slots_cow(tables, lens, slots)
+    assert e.value.status == pkv.KV_ERR_OOM
+    assert torch.equal(tables, t0) and torch.equal(lens, l0)
+    assert p.refcount(blk) == 3 and p.num_free() == 1
+    sub_t, sub_l, sub_s = tables[:2].clone(), lens[:2].clone(), slots[:2].clone()
+    with pytest.raises(pkv.KVError):               # two of three append: still two copies
+        p.append_slots_cow(sub_t, sub_l, sub_s)
+    assert p.refcount(blk) == 3 and p.num_free() == 1
+    sub_t, sub_l, sub_s = tables[:1].clone(), lens[:1].clone(), slots[:1].clone()
+    src, dst = p.append_slots_cow(sub_t, sub_l, sub_s)   # one appends: one copy
+    assert src == [blk] and dst == [int(sub_t[0, 0])] and dst[0] != blk
+    assert int(sub_s[0]) == dst[0] * 16 + 5 and int(sub_l[0]) == 6
+    assert p.refcount(blk) == 2 and p.refcount(dst[0]) == 1 and p.num_free() == 0
+    p.free([dst[0]])
+    bad = tables[:1].clone()
+    bad[0, 0] = dst[0]                              # a free block as the tail
+    with pytest.raises(pkv.KVError) as e:
+        p.append_slots_cow(bad, lens[:1].clone(), slots[:1].clone())
+    assert e.value.status == pkv.KV_ERR_STATE and p.num_free() == 1
