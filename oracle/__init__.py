@@ -16,6 +16,8 @@ Contents, each citing the passage it follows:
   head h reading kv head h // (Hq // Hkv) ("Scaling LLM serving", section
   "The KV cache", Share key/value heads). Implemented in plain C, float64,
   in ``pagedkv_oracle.c``.
+  With ``dtype="fp16"`` the inputs are IEEE binary16 instead of bf16 (2 bytes
+  per number for fp16 or bf16: "Module 23: Serving", section 23.1).
 * :func:`kv_cache_append` -- the byte-exact scatter of new tokens into their
   block slots, slot = block * 16 + offset ("Module 23: Serving", section 23.4:
   blocks are allocated as the sequence grows).
@@ -73,6 +75,10 @@ def _load():
             lib.oracle_paged_attention_decode.argtypes = [P, P, P, P, P, P, I, P, I, I, I, I, I,
                                                           ctypes.c_double]
             lib.oracle_paged_attention_decode.restype = I
+            lib.oracle_paged_attention_decode_fp16.argtypes = lib.oracle_paged_attention_decode.argtypes
+            lib.oracle_paged_attention_decode_fp16.restype = I
+            lib.oracle_widen.argtypes = [I, ctypes.c_uint16]
+            lib.oracle_widen.restype = ctypes.c_double
             lib.oracle_kv_cache_append.argtypes = [P, P, P, P, P, I, I, I, I]
             lib.oracle_kv_cache_append.restype = I
             lib.oracle_num_threads.argtypes = []
@@ -96,6 +102,23 @@ def bf16_bits(x) -> np.ndarray:
     if x.dtype != torch.bfloat16:
         raise TypeError(f"expected a bf16 tensor, got {x.dtype}")
     return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def fp16_bits(x) -> np.ndarray:
+    """Raw IEEE binary16 bit patterns (uint16) of a CPU float16 tensor or a uint16 array."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("expected fp16 bit patterns as uint16")
+        return np.ascontiguousarray(x)
+    import torch
+    if x.dtype != torch.float16:
+        raise TypeError(f"expected a float16 tensor, got {x.dtype}")
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def widen(kind: str, bits: int) -> float:
+    """The C oracle's exact widening of one 16-bit pattern ("bf16" or "fp16") to float64."""
+    return float(_load().oracle_widen(1 if kind == "fp16" else 0, int(bits)))
 
 
 def bf16_bits_to_float64(bits: np.ndarray) -> np.ndarray:
@@ -124,14 +147,18 @@ def kv_cache_bytes(n_layers: int, n_kv_heads: int, d_head: int, context_len: int
 # Attention oracle (C, float64).
 # ---------------------------------------------------------------------------
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float,
-                           return_weight_sums: bool = False):
+                           return_weight_sums: bool = False, dtype: str = "bf16"):
     """Reference decode attention in float64.
 
-    q [B,Hq,D], k_cache/v_cache [num_blocks,16,Hkv,D] as bf16 tensors or uint16
-    bit arrays; block_tables [B,W] int32; context_lens [B] int32.
+    q [B,Hq,D], k_cache/v_cache [num_blocks,16,Hkv,D] as bf16 (or, with
+    dtype="fp16", float16) tensors or uint16 bit arrays; block_tables [B,W]
+    int32; context_lens [B] int32.
     Returns out [B,Hq,D] float64 (and the per-(b,h) softmax weight sums).
     """
-    qb, kb, vb = bf16_bits(q), bf16_bits(k_cache), bf16_bits(v_cache)
+    if dtype not in ("bf16", "fp16"):
+        raise ValueError("dtype must be 'bf16' or 'fp16'")
+    unpack = fp16_bits if dtype == "fp16" else bf16_bits
+    qb, kb, vb = unpack(q), unpack(k_cache), unpack(v_cache)
     tables = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
     lens = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
     B, Hq, D = qb.shape
@@ -143,12 +170,17 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     W = tables.shape[1]
     out = np.empty((B, Hq, D), dtype=np.float64)
     wsum = np.empty((B, Hq), dtype=np.float64)
-    rc = _load().oracle_paged_attention_decode(_ptr(out), _ptr(wsum), _ptr(qb), _ptr(kb), _ptr(vb),
+    fn = _load().oracle_paged_attention_decode_fp16 if dtype == "fp16" else _load().oracle_paged_attention_decode
+    rc = fn(_ptr(out), _ptr(wsum), _ptr(qb), _ptr(kb), _ptr(vb),
                                                _ptr(tables), W, _ptr(lens), B, num_blocks,
                                                Hq, Hkv, D, float(scale))
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (status {rc})")
     return (out, wsum) if return_weight_sums else out
+
+
+def _is_fp16(x) -> bool:
+    return not isinstance(x, np.ndarray) and str(x.dtype) == "torch.float16"
 
 
 def kv_cache_append(k_cache, v_cache, k_new, v_new, slot_mapping):
@@ -157,8 +189,9 @@ def kv_cache_append(k_cache, v_cache, k_new, v_new, slot_mapping):
     For every i with slot_mapping[i] >= 0, cache[slot // 16][slot % 16] = new[i]
     for all heads, byte for byte; every other byte is unchanged.
     """
-    kc, vc = bf16_bits(k_cache).copy(), bf16_bits(v_cache).copy()
-    kn, vn = bf16_bits(k_new), bf16_bits(v_new)
+    unpack = fp16_bits if _is_fp16(k_cache) else bf16_bits
+    kc, vc = unpack(k_cache).copy(), unpack(v_cache).copy()
+    kn, vn = unpack(k_new), unpack(v_new)
     slots = np.ascontiguousarray(np.asarray(slot_mapping, dtype=np.int64))
     num_blocks, _, Hkv, D = kc.shape
     T = slots.shape[0]

@@ -22,6 +22,9 @@
  *   q            [B][Hq][D]                    bf16 bit patterns (uint16)
  *   k_cache      [num_blocks][16][Hkv][D]      bf16 bit patterns
  *   v_cache      [num_blocks][16][Hkv][D]      bf16 bit patterns
+ *   (oracle_paged_attention_decode_fp16: the same with IEEE binary16 bit
+ *   patterns; "Module 23: Serving", section 23.1: 2 bytes per number for
+ *   fp16 or bf16)
  *   block_tables [B][W]                        int32 physical block ids
  *   context_lens [B]                           int32 tokens cached (>= 0)
  *   out          [B][Hq][D]                    float64
@@ -49,6 +52,24 @@ static double bf16_bits_to_double(uint16_t bits)
     return (double)f;
 }
 
+/* IEEE 754 binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits.
+ * Exponent 0 holds zero and the subnormals (fraction * 2^-24), exponent 31
+ * infinity (fraction 0) and NaN. Every value is exact in double. */
+static double fp16_bits_to_double(uint16_t bits)
+{
+    const int sign = bits >> 15;
+    const int expo = (bits >> 10) & 0x1f;
+    const int frac = bits & 0x3ff;
+    double mag;
+    if (expo == 0)
+        mag = ldexp((double)frac, -24);
+    else if (expo == 31)
+        mag = frac ? NAN : INFINITY;
+    else
+        mag = ldexp((double)(1024 + frac), expo - 25);
+    return sign ? -mag : mag;
+}
+
 /* Step 1 of the definition: where logical token t of sequence b lives. */
 static size_t cache_row_offset(const int32_t *block_tables, int W, int b, int t,
                                int Hkv, int j, int D)
@@ -58,14 +79,14 @@ static size_t cache_row_offset(const int32_t *block_tables, int W, int b, int t,
     return (((size_t)phys * ORACLE_BLOCK_TOKENS + row) * Hkv + j) * (size_t)D;
 }
 
-int oracle_paged_attention_decode(double *out, double *weight_sums,
-                                  const uint16_t *q,
-                                  const uint16_t *k_cache,
-                                  const uint16_t *v_cache,
-                                  const int32_t *block_tables, int W,
-                                  const int32_t *context_lens, int B,
-                                  int num_blocks, int Hq, int Hkv, int D,
-                                  double scale)
+static int decode_any(double *out, double *weight_sums,
+                      const uint16_t *q,
+                      const uint16_t *k_cache,
+                      const uint16_t *v_cache,
+                      const int32_t *block_tables, int W,
+                      const int32_t *context_lens, int B,
+                      int num_blocks, int Hq, int Hkv, int D,
+                      double scale, double (*widen)(uint16_t))
 {
     if (B < 0 || W < 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_blocks < 0)
         return -1;
@@ -115,7 +136,7 @@ int oracle_paged_attention_decode(double *out, double *weight_sums,
             const uint16_t *kt = k_cache + cache_row_offset(block_tables, W, b, t, Hkv, j, D);
             double dot = 0.0;
             for (int d = 0; d < D; ++d)
-                dot += bf16_bits_to_double(qh[d]) * bf16_bits_to_double(kt[d]);
+                dot += widen(qh[d]) * widen(kt[d]);
             z[t] = scale * dot;
         }
 
@@ -136,7 +157,7 @@ int oracle_paged_attention_decode(double *out, double *weight_sums,
             const double w = z[t] / denom;
             const uint16_t *vt = v_cache + cache_row_offset(block_tables, W, b, t, Hkv, j, D);
             for (int d = 0; d < D; ++d)
-                o[d] += w * bf16_bits_to_double(vt[d]);
+                o[d] += w * widen(vt[d]);
             wsum += w;
         }
         if (weight_sums)
@@ -144,6 +165,39 @@ int oracle_paged_attention_decode(double *out, double *weight_sums,
         free(z);
     }
     return failed ? -2 : 0;
+}
+
+int oracle_paged_attention_decode(double *out, double *weight_sums,
+                                  const uint16_t *q,
+                                  const uint16_t *k_cache,
+                                  const uint16_t *v_cache,
+                                  const int32_t *block_tables, int W,
+                                  const int32_t *context_lens, int B,
+                                  int num_blocks, int Hq, int Hkv, int D,
+                                  double scale)
+{
+    return decode_any(out, weight_sums, q, k_cache, v_cache, block_tables, W, context_lens, B,
+                      num_blocks, Hq, Hkv, D, scale, bf16_bits_to_double);
+}
+
+int oracle_paged_attention_decode_fp16(double *out, double *weight_sums,
+                                       const uint16_t *q,
+                                       const uint16_t *k_cache,
+                                       const uint16_t *v_cache,
+                                       const int32_t *block_tables, int W,
+                                       const int32_t *context_lens, int B,
+                                       int num_blocks, int Hq, int Hkv, int D,
+                                       double scale)
+{
+    return decode_any(out, weight_sums, q, k_cache, v_cache, block_tables, W, context_lens, B,
+                      num_blocks, Hq, Hkv, D, scale, fp16_bits_to_double);
+}
+
+/* Widening of one bit pattern (kind 0: bf16, 1: fp16), exposed so the tests can
+ * check the conversions against an independent library over all 65536 codes. */
+double oracle_widen(int kind, uint16_t bits)
+{
+    return kind ? fp16_bits_to_double(bits) : bf16_bits_to_double(bits);
 }
 
 /*

@@ -306,6 +306,36 @@ def test_ref_pool_semantics(oracle_mod):
 
 
 # ---------------------------------------------------------------------------
+# fp16 inputs ("Module 23: Serving", section 23.1: 2 bytes per number, fp16 or bf16)
+# ---------------------------------------------------------------------------
+def test_widening_matches_libraries_for_every_code(oracle_mod):
+    codes = np.arange(65536, dtype=np.uint16)
+    for kind, ref in (("fp16", codes.view(np.float16).astype(np.float64)),
+                      ("bf16", torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).double().numpy())):
+        got = np.array([oracle_mod.widen(kind, c) for c in codes])
+        same = (got == ref) | (np.isnan(got) & np.isnan(ref))
+        assert same.all(), f"{kind}: first mismatch at code {int(np.argmin(same)):#06x}"
+        assert (np.signbit(got) == np.signbit(ref))[~np.isnan(ref)].all()
+
+
+def test_fp16_decode_matches_dense_attention(oracle_mod):
+    lens, Hq, Hkv, D = TINY_LENS, 4, 2, 8
+    g = torch.Generator().manual_seed(21)
+    q = torch.randn(len(lens), Hq, D, generator=g).half()
+    K = [torch.randn(c, Hkv, D, generator=g).half() for c in lens]
+    V = [torch.randn(c, Hkv, D, generator=g).half() for c in lens]
+    nb = sum(-(-c // 16) for c in lens) + 5
+    kp, vp, tab = paginate(K, V, lens, Hkv, D, nb, 3, 22, fill=np.uint16(0x7E00))   # fp16 NaN filler
+    scale = 1.0 / math.sqrt(D)
+    out = oracle_mod.paged_attention_decode(q, kp, vp, tab, np.array(lens, np.int32), scale, dtype="fp16")
+    ref = dense_reference(q, K, V, lens, Hq, Hkv, scale)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    # the same bit patterns read as bf16 give a different answer: the dtype is honoured
+    other = oracle_mod.paged_attention_decode(bits(q), kp, vp, tab, np.array(lens, np.int32), scale)
+    assert not np.allclose(np.nan_to_num(other), ref)
+
+
+# ---------------------------------------------------------------------------
 # reading through the table, and whole-block moves
 # ---------------------------------------------------------------------------
 def test_sequence_tokens_recovers_the_dense_sequence(oracle_mod):
