@@ -46,7 +46,7 @@ from paged_kv_cache_470_b200 import workloads  # noqa: E402  (no CUDA library ne
 
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_0p5b_gqa.txt")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_470_b200", "csrc", "decode.cu")
 
 
@@ -86,15 +86,22 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if it matches the current kernel source."""
+def profiled_traffic(cfg):
+    """DRAM bytes per decode launch from a committed ncu summary of this workload and element type,
+    if one matches the current kernel source (else None)."""
     try:
-        text = open(PROFILE_SUMMARY).read()
         src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
-        m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-        h = re.search(r"decode\.cu sha256\[:16\]:\s*([0-9a-f]+)", text)
-        if m and h and h.group(1) == src_hash:
-            return float(m.group(1))
+        for name in sorted(os.listdir(PROFILE_DIR)):
+            if not name.endswith(".txt"):
+                continue
+            text = open(os.path.join(PROFILE_DIR, name)).read()
+            m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+            h = re.search(r"decode\.cu sha256\[:16\]:\s*([0-9a-f]+)", text)
+            c = re.search(r"^config_id:\s*(\d+)", text, re.M)
+            e = re.search(r"^elem:\s*(\w+)", text, re.M)
+            if m and h and c and e and h.group(1) == src_hash and int(c.group(1)) == cfg.cid \
+                    and e.group(1) == cfg.elem:
+                return float(m.group(1))
     except OSError:
         pass
     return None
@@ -216,7 +223,7 @@ class Workload:
         gen = workloads.device_generator(cfg.seed + 1000 * rank, device)
         self.k, self.v = [], []
         for _ in range(cfg.n_layers):
-            k, v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device)
+            k, v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device, cfg.torch_dtype)
             self.k.append(k)
             self.v.append(v)
         self.q, self.k_new, self.v_new = workloads.make_step_inputs(cfg, gen, device)
@@ -355,7 +362,7 @@ class OracleSampler:
         import oracle
         self.oracle, self.cfg, self.layout = oracle, cfg, layout
         gen = workloads.device_generator(cfg.seed, "cpu")
-        self.k, self.v = workloads.make_layer_cache(layout.num_blocks, cfg.Hkv, cfg.D, gen, "cpu")
+        self.k, self.v = workloads.make_layer_cache(layout.num_blocks, cfg.Hkv, cfg.D, gen, "cpu", cfg.torch_dtype)
         q, kn, vn = workloads.make_step_inputs(cfg, gen, "cpu", n_layers=1)
         self.q, self.kn, self.vn = q[0], kn[0], vn[0]
         self.slots = layout.slot_mapping().numpy()
@@ -370,7 +377,8 @@ class OracleSampler:
         done_bytes, done_layers, t0 = 0, 0, time.perf_counter()
         while True:
             k2, v2 = self.oracle.kv_cache_append(self.k, self.v, self.kn, self.vn, self.slots)
-            self.oracle.paged_attention_decode(self.q, k2, v2, self.tables, self.lens, self.cfg.scale)
+            self.oracle.paged_attention_decode(self.q, k2, v2, self.tables, self.lens, self.cfg.scale,
+                                               dtype=self.cfg.elem)
             done_bytes += self.layer_bytes
             done_layers += 1
             if time.perf_counter() - t0 >= seconds:
@@ -391,11 +399,17 @@ def run_profile_step(args, cfg, device):
                       "status": pkv.read_status(wl.ws)}), flush=True)
 
 
+def pick_config(args):
+    """The workload named by --config, with --layers and --dtype applied."""
+    over = {"elem": args.dtype}
+    if args.layers:
+        over["n_layers"] = args.layers
+    return workloads.small_config(args.config, **over)
+
+
 def run_ours(args, world, rank, local):
     import paged_kv_cache_470_b200 as pkv
-    cfg = workloads.CONFIGS[args.config]
-    if args.layers:
-        cfg = workloads.small_config(args.config, n_layers=args.layers)
+    cfg = pick_config(args)
     device = torch.device("cuda", local if world > 1 else 0)
     if args.compute:
         pkv.set_option(pkv.KV_OPT_COMPUTE, {"tensor": 1, "cuda": 2}[args.compute])
@@ -446,7 +460,7 @@ def run_ours(args, world, rank, local):
         kern_ms = iso_ms
         kern_how = "CUDA events around single launches, layers cycled"
     achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
-    traffic = profiled_traffic()
+    traffic = profiled_traffic(cfg)
 
     e2e_ms, h2d, d2h = e2e_measure(wl, max(args.steps // 4, 3), args.warmup, world)
     e2e_ms = dist_max(e2e_ms, world)
@@ -472,12 +486,12 @@ def run_ours(args, world, rank, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": cfg.elem,
         "data": "synthetic",
         "seq_layers_per_s": round(cfg.batch * cfg.n_layers * world / (ms * 1e-3), 1),
         "pct_of_nominal_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
         "pct_of_measured_hbm": round(100 * value / world / peak, 2),
-        "config": {"workload": cfg.name, "config_id": cfg.cid, "layers": cfg.n_layers, "batch": cfg.batch,
+        "config": {"workload": cfg.name, "config_id": cfg.cid, "elem": cfg.elem, "layers": cfg.n_layers, "batch": cfg.batch,
                    "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "block_tokens": 16,
                    "mean_context": round(sum(lens) / len(lens), 1),
                    "kv_bytes_per_step": lb_unique["kv"] * cfg.n_layers,
@@ -514,7 +528,7 @@ def run_reference(args, world, rank):
     """The oracle on the host cores, on bounded samples of the same workload."""
     if rank != 0:
         return
-    cfg = workloads.CONFIGS[args.config]
+    cfg = pick_config(args)
     layout = workloads.draw_layout(cfg)
     total_steps = args.steps + args.warmup
     per_step = max(0.05, min(2.0, args.reference_budget / max(total_steps, 1)))
@@ -534,7 +548,7 @@ def run_reference(args, world, rank):
             "ms_per_step": round(1e3 * s_all / args.steps, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "seq_layers_per_s": round(n_all / s_all, 2),
-            "config": {"workload": cfg.name, "config_id": cfg.cid},
+            "config": {"workload": cfg.name, "config_id": cfg.cid, "elem": cfg.elem},
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -557,6 +571,7 @@ def main(argv=None):
     ap.add_argument("--grid", type=int, default=0, help="decode CTAs per launch (0: one per SM)")
     ap.add_argument("--combine-kernel", action="store_true", help="split-K merge in a separate kernel")
     ap.add_argument("--head-group", type=int, default=0, help="kv heads per work unit (0: auto)")
+    ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16", help="element type of q, K, V and out")
     ap.add_argument("--separate-append", action="store_true",
                     help="append with kv_cache_append, then paged_attention_decode (two launches per layer)")
     args = ap.parse_args(argv)

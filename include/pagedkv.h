@@ -35,13 +35,16 @@
  *   - Return value: KV_OK (0) or a negative kv_status. Argument checks happen on
  *     the host before anything is enqueued; on KV_ERR_ARG nothing is launched.
  *     KV_ERR_CUDA means a launch failed (cudaGetLastError was not cudaSuccess).
- *   - Element type: dtype must be KV_DTYPE_BF16. Head dimension D must be 64 or
- *     128. Block size is fixed at KV_BLOCK_TOKENS = 16 tokens.
+ *   - Element type: dtype is KV_DTYPE_BF16 or KV_DTYPE_FP16 (2 bytes per
+ *     number either way: "Module 23: Serving", section 23.1, equation
+ *     Memory_KV), the same for q, out, the caches and the new tokens of a call.
+ *     Arithmetic is fp32 whatever the element type. Head dimension D must be 64
+ *     or 128. Block size is fixed at KV_BLOCK_TOKENS = 16 tokens.
  *
- * Layouts (row-major):
- *   k_cache, v_cache   [num_blocks][16][Hkv][D]  bf16, one tensor each for K, V
- *   q, out             [B][Hq][D]               bf16
- *   k_new, v_new       [T][Hkv][D]              bf16
+ * Layouts (row-major; "elem" = bf16 or fp16 as dtype says):
+ *   k_cache, v_cache   [num_blocks][16][Hkv][D]  elem, one tensor each for K, V
+ *   q, out             [B][Hq][D]               elem
+ *   k_new, v_new       [T][Hkv][D]              elem
  *   slot_mapping       [T]                      int64; slot = block*16 + offset,
  *                                                negative = padding (skipped)
  *   block_tables       [B][W]                   int32 physical block ids; row b
@@ -130,9 +133,10 @@ KV_API kv_status paged_attention_workspace_init(void *workspace, size_t workspac
  * and j = h / (Hq / Hkv):
  *   K_t = k_cache[block_tables[b][t/16]][t%16][j][:],  V_t likewise, t < c
  *   out[b][h][:] = sum_t softmax_t(scale * <q[b][h], K_t>) V_t
- * computed with fp32 arithmetic (bf16 inputs, bf16 output). c = 0 gives
- * out[b][h][:] = 0. The result does not depend on which physical blocks hold
- * the tokens, only on the logical order, and is bitwise reproducible.
+ * computed with fp32 arithmetic (16-bit inputs and output of the element
+ * type). c = 0 gives out[b][h][:] = 0. The result does not depend on which
+ * physical blocks hold the tokens, only on the logical order, and is bitwise
+ * reproducible.
  *
  * q, out, k_cache, v_cache, block_tables, context_lens, workspace: device
  * pointers (the first four 16-byte aligned, workspace 256-byte aligned).
@@ -165,7 +169,7 @@ KV_API kv_status paged_attention_read_status(const void *workspace, int32_t *sta
  * Append fused into decode: the same result as kv_cache_append(k_new, v_new,
  * k_cache, v_cache, slot_mapping, T = B, ...) followed by
  * paged_attention_decode(...), in one kernel launch. k_new/v_new are
- * [B][Hkv][D] bf16 (16-byte aligned), slot_mapping [B] int64 (device).
+ * [B][Hkv][D] elem (16-byte aligned), slot_mapping [B] int64 (device).
  * Sequence b's new token must be its last cached token: slot_mapping[b] ==
  * block_tables[b][(c-1)/16] * 16 + (c-1) % 16 with c = context_lens[b], and
  * its block must not be read by any other sequence of the batch (true for
@@ -214,7 +218,7 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
 
 /*
  * Process-wide tuning switches (defaults are the tuned choices).
- *   KV_OPT_COMPUTE:   0 auto, 1 tensor cores (mma.sync bf16), 2 CUDA cores
+ *   KV_OPT_COMPUTE:   0 auto, 1 tensor cores (mma.sync, 16-bit inputs), 2 CUDA cores
  *   KV_OPT_COMBINE:   0 split-K merge fused into the last CTA of each work
  *                     item, 1 separate combine kernel
  *   KV_OPT_GRID:      0 auto (CTAs resident on all SMs), n > 0 launch n CTAs

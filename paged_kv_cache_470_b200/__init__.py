@@ -102,14 +102,18 @@ def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
 # ---------------------------------------------------------------------------
 def kv_cache_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                     slot_mapping: torch.Tensor, error_flag: torch.Tensor | None = None, stream=None) -> None:
-    """Scatter k_new/v_new [T,Hkv,D] into the caches [num_blocks,16,Hkv,D] at slot_mapping [T] (int64)."""
+    """Scatter k_new/v_new [T,Hkv,D] into the caches [num_blocks,16,Hkv,D] at slot_mapping [T] (int64).
+
+    All four tensors are bfloat16, or all float16.
+    """
     T, Hkv, D = k_new.shape
     num_blocks = k_cache.shape[0]
+    dt, code = k_cache.dtype, _cache_dtype(k_cache)
     ef = _dev(error_flag, "error_flag", torch.int32) if error_flag is not None else None
     _check("kv_cache_append", _lib.kv_cache_append(
-        _dev(k_new, "k_new", torch.bfloat16), _dev(v_new, "v_new", torch.bfloat16),
-        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
-        _dev(slot_mapping, "slot_mapping", torch.int64), T, num_blocks, Hkv, D, KV_DTYPE_BF16, ef,
+        _dev(k_new, "k_new", dt), _dev(v_new, "v_new", dt),
+        _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(slot_mapping, "slot_mapping", torch.int64), T, num_blocks, Hkv, D, code, ef,
         _stream_handle(stream)))
 
 
@@ -128,16 +132,20 @@ def make_workspace(B: int, Hq: int, Hkv: int, D: int, device=None) -> torch.Tens
 def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                            block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
                            workspace: torch.Tensor, stream=None) -> torch.Tensor:
-    """out[B,Hq,D] = softmax(scale * q K^T) V over each sequence's paged cache."""
+    """out[B,Hq,D] = softmax(scale * q K^T) V over each sequence's paged cache.
+
+    out, q and the caches are all bfloat16, or all float16.
+    """
     B, Hq, D = q.shape
     num_blocks, _, Hkv, Dk = k_cache.shape
     if Dk != D or tuple(out.shape) != (B, Hq, D) or block_tables.dim() != 2 or block_tables.shape[0] != B:
         raise ValueError("shape mismatch")
+    dt, code = k_cache.dtype, _cache_dtype(k_cache)
     _check("paged_attention_decode", _lib.paged_attention_decode(
-        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
-        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(out, "out", dt), _dev(q, "q", dt),
+        _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
-        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), KV_DTYPE_BF16,
+        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
     return out
 
@@ -151,13 +159,14 @@ def paged_attention_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: tor
     num_blocks, _, Hkv, Dk = k_cache.shape
     if Dk != D or tuple(out.shape) != (B, Hq, D) or tuple(k_new.shape) != (B, Hkv, D):
         raise ValueError("shape mismatch")
+    dt, code = k_cache.dtype, _cache_dtype(k_cache)
     _check("paged_attention_decode_append", _lib.paged_attention_decode_append(
-        _dev(out, "out", torch.bfloat16), _dev(q, "q", torch.bfloat16),
-        _dev(k_new, "k_new", torch.bfloat16), _dev(v_new, "v_new", torch.bfloat16),
-        _dev(k_cache, "k_cache", torch.bfloat16), _dev(v_cache, "v_cache", torch.bfloat16),
+        _dev(out, "out", dt), _dev(q, "q", dt),
+        _dev(k_new, "k_new", dt), _dev(v_new, "v_new", dt),
+        _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
         _dev(slot_mapping, "slot_mapping", torch.int64),
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
-        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), KV_DTYPE_BF16,
+        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
     return out
 

@@ -50,7 +50,7 @@ extern "C" kv_status kv_cache_append(const void *k_new, const void *v_new, void 
                                      const int64_t *slot_mapping, int T, int num_blocks, int Hkv, int D, int dtype,
                                      int32_t *error_flag, kv_stream_t stream)
 {
-    if (T < 0 || num_blocks < 1 || Hkv < 1 || dtype != KV_DTYPE_BF16 || (D != 64 && D != 128))
+    if (T < 0 || num_blocks < 1 || Hkv < 1 || (dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_FP16) || (D != 64 && D != 128))
         return KV_ERR_ARG;
     if (T == 0)
         return KV_OK;

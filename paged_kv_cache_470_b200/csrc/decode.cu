@@ -33,11 +33,16 @@
 //
 // Two consumer arithmetic paths:
 //  * tensor cores: S^T[16 tokens x 8 heads] = K_blk * Q^T with
-//    mma.sync.m16n8k16 (bf16 in, fp32 accumulate; the 16 tokens of a block are
+//    mma.sync.m16n8k16 (16-bit in, fp32 accumulate; the 16 tokens of a block are
 //    the M dimension, the kv head's query heads the N dimension), then
-//    O^T[D x 8] += V_blk^T * P^T, with the probabilities split into a bf16
-//    high part and a bf16 residual so that P keeps ~16 significant bits.
-//  * CUDA cores: fp32 FMAs on values unpacked from bf16.
+//    O^T[D x 8] += V_blk^T * P^T, with the probabilities split into a 16-bit
+//    high part and a 16-bit residual so that P keeps ~16 (bf16) or ~22 (fp16)
+//    significant bits.
+//  * CUDA cores: fp32 FMAs on values unpacked from 16 bits.
+//
+// q, the cache and out are all bf16 or all fp16 (the element type E); the
+// cache holds 2 bytes per number either way ("Module 23: Serving", section
+// 23.1).
 #include "pkv_device.cuh"
 #include "pagedkv.h"
 
@@ -56,7 +61,7 @@ constexpr int kThreads = kConsumerThreads + 64;
 constexpr int kPieceQueue = 4;                    // consumer -> helper queue of finished split pieces
 constexpr int kGroupMax = 8;            // query heads per kv head per work item
 constexpr int kMaxHG = 4;               // kv heads per work unit
-constexpr int kHeadTileBytes = 2048;    // one kv head: 16 rows x 64 bf16, 128B-swizzled
+constexpr int kHeadTileBytes = 2048;    // one kv head: 16 rows x 64 elements, 128B-swizzled
 constexpr int kMergeSlots = 4;          // warps that hand their state over per merge round
 constexpr int kCtasPerSm = 1;
 constexpr int kStatusBytes = 256;
@@ -89,8 +94,8 @@ struct Geo {
 };
 
 struct DecodeArgs {
-    __nv_bfloat16 *out;
-    const __nv_bfloat16 *q;
+    uint16_t *out;        // [B][Hq][D] elements of type E
+    const uint16_t *q;    // [B][Hq][D]
     const int32_t *block_tables;
     const int32_t *context_lens;
     float *part_acc;     // [slots][kMaxHG][8][D]
@@ -110,8 +115,8 @@ struct DecodeArgs {
     // fused append (append != 0): this step's token of sequence b is k_new/v_new[b],
     // at slot slots[b], which must be position context_lens[b] - 1 of sequence b
     int append;
-    const uint4 *k_new, *v_new;   // [B][Hkv][D] bf16, as 16-byte chunks
-    uint4 *k_cache, *v_cache;     // [num_blocks][16][Hkv][D] bf16, as 16-byte chunks
+    const uint4 *k_new, *v_new;   // [B][Hkv][D], as 16-byte chunks
+    uint4 *k_cache, *v_cache;     // [num_blocks][16][Hkv][D], as 16-byte chunks
     const int64_t *slots;         // [B]
 };
 
@@ -259,14 +264,14 @@ __device__ __forceinline__ ItemOut item_out(const DecodeArgs &a, const Cursor &c
 // ---------------------------------------------------------------------------
 // Per-warp consumer state and arithmetic (one kv head of each unit).
 // ---------------------------------------------------------------------------
-template <int D, int PATH, int NH>
+template <class E, int D, int PATH, int NH>
 struct Consumer;
 
 // Tensor-core path. Lane (r = lane/4, c = lane%4) holds scores of tokens r and
 // r+8 for query heads 2c and 2c+1, and the accumulator O^T rows d = 16*mt + r
 // (+8) for the same two heads.
-template <int D, int NH>
-struct Consumer<D, kPathMma, NH> {
+template <class E, int D, int NH>
+struct Consumer<E, D, kPathMma, NH> {
     static constexpr int kTiles = D / 64;
     static constexpr int kMt = D / 16;
     static constexpr int kRegs = kMt * 4 + 4;
@@ -327,7 +332,7 @@ struct Consumer<D, kPathMma, NH> {
                 const int tile = kk >> 2, kc = kk & 3;
                 uint32_t af[4];
                 ldmatrix_x4(af, kbase + tile * tile_stride + swz(row, (kc << 1) + (mi >> 1)));
-                mma_bf16_16816(s, af, qf[kk][0], qf[kk][1]);
+                E::mma(s, af, qf[kk][0], qf[kk][1]);
             }
         }
         const bool v0 = r < valid, v1 = (r + 8) < valid;
@@ -349,10 +354,10 @@ struct Consumer<D, kPathMma, NH> {
         const float p2 = exp2f(s2 - mn0), p3 = exp2f(s3 - mn1);
         l0 = l0 * al0 + (p0 + p2);
         l1 = l1 * al1 + (p1 + p3);
-        // P^T as bf16 high part plus bf16 residual, transposed into B fragments
-        const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
-        const uint32_t r01 = pack_bf16x2(p0 - bf16lo_to_f32(h01), p1 - bf16hi_to_f32(h01));
-        const uint32_t r23 = pack_bf16x2(p2 - bf16lo_to_f32(h23), p3 - bf16hi_to_f32(h23));
+        // P^T as a 16-bit high part plus a 16-bit residual, transposed into B fragments
+        const uint32_t h01 = E::pack(p0, p1), h23 = E::pack(p2, p3);
+        const uint32_t r01 = E::pack(p0 - E::lo(h01), p1 - E::hi(h01));
+        const uint32_t r23 = E::pack(p2 - E::lo(h23), p3 - E::hi(h23));
         const uint32_t bh0 = movmatrix_trans(h01), bh1 = movmatrix_trans(h23);
         const uint32_t bl0 = movmatrix_trans(r01), bl1 = movmatrix_trans(r23);
         // O^T [D x 8] += V_blk^T [D x 16] * P^T [16 x 8]
@@ -366,8 +371,8 @@ struct Consumer<D, kPathMma, NH> {
             const int tile = mt >> 2, kc = mt & 3;
             uint32_t af[4];
             ldmatrix_x4_trans(af, vbase + tile * tile_stride + swz(vrow, (kc << 1) + (mi & 1)));
-            mma_bf16_16816(acc[mt], af, bh0, bh1);
-            mma_bf16_16816(acc[mt], af, bl0, bl1);
+            E::mma(acc[mt], af, bh0, bh1);
+            E::mma(acc[mt], af, bl0, bl1);
         }
     }
 
@@ -518,18 +523,18 @@ struct Consumer<D, kPathMma, NH> {
         const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
         const int n0 = 2 * c, n1 = 2 * c + 1;
         const float i0 = 1.f / l0, i1 = 1.f / l1;
-        __nv_bfloat16 *o0 = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n0) * D;
-        __nv_bfloat16 *o1 = o0 + D;
+        uint16_t *o0 = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n0) * D;
+        uint16_t *o1 = o0 + D;
 #pragma unroll
         for (int mt = 0; mt < kMt; ++mt) {
             const int d = mt * 16 + r;
             if (n0 < o.gc) {
-                o0[d] = __float2bfloat16(acc[mt][0] * i0);
-                o0[d + 8] = __float2bfloat16(acc[mt][2] * i0);
+                o0[d] = E::from_f32(acc[mt][0] * i0);
+                o0[d + 8] = E::from_f32(acc[mt][2] * i0);
             }
             if (n1 < o.gc) {
-                o1[d] = __float2bfloat16(acc[mt][1] * i1);
-                o1[d + 8] = __float2bfloat16(acc[mt][3] * i1);
+                o1[d] = E::from_f32(acc[mt][1] * i1);
+                o1[d + 8] = E::from_f32(acc[mt][3] * i1);
             }
         }
     }
@@ -568,12 +573,12 @@ struct Consumer<D, kPathMma, NH> {
 
 // CUDA-core path. QK: lane (t = lane/2, half = lane%2) dots token t's half row
 // with every query head; PV: lane owns D/32 output columns for every head.
-template <int D, int NH>
-struct Consumer<D, kPathSimt, NH> {
-    static constexpr int E = D / 32;
+template <class E, int D, int NH>
+struct Consumer<E, D, kPathSimt, NH> {
+    static constexpr int C = D / 32;     // output columns per lane
     static constexpr int CPH = D / 16;
-    static constexpr int kRegs = NH * E + 2 * NH;
-    float acc[NH][E];
+    static constexpr int kRegs = NH * C + 2 * NH;
+    float acc[NH][C];
     float m[NH], l[NH];
 
     // The CUDA-core path stages the whole item's q in shared memory instead.
@@ -584,7 +589,7 @@ struct Consumer<D, kPathSimt, NH> {
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
 #pragma unroll
-            for (int e = 0; e < E; ++e)
+            for (int e = 0; e < C; ++e)
                 acc[n][e] = 0.f;
             m[n] = -INFINITY;
             l[n] = 0.f;
@@ -605,9 +610,8 @@ struct Consumer<D, kPathSimt, NH> {
         for (int cc = 0; cc < CPH; ++cc) {
             const int dcol = half * (D / 2) + cc * 8;
             const uint4 kv = lds128(kbase + (dcol >> 6) * tile_stride + swz(t, (dcol & 63) >> 3));
-            const float k0 = bf16lo_to_f32(kv.x), k1 = bf16hi_to_f32(kv.x), k2 = bf16lo_to_f32(kv.y),
-                        k3 = bf16hi_to_f32(kv.y), k4 = bf16lo_to_f32(kv.z), k5 = bf16hi_to_f32(kv.z),
-                        k6 = bf16lo_to_f32(kv.w), k7 = bf16hi_to_f32(kv.w);
+            const float k0 = E::lo(kv.x), k1 = E::hi(kv.x), k2 = E::lo(kv.y), k3 = E::hi(kv.y),
+                        k4 = E::lo(kv.z), k5 = E::hi(kv.z), k6 = E::lo(kv.w), k7 = E::hi(kv.w);
             const float *qs = q_s + dcol + half * 4;
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
@@ -643,34 +647,34 @@ struct Consumer<D, kPathSimt, NH> {
                 p_s[t * kGroupMax + n] = p;
         }
         __syncwarp();
-        const int d0 = lane * E;
+        const int d0 = lane * C;
         const uint32_t vcol = (d0 >> 6) * tile_stride;
         const int chunk = (d0 & 63) >> 3, within = d0 & 7;
 #pragma unroll
         for (int n = 0; n < NH; ++n)
 #pragma unroll
-            for (int e = 0; e < E; ++e)
+            for (int e = 0; e < C; ++e)
                 acc[n][e] *= al[n];
         for (int tt = 0; tt < valid; ++tt) {
             const uint32_t addr = vbase + vcol + swz(tt, chunk) + within * 2;
-            float v[E];
-            if constexpr (E == 4) {
+            float v[C];
+            if constexpr (C == 4) {
                 const uint2 w = lds64(addr);
-                v[0] = bf16lo_to_f32(w.x);
-                v[1] = bf16hi_to_f32(w.x);
-                v[2] = bf16lo_to_f32(w.y);
-                v[3] = bf16hi_to_f32(w.y);
+                v[0] = E::lo(w.x);
+                v[1] = E::hi(w.x);
+                v[2] = E::lo(w.y);
+                v[3] = E::hi(w.y);
             } else {
                 const uint32_t w = lds32(addr);
-                v[0] = bf16lo_to_f32(w);
-                v[1] = bf16hi_to_f32(w);
+                v[0] = E::lo(w);
+                v[1] = E::hi(w);
             }
             const float *pr = p_s + tt * kGroupMax;
 #pragma unroll
             for (int n = 0; n < NH; ++n) {
                 const float pn = pr[n];
 #pragma unroll
-                for (int e = 0; e < E; ++e)
+                for (int e = 0; e < C; ++e)
                     acc[n][e] = fmaf(pn, v[e], acc[n][e]);
             }
         }
@@ -692,10 +696,10 @@ struct Consumer<D, kPathSimt, NH> {
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
 #pragma unroll
-            for (int e = 0; e < E; ++e)
-                slot[(n * E + e) * 32 + lane] = acc[n][e];
-            slot[(NH * E + n) * 32 + lane] = m[n];
-            slot[(NH * E + NH + n) * 32 + lane] = l[n];
+            for (int e = 0; e < C; ++e)
+                slot[(n * C + e) * 32 + lane] = acc[n][e];
+            slot[(NH * C + n) * 32 + lane] = m[n];
+            slot[(NH * C + NH + n) * 32 + lane] = l[n];
         }
     }
 
@@ -704,18 +708,18 @@ struct Consumer<D, kPathSimt, NH> {
         const int lane = threadIdx.x & 31;
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
-            const float pm = slot[(NH * E + n) * 32 + lane], pl = slot[(NH * E + NH + n) * 32 + lane];
+            const float pm = slot[(NH * C + n) * 32 + lane], pl = slot[(NH * C + NH + n) * 32 + lane];
             const float M = fmaxf(m[n], pm);
             const float a = rescale(m[n], M), b = rescale(pm, M);
 #pragma unroll
-            for (int e = 0; e < E; ++e)
-                acc[n][e] = acc[n][e] * a + slot[(n * E + e) * 32 + lane] * b;
+            for (int e = 0; e < C; ++e)
+                acc[n][e] = acc[n][e] * a + slot[(n * C + e) * 32 + lane] * b;
             l[n] = l[n] * a + pl * b;
             m[n] = M;
         }
     }
 
-    // As Consumer<D, kPathMma>::merge_solo: same order and arithmetic as merge_pieces_global.
+    // As Consumer<E, D, kPathMma>::merge_solo: same order and arithmetic as merge_pieces_global.
     __device__ __forceinline__ void merge_solo(const DecodeArgs &a, const ItemOut &o, int item, int first_cta,
                                                int last_cta)
     {
@@ -725,9 +729,9 @@ struct Consumer<D, kPathSimt, NH> {
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
             float M = -INFINITY, L = 0.f;
-            float O[E];
+            float O[C];
 #pragma unroll
-            for (int e = 0; e < E; ++e)
+            for (int e = 0; e < C; ++e)
                 O[e] = 0.f;
             for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
                 float mv[kMergeBatch], lv[kMergeBatch];
@@ -753,7 +757,7 @@ struct Consumer<D, kPathSimt, NH> {
                 const float sc = rescale(M, Mb);
                 L *= sc;
 #pragma unroll
-                for (int e = 0; e < E; ++e)
+                for (int e = 0; e < C; ++e)
                     O[e] *= sc;
 #pragma unroll
                 for (int j = 0; j < kMergeBatch; ++j) {
@@ -764,19 +768,19 @@ struct Consumer<D, kPathSimt, NH> {
                         continue;
                     if (cc == self) {
 #pragma unroll
-                        for (int e = 0; e < E; ++e)
+                        for (int e = 0; e < C; ++e)
                             O[e] = fmaf(w, acc[n][e], O[e]);
                     } else {
                         const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase + n;
 #pragma unroll
-                        for (int e = 0; e < E; ++e)
-                            O[e] = fmaf(w, __ldcg(a.part_acc + h * D + lane * E + e), O[e]);
+                        for (int e = 0; e < C; ++e)
+                            O[e] = fmaf(w, __ldcg(a.part_acc + h * D + lane * C + e), O[e]);
                     }
                 }
                 M = Mb;
             }
 #pragma unroll
-            for (int e = 0; e < E; ++e)
+            for (int e = 0; e < C; ++e)
                 acc[n][e] = O[e];
             m[n] = M;
             l[n] = L;
@@ -790,10 +794,10 @@ struct Consumer<D, kPathSimt, NH> {
         for (int n = 0; n < NH; ++n) {
             if (n < o.gc) {
                 const float inv = 1.f / l[n];
-                __nv_bfloat16 *dst = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n) * D + lane * E;
+                uint16_t *dst = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n) * D + lane * C;
 #pragma unroll
-                for (int e = 0; e < E; ++e)
-                    dst[e] = __float2bfloat16(acc[n][e] * inv);
+                for (int e = 0; e < C; ++e)
+                    dst[e] = E::from_f32(acc[n][e] * inv);
             }
         }
     }
@@ -805,9 +809,9 @@ struct Consumer<D, kPathSimt, NH> {
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
             if (n < o.gc) {
-                float *dst = a.part_acc + (head0 + n) * D + lane * E;
+                float *dst = a.part_acc + (head0 + n) * D + lane * C;
 #pragma unroll
-                for (int e = 0; e < E; ++e)
+                for (int e = 0; e < C; ++e)
                     dst[e] = acc[n][e];
                 if (lane == 0) {
                     a.part_ml[(head0 + n) * 2] = m[n];
@@ -823,7 +827,7 @@ struct Consumer<D, kPathSimt, NH> {
 // thread merges two groups of four output columns at a time, and all loads
 // for up to four pieces are issued before any is used, so a merge costs
 // about one memory round trip per four pieces.
-template <int D>
+template <class E, int D>
 __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int item, int first_cta, int last_cta,
                                                     int b, int k, int tid, int nthreads)
 {
@@ -900,11 +904,9 @@ __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int ite
             const int hh = static_cast<int>(head[e] / kGroupMax), n = static_cast<int>(head[e] % kGroupMax);
             const int h = (hg * a.hg + hh) * a.group + hc * kGroupMax + n;
             const float inv = 1.f / L[e];
-            __nv_bfloat162 lo = __floats2bfloat162_rn(O[e].x * inv, O[e].y * inv);
-            __nv_bfloat162 hi = __floats2bfloat162_rn(O[e].z * inv, O[e].w * inv);
             uint2 packed;
-            packed.x = *reinterpret_cast<uint32_t *>(&lo);
-            packed.y = *reinterpret_cast<uint32_t *>(&hi);
+            packed.x = E::pack(O[e].x * inv, O[e].y * inv);
+            packed.y = E::pack(O[e].z * inv, O[e].w * inv);
             *reinterpret_cast<uint2 *>(a.out + (static_cast<size_t>(b) * a.Hq + h) * D + col[e]) = packed;
         }
     }
@@ -977,9 +979,9 @@ __device__ __forceinline__ void zero_empty_outputs(const DecodeArgs &a, int tid,
         if (c < 0 || c > a.W * kBlockTokens)
             atomicOr(a.status, KV_STATUS_BAD_CONTEXT);
         if (clamp_ctx(c, a.W) == 0) {
-            __nv_bfloat16 *o = a.out + static_cast<size_t>(b) * a.Hq * D;
+            uint16_t *o = a.out + static_cast<size_t>(b) * a.Hq * D;
             for (int i = 0; i < a.Hq * D; ++i)
-                o[i] = __float2bfloat16(0.f);
+                o[i] = 0;  // +0.0 in both element types
         }
     }
 }
@@ -999,7 +1001,7 @@ __device__ __forceinline__ int load_block_ids(const DecodeArgs &a, const Cursor 
     return blk;
 }
 
-template <int D, int PATH, int NH>
+template <class E, int D, int PATH, int NH>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeArgs a)
@@ -1185,7 +1187,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             last = __shfl_sync(kFull, last, 0);
             if (last) {
-                merge_pieces_global<D>(a, item, first_cta, last_cta, b, kk, lane, 32);
+                merge_pieces_global<E, D>(a, item, first_cta, last_cta, b, kk, lane, 32);
                 __syncwarp();
                 if (lane == 0)
                     a.counters[item] = 0;
@@ -1201,7 +1203,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int hh = warp % a.hg;          // kv head within the group
     const int stream = warp / a.hg;      // which units: u % streams == stream
     const int NS = a.streams;
-    Consumer<D, PATH, NH> st;
+    Consumer<E, D, PATH, NH> st;
     float *q_s = scratch + hh * kGroupMax * G::kQStride;                         // CUDA-core path only
     float *p_s = scratch + kMaxHG * kGroupMax * G::kQStride + warp * 16 * kGroupMax;
     st.prefetch_q(a, item_out(a, cur0, hh));  // q is never written by this library: no wait needed
@@ -1237,8 +1239,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int rem = idx - h2 * per;
                 const int n = rem / D, d = rem - n * D;
                 const int h = (hg * a.hg + h2) * a.group + hc * kGroupMax + n;
-                const float v = (n < o.gc) ? __bfloat162float(a.q[(static_cast<size_t>(cur.b) * a.Hq + h) * D + d])
-                                           : 0.f;
+                const float v = (n < o.gc) ? E::to_f32(a.q[(static_cast<size_t>(cur.b) * a.Hq + h) * D + d]) : 0.f;
                 scratch[(h2 * kGroupMax + n) * G::kQStride + d + ((d >= D / 2) ? 4 : 0)] = v;
             }
             named_barrier(1, kConsumerThreads);
@@ -1296,10 +1297,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int slot_giver = (stream / (2 * step)) * a.hg + hh;
             const int slot_taker = ((stream + step) / (2 * step)) * a.hg + hh;
             if (giver)
-                st.save(scratch + slot_giver * Consumer<D, PATH, NH>::kRegs * 32);
+                st.save(scratch + slot_giver * Consumer<E, D, PATH, NH>::kRegs * 32);
             named_barrier(1, kConsumerThreads);
             if (taker)
-                st.merge(scratch + slot_taker * Consumer<D, PATH, NH>::kRegs * 32);
+                st.merge(scratch + slot_taker * Consumer<E, D, PATH, NH>::kRegs * 32);
             named_barrier(1, kConsumerThreads);
         }
 
@@ -1350,7 +1351,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 }
                 named_barrier(1, kConsumerThreads);
                 if (misc[kMiscLast]) {
-                    merge_pieces_global<D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads);
+                    merge_pieces_global<E, D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads);
                     if (tid == 0)
                         a.counters[item] = 0;
                 }
@@ -1374,7 +1375,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // Separate split-K combine: one CTA per work item.
-template <int D>
+template <class E, int D>
 __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int grid_ctas)
 {
     __shared__ int red[2][4];
@@ -1411,7 +1412,7 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int gr
     const int first_cta = item_start / chunk, last_cta = (item_start + n - 1) / chunk;
     if (first_cta == last_cta)
         return;
-    merge_pieces_global<D>(a, item, first_cta, last_cta, b, k, threadIdx.x, 128);
+    merge_pieces_global<E, D>(a, item, first_cta, last_cta, b, k, threadIdx.x, 128);
 }
 
 }  // namespace pkv
@@ -1505,7 +1506,7 @@ EncodeTiledFn encode_fn()
 // are (column, row, kv head, block) -- rows inside heads, so each head's 16
 // rows land as one contiguous 128B-swizzled 2 KB tile -- with a box of
 // 64 columns x 16 rows x HG heads x 1 block.
-bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv, int D, int hg)
+bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv, int D, int hg, int dtype)
 {
     EncodeTiledFn enc = encode_fn();
     if (!enc)
@@ -1516,25 +1517,22 @@ bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv,
                                    static_cast<cuuint64_t>(16) * Hkv * D * 2};
     const cuuint32_t box[4] = {64, 16, static_cast<cuuint32_t>(hg), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(cache), dims, strides, box, estr,
+    const CUtensorMapDataType dt =
+        dtype == KV_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(tm, dt, 4, const_cast<void *>(cache), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 using DecodeFn = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
 
-template <int D, int PATH, int NH>
-struct KernelInfo {
-    static DecodeFn fn() { return decode_kernel<D, PATH, NH>; }
-    static int smem() { return Geo<D>::kSmemBytes; }
-};
-
-DecodeFn pick_kernel(int D, int path, int nh, int *smem)
+template <class E>
+DecodeFn pick_kernel_for(int D, int path, int nh, int *smem)
 {
 #define PKV_CASE(DD, PP, NN)                          \
     if (D == DD && path == PP && nh == NN) {          \
-        *smem = KernelInfo<DD, PP, NN>::smem();       \
-        return KernelInfo<DD, PP, NN>::fn();          \
+        *smem = Geo<DD>::kSmemBytes;                  \
+        return decode_kernel<E, DD, PP, NN>;          \
     }
     PKV_CASE(64, kPathMma, 8)
     PKV_CASE(128, kPathMma, 8)
@@ -1548,6 +1546,12 @@ DecodeFn pick_kernel(int D, int path, int nh, int *smem)
     PKV_CASE(128, kPathSimt, 8)
 #undef PKV_CASE
     return nullptr;
+}
+
+DecodeFn pick_kernel(int dtype, int D, int path, int nh, int *smem)
+{
+    return dtype == KV_DTYPE_FP16 ? pick_kernel_for<ElemF16>(D, path, nh, smem)
+                                  : pick_kernel_for<ElemBf16>(D, path, nh, smem);
 }
 
 // Per (kernel, device): dynamic shared memory opted in, and resident CTAs per SM.
@@ -1607,7 +1611,7 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
                              int Hkv, int D, float scale, int dtype, void *workspace, size_t workspace_bytes,
                              kv_stream_t stream)
 {
-    if (dtype != KV_DTYPE_BF16 || B < 0 || max_blocks_per_seq < 1 || num_blocks < 1 || Hq < 1 || Hkv < 1 ||
+    if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_FP16) || B < 0 || max_blocks_per_seq < 1 || num_blocks < 1 || Hq < 1 || Hkv < 1 ||
         Hq % Hkv != 0 || (D != 64 && D != 128))
         return KV_ERR_ARG;
     if (B == 0)
@@ -1642,7 +1646,7 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
         nh = gmin <= 1 ? 1 : gmin <= 2 ? 2 : gmin <= 4 ? 4 : 8;
     }
     int smem = 0;
-    DecodeFn fn = pick_kernel(D, path, nh, &smem);
+    DecodeFn fn = pick_kernel(dtype, D, path, nh, &smem);
     if (!fn)
         return KV_ERR_ARG;
     const int occ = prepare_kernel(fn, smem, dev);
@@ -1670,14 +1674,14 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
         return KV_ERR_ARG;
 
     CUtensorMap tmK, tmV;
-    if (!make_cache_map(&tmK, k_cache, num_blocks, Hkv, D, hg) ||
-        !make_cache_map(&tmV, v_cache, num_blocks, Hkv, D, hg))
+    if (!make_cache_map(&tmK, k_cache, num_blocks, Hkv, D, hg, dtype) ||
+        !make_cache_map(&tmV, v_cache, num_blocks, Hkv, D, hg, dtype))
         return KV_ERR_CUDA;
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
     DecodeArgs a;
-    a.out = static_cast<__nv_bfloat16 *>(out);
-    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.out = static_cast<uint16_t *>(out);
+    a.q = static_cast<const uint16_t *>(q);
     a.block_tables = block_tables;
     a.context_lens = context_lens;
     a.part_acc = reinterpret_cast<float *>(ws + L.off_acc);
@@ -1733,8 +1737,13 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
         c2.stream = st;
         c2.attrs = attr;
         c2.numAttrs = 1;
-        cudaError_t e = (D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<64>, a, grid)
-                                  : cudaLaunchKernelEx(&c2, combine_kernel<128>, a, grid);
+        cudaError_t e;
+        if (dtype == KV_DTYPE_FP16)
+            e = (D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<ElemF16, 64>, a, grid)
+                          : cudaLaunchKernelEx(&c2, combine_kernel<ElemF16, 128>, a, grid);
+        else
+            e = (D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<ElemBf16, 64>, a, grid)
+                          : cudaLaunchKernelEx(&c2, combine_kernel<ElemBf16, 128>, a, grid);
         if (e != cudaSuccess)
             return KV_ERR_CUDA;
     }

@@ -1,10 +1,12 @@
 // Device-side building blocks for the paged KV cache kernels (sm_100a):
 // mbarrier waits with a time limit, TMA tile loads, programmatic dependent
-// launch, warp-level bf16 tensor-core MMA and register transposes.
+// launch, warp-level bf16/fp16 tensor-core MMA and register transposes, and
+// the two 16-bit element types of the cache.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -153,6 +155,58 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 }
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// D[16x8] += A[16x16] * B[16x8], fp16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Element types of q, the cache and out. A 32-bit word holds two elements,
+// the lower-addressed one in its low half. Conversions to 16 bits round to
+// nearest even.
+struct ElemBf16 {
+    static constexpr int kDtype = 0;  // KV_DTYPE_BF16
+    __device__ static __forceinline__ float lo(uint32_t w) { return bf16lo_to_f32(w); }
+    __device__ static __forceinline__ float hi(uint32_t w) { return bf16hi_to_f32(w); }
+    __device__ static __forceinline__ float to_f32(uint16_t x) { return __uint_as_float(static_cast<uint32_t>(x) << 16); }
+    __device__ static __forceinline__ uint32_t pack(float l, float h) { return pack_bf16x2(l, h); }
+    __device__ static __forceinline__ uint16_t from_f32(float x)
+    {
+        return __bfloat16_as_ushort(__float2bfloat16(x));
+    }
+    __device__ static __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+    {
+        mma_bf16_16816(d, a, b0, b1);
+    }
+};
+
+struct ElemF16 {
+    static constexpr int kDtype = 1;  // KV_DTYPE_FP16
+    __device__ static __forceinline__ float lo(uint32_t w)
+    {
+        return __half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xffffu)));
+    }
+    __device__ static __forceinline__ float hi(uint32_t w)
+    {
+        return __half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)));
+    }
+    __device__ static __forceinline__ float to_f32(uint16_t x) { return __half2float(__ushort_as_half(x)); }
+    __device__ static __forceinline__ uint32_t pack(float l, float h)
+    {
+        __half2 v = __floats2half2_rn(l, h);
+        return *reinterpret_cast<uint32_t *>(&v);
+    }
+    __device__ static __forceinline__ uint16_t from_f32(float x) { return __half_as_ushort(__float2half_rn(x)); }
+    __device__ static __forceinline__ void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+    {
+        mma_f16_16816(d, a, b0, b1);
+    }
+};
 
 // Named barrier over the first `threads` threads of the CTA (id 0 is __syncthreads).
 __device__ __forceinline__ void named_barrier(int id, int threads)

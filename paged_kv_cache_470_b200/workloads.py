@@ -58,6 +58,11 @@ class DecodeConfig:
     redraw_fraction: float = 0.0
     lognormal_mean: float = 0.0
     lognormal_sigma: float = 0.0
+    elem: str = "bf16"            # element type of q, K, V and out: "bf16" or "fp16"
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float16 if self.elem == "fp16" else torch.bfloat16
 
     @property
     def group(self) -> int:
@@ -186,26 +191,27 @@ def draw_layout(cfg: DecodeConfig, context_lens=None, seed=None) -> BatchLayout:
                        prefix, order[cursor:])
 
 
-def random_bf16(shape, gen: torch.Generator, device) -> torch.Tensor:
-    """N(0, 1) drawn in fp32 on ``device`` and rounded to bf16."""
+def random_bf16(shape, gen: torch.Generator, device, dtype=torch.bfloat16) -> torch.Tensor:
+    """N(0, 1) drawn in fp32 on ``device`` and rounded to bf16 (or to ``dtype``)."""
     x = torch.empty(shape, dtype=torch.float32, device=device)
     x.normal_(0.0, 1.0, generator=gen)
-    return x.to(torch.bfloat16)
+    return x.to(dtype)
 
 
-def make_layer_cache(num_blocks: int, Hkv: int, D: int, gen: torch.Generator, device):
-    """One layer's K and V pools, [num_blocks, 16, Hkv, D] bf16 each, every byte random."""
-    k = random_bf16((num_blocks, BLOCK_TOKENS, Hkv, D), gen, device)
-    v = random_bf16((num_blocks, BLOCK_TOKENS, Hkv, D), gen, device)
+def make_layer_cache(num_blocks: int, Hkv: int, D: int, gen: torch.Generator, device, dtype=torch.bfloat16):
+    """One layer's K and V pools, [num_blocks, 16, Hkv, D] bf16 (or dtype) each, every byte random."""
+    k = random_bf16((num_blocks, BLOCK_TOKENS, Hkv, D), gen, device, dtype)
+    v = random_bf16((num_blocks, BLOCK_TOKENS, Hkv, D), gen, device, dtype)
     return k, v
 
 
 def make_step_inputs(cfg: DecodeConfig, gen: torch.Generator, device, n_layers=None):
-    """Per-layer q [B,Hq,D] and new-token K/V [B,Hkv,D], all bf16."""
+    """Per-layer q [B,Hq,D] and new-token K/V [B,Hkv,D], all of the config's element type."""
     L = cfg.n_layers if n_layers is None else n_layers
-    q = random_bf16((L, cfg.batch, cfg.Hq, cfg.D), gen, device)
-    k_new = random_bf16((L, cfg.batch, cfg.Hkv, cfg.D), gen, device)
-    v_new = random_bf16((L, cfg.batch, cfg.Hkv, cfg.D), gen, device)
+    dt = cfg.torch_dtype
+    q = random_bf16((L, cfg.batch, cfg.Hq, cfg.D), gen, device, dt)
+    k_new = random_bf16((L, cfg.batch, cfg.Hkv, cfg.D), gen, device, dt)
+    v_new = random_bf16((L, cfg.batch, cfg.Hkv, cfg.D), gen, device, dt)
     return q, k_new, v_new
 
 

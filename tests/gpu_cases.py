@@ -21,7 +21,7 @@ class Case:
         gen = workloads.device_generator(cfg.seed if seed is None else seed, device)
         self.k, self.v = [], []
         for _ in range(n_layers):
-            k, v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device)
+            k, v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device, cfg.torch_dtype)
             self.k.append(k)
             self.v.append(v)
         self.q, self.k_new, self.v_new = workloads.make_step_inputs(cfg, gen, device, n_layers)
@@ -42,7 +42,7 @@ def oracle_step(oracle_mod, case, layer, host=None):
     q, k, v, kn, vn = host if host is not None else case.host_inputs(layer)
     k2, v2 = oracle_mod.kv_cache_append(k, v, kn, vn, case.layout.slot_mapping().numpy())
     out = oracle_mod.paged_attention_decode(q, k2, v2, case.layout.block_tables.numpy(),
-                                            case.layout.context_lens.numpy(), case.cfg.scale)
+                                            case.layout.context_lens.numpy(), case.cfg.scale, dtype=case.cfg.elem)
     return k2, v2, out
 
 
