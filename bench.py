@@ -31,6 +31,7 @@ import hashlib
 import json
 import math
 import os
+import random
 import re
 import statistics
 import sys
@@ -330,6 +331,53 @@ def decode_kernel_duration_ms(wl, reps=5):
     return sum(times) / len(times), len(times)
 
 
+def block_moves_measure(wl, peak, reps=10):
+    """Whole-block moves over every layer's K and V cache, one launch per call: swap-out staging (gather) and
+    swap-in (scatter) of the blocks of a tenth of the batch's sequences, and copy-on-write copies of as many of
+    them into free blocks. Algorithmic bytes = every moved block read once and written once. Not part of the
+    timed step; the scatter writes back the bytes the gather read, the copies land in blocks no table uses."""
+    pkv, cfg, layout = wl.pkv, wl.cfg, wl.layout
+    rng = random.Random(cfg.seed)
+    lens = layout.context_lens.tolist()
+    tables = layout.block_tables
+    victims = rng.sample(range(cfg.batch), max(1, cfg.batch // 10))
+    ids = [int(x) for b in victims for x in tables[b, :-(-lens[b] // 16)].tolist()]
+    used = set(int(x) for x in tables.flatten().tolist() if x >= 0)
+    free = [i for i in range(layout.num_blocks) if i not in used]
+    caches = [t for layer in range(cfg.n_layers) for t in (wl.k[layer], wl.v[layer])]
+    dev = wl.q.device
+    blk_bytes = 16 * cfg.Hkv * cfg.D * wl.k[0].element_size()
+    ids_d = torch.tensor(ids, dtype=torch.int32, device=dev)
+    n_copy = min(len(ids), len(free))
+    src_d = ids_d[:n_copy].contiguous()
+    dst_d = torch.tensor(free[:n_copy], dtype=torch.int32, device=dev)
+    staged = torch.empty((len(caches), len(ids), 16, cfg.Hkv, cfg.D), dtype=wl.k[0].dtype, device=dev)
+    flag = torch.zeros(1, dtype=torch.int32, device=dev)
+    ops = {"gather": (lambda: pkv.kv_cache_gather_blocks(staged, caches, ids_d, error_flag=flag), len(ids)),
+           "scatter": (lambda: pkv.kv_cache_scatter_blocks(caches, staged, ids_d, error_flag=flag), len(ids)),
+           "copy": (lambda: pkv.kv_cache_copy_blocks(caches, src_d, dst_d, error_flag=flag), n_copy)}
+    res = {"blocks_swapped": len(ids), "blocks_copied": n_copy, "tensors": len(caches), "bytes_per_block": blk_bytes,
+           "timing": "CUDA events, mean of %d launches after 2 warm-up launches" % reps}
+    stream = torch.cuda.current_stream()
+    for name, (fn, n) in ops.items():
+        if n == 0:
+            continue
+        for _ in range(2):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        gbs = 2 * n * len(caches) * blk_bytes / (ms * 1e-3) / 1e9
+        res[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 1), "frac": round(gbs / peak, 4)}
+    res["status"] = int(flag.item())
+    del staged
+    return res
+
+
 def e2e_measure(wl, steps, warmup, world):
     """The same step through the C ABI with host buffers: H2D of the step's inputs, D2H of its outputs."""
     cfg = wl.cfg
@@ -419,6 +467,8 @@ def run_ours(args, world, rank, local):
         pkv.set_option(pkv.KV_OPT_COMBINE, 1)
     if args.head_group:
         pkv.set_option(pkv.KV_OPT_HEAD_GROUP, args.head_group)
+    if args.item_cost:
+        pkv.set_option(pkv.KV_OPT_ITEM_COST, args.item_cost)
     if args.profile_step:
         return run_profile_step(args, cfg, device)
     wl = Workload(cfg, device, rank)
@@ -463,6 +513,7 @@ def run_ours(args, world, rank, local):
     traffic = profiled_traffic(cfg)
 
     e2e_ms, h2d, d2h = e2e_measure(wl, max(args.steps // 4, 3), args.warmup, world)
+    moves = block_moves_measure(wl, peak)
     e2e_ms = dist_max(e2e_ms, world)
 
     cpu = None
@@ -519,6 +570,7 @@ def run_ours(args, world, rank, local):
         "clocks": clk.summary(),
         "device_status": status,
         "cpu_baseline": cpu,
+        "block_moves": moves,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -571,6 +623,8 @@ def main(argv=None):
     ap.add_argument("--grid", type=int, default=0, help="decode CTAs per launch (0: one per SM)")
     ap.add_argument("--combine-kernel", action="store_true", help="split-K merge in a separate kernel")
     ap.add_argument("--head-group", type=int, default=0, help="kv heads per work unit (0: auto)")
+    ap.add_argument("--item-cost", type=int, default=0,
+                    help="work positions charged per work item when dividing work between CTAs (0 auto, -1 none)")
     ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16", help="element type of q, K, V and out")
     ap.add_argument("--separate-append", action="store_true",
                     help="append with kv_cache_append, then paged_attention_decode (two launches per layer)")

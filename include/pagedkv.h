@@ -223,13 +223,18 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
  *                     item, 1 separate combine kernel
  *   KV_OPT_GRID:      0 auto (CTAs resident on all SMs), n > 0 launch n CTAs
  *                     (n is capped by what the workspace was sized for)
- *   KV_OPT_MIN_CHUNK: 0 auto, n > 0 minimum work units (KV blocks of one
- *                     kv-head group) per CTA
+ *   KV_OPT_MIN_CHUNK: 0 auto, n > 0 minimum work positions per CTA
  *   KV_OPT_PRODUCER_LANES: 0 auto, 1/2/4/8 lanes of the producer warp that
  *                     issue tile loads
  *   KV_OPT_HEAD_GROUP: 0 auto (4 if it divides Hkv, else 2 or 1), or 1/2/4 kv
  *                     heads per work unit when it divides Hkv. It changes
  *                     paged_attention_workspace_size: set it before sizing.
+ *   KV_OPT_ITEM_COST: how the work is divided between CTAs. Every work unit
+ *                     (one KV block of one kv-head group) is one work
+ *                     position and every work item (a sequence's kv-head
+ *                     group and query-head chunk) adds this many more for its
+ *                     fixed cost; CTAs take equal ranges of positions.
+ *                     0 auto, -1 none, 1..64 that many.
  * Returns KV_ERR_ARG for an unknown key or value.
  */
 #define KV_OPT_COMPUTE 1
@@ -238,6 +243,7 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
 #define KV_OPT_MIN_CHUNK 4
 #define KV_OPT_PRODUCER_LANES 5
 #define KV_OPT_HEAD_GROUP 6
+#define KV_OPT_ITEM_COST 7
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

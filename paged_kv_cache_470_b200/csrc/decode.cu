@@ -89,7 +89,7 @@ struct Geo {
     static constexpr int kOffBar = kOffScratch + kScratchBytes;
     static constexpr int kOffQBar = kOffBar + 2 * kMaxStages * 8;    // piece queue: full[4], empty[4]
     static constexpr int kOffMisc = kOffQBar + 2 * kPieceQueue * 8;
-    static constexpr int kMiscInts = 48;
+    static constexpr int kMiscInts = 64;
     static constexpr int kSmemBytes = kOffMisc + kMiscInts * 4 + 1024;  // + room to align the base
 };
 
@@ -110,6 +110,7 @@ struct DecodeArgs {
     int stages, stage_bytes, tile_stride;  // ring geometry; tile_stride = HG * 2048
     int prod_lanes;      // producer lanes issuing TMA
     int min_chunk;
+    int item_cost;       // work positions charged per work item on top of its units
     int fused;
     float scale_log2;    // scale * log2(e)
     // fused append (append != 0): this step's token of sequence b is k_new/v_new[b],
@@ -124,12 +125,17 @@ struct DecodeArgs {
 enum {
     kMiscAbort = 0,
     kMiscLocB = 1,
-    kMiscLocR = 2,
     kMiscSolo = 3,      // this piece's item has all its other pieces finished
     kMiscZero = 4,
     kMiscLast = 5,      // the CTA's final piece completed its item: merge it
-    kMiscWarpSums = 6,  // 10 ints
     kMiscQueue = 16,    // kPieceQueue descriptors of 5 ints: item, first cta, last cta, b, k
+    kMiscLocK = 36,     // item and block offset of the CTA's first unit (sequence in kMiscLocB)
+    kMiscLocOff = 37,
+    kMiscLocPos = 38,   // work position of that item's first unit
+    kMiscStartU = 39,   // units before the CTA's range, and before its end
+    kMiscEndU = 40,
+    kMiscEndFound = 41,
+    kMiscScan64 = 44,   // 10 64-bit warp sums (ints 44..63)
 };
 
 __device__ __forceinline__ int clamp_ctx(int c, int W)
@@ -140,23 +146,23 @@ __device__ __forceinline__ int seq_ctx(const DecodeArgs &a, int b) { return clam
 __device__ __forceinline__ int ctx_blocks(int c) { return (c + kBlockTokens - 1) / kBlockTokens; }
 
 // Inclusive scan over all kThreads threads; *total receives the sum.
-__device__ __forceinline__ int block_scan_incl(int v, volatile int *warp_sums, int *total)
+__device__ __forceinline__ long long block_scan_incl64(long long v, volatile long long *warp_sums, long long *total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int x = v;
+    long long x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(kFull, x, o);
+        const long long y = __shfl_up_sync(kFull, x, o);
         if (lane >= o)
             x += y;
     }
     if (lane == 31)
         warp_sums[warp] = x;
     __syncthreads();
-    int pre = 0, tot = 0;
+    long long pre = 0, tot = 0;
 #pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) {
-        const int s = warp_sums[w];
+        const long long s = warp_sums[w];
         pre += (w < warp) ? s : 0;
         tot += s;
     }
@@ -165,16 +171,30 @@ __device__ __forceinline__ int block_scan_incl(int v, volatile int *warp_sums, i
     return x + pre;
 }
 
+// Work positions. The units of all items are laid end to end, and each item of
+// a non-empty sequence is preceded by a.item_cost positions that stand for its
+// fixed cost (query loads, the merge of the consumer streams, the store or the
+// split-K hand-off). CTAs take equal ranges of positions, so a CTA that starts
+// more items gets fewer units. Per sequence, the scan carries
+// (positions << 24) + (1 if the sequence has blocks).
+constexpr int kNonEmptyBits = 24;
+__device__ __forceinline__ long long seq_scan_value(const DecodeArgs &a, int n)
+{
+    return n > 0 ? ((static_cast<long long>(a.items_per_seq) * (n + a.item_cost)) << kNonEmptyBits) + 1 : 0;
+}
+
 struct Cursor {
     int b;     // sequence
     int k;     // item within the sequence: head group * hchunks + query-head chunk
     int off;   // block offset within the sequence
     int ctx;   // tokens of sequence b (clamped)
     int n;     // blocks of sequence b
+    int pos;   // work position of the item's first unit
 };
 
 __device__ __forceinline__ void cursor_next_item(const DecodeArgs &a, Cursor &c)
 {
+    c.pos += c.n + a.item_cost;
     c.off = 0;
     if (++c.k == a.items_per_seq) {
         c.k = 0;
@@ -212,21 +232,22 @@ __device__ __forceinline__ void sts128_zero(uint32_t addr)
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside one head's 128B-swizzled tile.
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
-// Split-K counters. A finished piece releases its partial with a release
-// atomic (the writes of the other threads are ordered before it by a bar.sync);
-// a CTA that observes a count (relaxed load or the atomic's result) and then
-// merges issues an acquire fence first. Neither the relaxed load nor the
-// release atomic makes the issuing thread wait for the round trip.
+// Split-K counters. A finished piece is counted in with an acq_rel atomic (the
+// writes of its other threads are ordered before it by a bar.sync); the one
+// whose count completes the item has, by the same atomic, acquired the other
+// pieces' partials. A CTA that sees a complete count by a relaxed load (read
+// early, so the load's round trip is hidden) issues an acquire fence before
+// merging.
 __device__ __forceinline__ int ld_relaxed_gpu(const int32_t *p)
 {
     int v;
     asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ int atom_add_release_gpu(int32_t *p, int v)
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int32_t *p, int v)
 {
     int prev;
-    asm volatile("atom.release.gpu.global.add.s32 %0, [%1], %2;" : "=r"(prev) : "l"(p), "r"(v) : "memory");
+    asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(prev) : "l"(p), "r"(v) : "memory");
     return prev;
 }
 __device__ __forceinline__ void fence_acquire_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
@@ -1030,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mbar_fence_init();
         misc[kMiscAbort] = 0;
         misc[kMiscLocB] = -1;
-        misc[kMiscLocR] = 0;
+        misc[kMiscEndFound] = 0;
         misc[kMiscZero] = 0;
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -1040,37 +1061,52 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     __syncthreads();
 
     // ---- split plan (reads only tables and lengths: no wait needed yet) ----
-    int my_blocks = 0;
+    volatile long long *scan64 = reinterpret_cast<volatile long long *>(misc + kMiscScan64);
+    const int w = a.item_cost;
+    long long mine = 0;
     for (int b = tid; b < a.B; b += kThreads)
-        my_blocks += ctx_blocks(seq_ctx(a, b));
-    int sum_blocks;
-    block_scan_incl(my_blocks, misc + kMiscWarpSums, &sum_blocks);
-    const int total = sum_blocks * a.items_per_seq;
+        mine += seq_scan_value(a, ctx_blocks(seq_ctx(a, b)));
+    long long sum64;
+    block_scan_incl64(mine, scan64, &sum64);
+    const int total = static_cast<int>(sum64 >> kNonEmptyBits);  // work positions
     int chunk = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
     if (chunk < a.min_chunk)
         chunk = a.min_chunk;
     const int start = static_cast<int>(blockIdx.x) * chunk;
-    const int count = min(chunk, total - start);
+    const int end = min(start + chunk, total);
 
-    if (count > 0) {
-        int running = 0;
+    if (start < total) {
+        // locate the CTA's first unit and count the units in [start, end)
+        long long running = 0;
         for (int base_b = 0; base_b < a.B; base_b += kThreads) {
             const int b = base_b + tid;
             const int n = (b < a.B) ? ctx_blocks(seq_ctx(a, b)) : 0;
-            int tot;
-            const int incl = block_scan_incl(n, misc + kMiscWarpSums, &tot);
-            const int lo = (running + incl - n) * a.items_per_seq;
-            const int hi = (running + incl) * a.items_per_seq;
+            const long long v = seq_scan_value(a, n);
+            long long tot;
+            const long long before = running + block_scan_incl64(v, scan64, &tot) - v;
+            const int lo = static_cast<int>(before >> kNonEmptyBits);
+            const int hi = lo + static_cast<int>(v >> kNonEmptyBits);
+            const int units_before = lo - w * a.items_per_seq * static_cast<int>(before & ((1 << kNonEmptyBits) - 1));
             if (n > 0 && start >= lo && start < hi) {
+                const int r = start - lo, k = r / (n + w), rr = r - k * (n + w);
                 misc[kMiscLocB] = b;
-                misc[kMiscLocR] = start - lo;
+                misc[kMiscLocK] = k;
+                misc[kMiscLocOff] = max(0, rr - w);
+                misc[kMiscLocPos] = lo + k * (n + w) + w;
+                misc[kMiscStartU] = units_before + k * n + max(0, rr - w);
+            }
+            if (n > 0 && end - 1 >= lo && end - 1 < hi) {
+                const int r = end - 1 - lo, k = r / (n + w), rr = r - k * (n + w);
+                misc[kMiscEndU] = units_before + k * n + max(0, rr - w) + (rr >= w ? 1 : 0);
+                misc[kMiscEndFound] = 1;
             }
             running += tot;
             __syncthreads();
-            if (misc[kMiscLocB] >= 0)
+            if (misc[kMiscEndFound])
                 break;
         }
     }
+    const int count = start < total ? misc[kMiscEndU] - misc[kMiscStartU] : 0;
 
     if (count <= 0) {
         grid_dependency_wait();
@@ -1084,11 +1120,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     cur0.b = misc[kMiscLocB];
     cur0.ctx = seq_ctx(a, cur0.b);
     cur0.n = ctx_blocks(cur0.ctx);
-    {
-        const int r = misc[kMiscLocR];
-        cur0.k = r / cur0.n;
-        cur0.off = r - cur0.k * cur0.n;
-    }
+    cur0.k = misc[kMiscLocK];
+    cur0.off = misc[kMiscLocOff];
+    cur0.pos = misc[kMiscLocPos];
     volatile int *abort_flag = misc + kMiscAbort;
     const uint32_t ring = base_s;
 
@@ -1181,9 +1215,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 break;
             int last = 0;
             if (lane == 0) {
-                last = atom_add_release_gpu(a.counters + item, 1) == last_cta - first_cta;
-                if (last)
-                    fence_acquire_gpu();
+                last = atom_add_acq_rel_gpu(a.counters + item, 1) == last_cta - first_cta;
             }
             last = __shfl_sync(kFull, last, 0);
             if (last) {
@@ -1223,9 +1255,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int item = cur.b * a.items_per_seq + cur.k;
         const int hg = cur.k / a.hchunks, hc = cur.k - hg * a.hchunks;
         const ItemOut o = item_out(a, cur, hh);
-        const int item_start = start + u - cur.off;
-        const int first_cta = item_start / chunk;
-        const int last_cta = (item_start + cur.n - 1) / chunk;
+        const int first_cta = cur.pos / chunk;
+        const int last_cta = (cur.pos + cur.n - 1) / chunk;
         const bool single = first_cta == last_cta;
         // pieces of this item already finished elsewhere: read by thread 0 when it
         // starts its last unit of the piece, used at the epilogue
@@ -1344,9 +1375,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             } else {
                 // the CTA's last piece: count it in and merge here if it completed the item
                 if (tid == 0) {
-                    const bool last = atom_add_release_gpu(a.counters + item, 1) == last_cta - first_cta;
-                    if (last)
-                        fence_acquire_gpu();
+                    const bool last = atom_add_acq_rel_gpu(a.counters + item, 1) == last_cta - first_cta;
                     misc[kMiscLast] = last ? 1 : 0;
                 }
                 named_barrier(1, kConsumerThreads);
@@ -1383,11 +1412,13 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int gr
     grid_launch_dependents();
     const int item = blockIdx.x;
     const int b = item / a.items_per_seq, k = item - b * a.items_per_seq;
+    // work positions, as the decode kernel counts them
     int pre = 0, tot = 0;
     for (int bb = threadIdx.x; bb < a.B; bb += 128) {
         const int n = ctx_blocks(seq_ctx(a, bb));
-        tot += n;
-        pre += (bb < b) ? n : 0;
+        const int wpos = n > 0 ? a.items_per_seq * (n + a.item_cost) : 0;
+        tot += wpos;
+        pre += (bb < b) ? wpos : 0;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -1404,12 +1435,11 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int gr
     const int n = ctx_blocks(seq_ctx(a, b));
     if (n == 0)
         return;
-    const int total = tot * a.items_per_seq;
-    int chunk = (total + grid_ctas - 1) / grid_ctas;
+    int chunk = (tot + grid_ctas - 1) / grid_ctas;
     if (chunk < a.min_chunk)
         chunk = a.min_chunk;
-    const int item_start = pre * a.items_per_seq + k * n;
-    const int first_cta = item_start / chunk, last_cta = (item_start + n - 1) / chunk;
+    const int item_pos = pre + k * (n + a.item_cost) + a.item_cost;  // its first unit
+    const int first_cta = item_pos / chunk, last_cta = (item_pos + n - 1) / chunk;
     if (first_cta == last_cta)
         return;
     merge_pieces_global<E, D>(a, item, first_cta, last_cta, b, k, threadIdx.x, 128);
@@ -1430,7 +1460,21 @@ std::atomic<int> g_opt_grid{0};
 std::atomic<int> g_opt_min_chunk{0};
 std::atomic<int> g_opt_prod_lanes{0};
 std::atomic<int> g_opt_head_group{0};
+std::atomic<int> g_opt_item_cost{0};
 constexpr int kDefaultMinChunk = 4;
+
+// Work positions charged per work item (its fixed cost, in units of one work
+// unit's streaming time): the KV_OPT_ITEM_COST setting, else a default that
+// stands for about 1 us of per-item work at full bandwidth per SM.
+int item_cost(int D)
+{
+    const int v = g_opt_item_cost.load();
+    if (v < 0)
+        return 0;
+    if (v > 0)
+        return v;
+    return D == 64 ? 3 : 6;
+}
 
 constexpr int kMaxDevices = 64;
 
@@ -1624,7 +1668,9 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     const int group = Hq / Hkv;
     const int hg = heads_per_unit(Hkv);
     const int hchunks = (group + kGroupMax - 1) / kGroupMax;
-    if (static_cast<long long>(B) * max_blocks_per_seq * (Hkv / hg) * hchunks >= (1ll << 31))
+    const int cost = item_cost(D);
+    if (static_cast<long long>(B) * (max_blocks_per_seq + cost) * (Hkv / hg) * hchunks >= (1ll << 31) ||
+        B >= (1 << 24))
         return KV_ERR_ARG;
 
     int dev = 0;
@@ -1704,6 +1750,7 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     a.prod_lanes = lanes;
     const int mc = g_opt_min_chunk.load();
     a.min_chunk = mc > 0 ? mc : kDefaultMinChunk;
+    a.item_cost = cost;
     const int combine_mode = g_opt_combine.load();
     a.fused = combine_mode == 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;
@@ -1876,6 +1923,11 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_head_group.store(value);
         return KV_OK;
+    case KV_OPT_ITEM_COST:
+        if (value < -1 || value > 64)
+            return KV_ERR_ARG;
+        g_opt_item_cost.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -1896,6 +1948,8 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_prod_lanes.load();
     case KV_OPT_HEAD_GROUP:
         return g_opt_head_group.load();
+    case KV_OPT_ITEM_COST:
+        return g_opt_item_cost.load();
     default:
         return -1;
     }

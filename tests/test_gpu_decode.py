@@ -20,7 +20,7 @@ PATHS = {"tensor_cores": 1, "cuda_cores": 2}
 def _default_options(pkv):
     yield
     for key in (pkv.KV_OPT_COMPUTE, pkv.KV_OPT_COMBINE, pkv.KV_OPT_GRID, pkv.KV_OPT_MIN_CHUNK,
-                pkv.KV_OPT_PRODUCER_LANES, pkv.KV_OPT_HEAD_GROUP):
+                pkv.KV_OPT_PRODUCER_LANES, pkv.KV_OPT_HEAD_GROUP, pkv.KV_OPT_ITEM_COST):
         pkv.set_option(key, 0)
 
 
@@ -74,6 +74,18 @@ def test_many_split_pieces(pkv, oracle_mod, cuda_device, cid, grid, min_chunk):
     cfg = workloads.small_config(cid, batch=6, ctx_lo=1, ctx_hi=1500, W=96, n_layers=1)
     case = Case(cfg, cuda_device)
     run_and_check(pkv, oracle_mod, case, what=f"config {cid} shape, grid {grid} min_chunk {min_chunk}")
+
+
+@pytest.mark.parametrize("cost", [-1, 1, 7, 64])
+@pytest.mark.parametrize("cid", [2, 5])
+def test_item_cost_changes_only_the_split(pkv, oracle_mod, cuda_device, cid, cost):
+    """Charging items more or less (so CTAs get different ranges) gives the same answers."""
+    pkv.set_option(pkv.KV_OPT_ITEM_COST, cost)
+    pkv.set_option(pkv.KV_OPT_GRID, 37)
+    cfg = workloads.small_config(cid, batch=11, ctx_lo=1, ctx_hi=1200, W=80, n_layers=1, shared_fraction=0.0,
+                                 lognormal_mean=600.0)
+    case = Case(cfg, cuda_device)
+    run_and_check(pkv, oracle_mod, case, what=f"config {cid} shape, item cost {cost}")
 
 
 @pytest.mark.parametrize("hg", [1, 2, 4])
