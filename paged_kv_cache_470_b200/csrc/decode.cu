@@ -84,7 +84,8 @@ struct Geo {
     static constexpr int kQStride = D + 8;                      // second half shifted by 4 floats
     static constexpr int kQBytes = kMaxHG * kGroupMax * kQStride * 4;
     static constexpr int kPBytes = kConsumerWarps * 16 * kGroupMax * 4;
-    static constexpr int kScratchBytes = cmax(kMergeBytes, kQBytes + kPBytes);
+    static constexpr int kOwnBytes = kMaxHG * kGroupMax * (D + 2) * 4;  // a piece's state, for the solo merge
+    static constexpr int kScratchBytes = cmax(cmax(kMergeBytes, kQBytes + kPBytes), kOwnBytes);
     static constexpr int kOffScratch = kRingBytes;
     static constexpr int kOffBar = kOffScratch + kScratchBytes;
     static constexpr int kOffQBar = kOffBar + 2 * kMaxStages * 8;    // piece queue: full[4], empty[4]
@@ -443,102 +444,6 @@ struct Consumer<E, D, kPathMma, NH> {
         m1 = M1;
     }
 
-    // All other pieces of this split item are finished: merge them with this
-    // warp's state, in the same order and arithmetic as merge_pieces_global, so
-    // the result does not depend on which CTA merges.
-    __device__ __forceinline__ void merge_solo(const DecodeArgs &a, const ItemOut &o, int item, int first_cta,
-                                               int last_cta)
-    {
-        const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
-        const int self = static_cast<int>(blockIdx.x);
-        const size_t hbase = static_cast<size_t>(o.hh) * kGroupMax;
-        const int n0 = 2 * c, n1 = 2 * c + 1;
-        float M0 = -INFINITY, M1 = -INFINITY, L0 = 0.f, L1 = 0.f;
-        float O[kMt][4];
-#pragma unroll
-        for (int mt = 0; mt < kMt; ++mt)
-            O[mt][0] = O[mt][1] = O[mt][2] = O[mt][3] = 0.f;
-        for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
-            float mv0[kMergeBatch], mv1[kMergeBatch], lv0[kMergeBatch], lv1[kMergeBatch];
-#pragma unroll
-            for (int j = 0; j < kMergeBatch; ++j) {
-                const int cc = c0 + j;
-                if (cc > last_cta) {
-                    mv0[j] = mv1[j] = -INFINITY;
-                    lv0[j] = lv1[j] = 0.f;
-                } else if (cc == self) {
-                    mv0[j] = m0;
-                    mv1[j] = m1;
-                    lv0[j] = l0;
-                    lv1[j] = l1;
-                } else {
-                    const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase;
-                    mv0[j] = __ldcg(a.part_ml + (h + n0) * 2);
-                    lv0[j] = __ldcg(a.part_ml + (h + n0) * 2 + 1);
-                    mv1[j] = __ldcg(a.part_ml + (h + n1) * 2);
-                    lv1[j] = __ldcg(a.part_ml + (h + n1) * 2 + 1);
-                }
-            }
-            float Mb0 = M0, Mb1 = M1;
-#pragma unroll
-            for (int j = 0; j < kMergeBatch; ++j) {
-                Mb0 = fmaxf(Mb0, mv0[j]);
-                Mb1 = fmaxf(Mb1, mv1[j]);
-            }
-            const float sc0 = rescale(M0, Mb0), sc1 = rescale(M1, Mb1);
-            L0 *= sc0;
-            L1 *= sc1;
-#pragma unroll
-            for (int mt = 0; mt < kMt; ++mt) {
-                O[mt][0] *= sc0;
-                O[mt][1] *= sc1;
-                O[mt][2] *= sc0;
-                O[mt][3] *= sc1;
-            }
-#pragma unroll
-            for (int j = 0; j < kMergeBatch; ++j) {
-                const int cc = c0 + j;
-                const float w0 = rescale(mv0[j], Mb0), w1 = rescale(mv1[j], Mb1);
-                L0 = fmaf(w0, lv0[j], L0);
-                L1 = fmaf(w1, lv1[j], L1);
-                if (cc > last_cta)
-                    continue;  // a padding piece adds exact zeros
-                if (cc == self) {
-#pragma unroll
-                    for (int mt = 0; mt < kMt; ++mt) {
-                        O[mt][0] = fmaf(w0, acc[mt][0], O[mt][0]);
-                        O[mt][1] = fmaf(w1, acc[mt][1], O[mt][1]);
-                        O[mt][2] = fmaf(w0, acc[mt][2], O[mt][2]);
-                        O[mt][3] = fmaf(w1, acc[mt][3], O[mt][3]);
-                    }
-                } else {
-                    const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase;
-                    const float *p0 = a.part_acc + (h + n0) * D;
-                    const float *p1 = a.part_acc + (h + n1) * D;
-#pragma unroll
-                    for (int mt = 0; mt < kMt; ++mt) {
-                        const int d = mt * 16 + r;
-                        O[mt][0] = fmaf(w0, __ldcg(p0 + d), O[mt][0]);
-                        O[mt][1] = fmaf(w1, __ldcg(p1 + d), O[mt][1]);
-                        O[mt][2] = fmaf(w0, __ldcg(p0 + d + 8), O[mt][2]);
-                        O[mt][3] = fmaf(w1, __ldcg(p1 + d + 8), O[mt][3]);
-                    }
-                }
-            }
-            M0 = Mb0;
-            M1 = Mb1;
-        }
-#pragma unroll
-        for (int mt = 0; mt < kMt; ++mt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                acc[mt][i] = O[mt][i];
-        m0 = M0;
-        m1 = M1;
-        l0 = L0;
-        l1 = L1;
-    }
-
     __device__ __forceinline__ void store_final(const DecodeArgs &a, const ItemOut &o) const
     {
         const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
@@ -560,13 +465,16 @@ struct Consumer<E, D, kPathMma, NH> {
         }
     }
 
-    __device__ __forceinline__ void store_partial(const DecodeArgs &a, const ItemOut &o) const
+    // This warp's unnormalised state for its kv head, in the piece layout
+    // [kv head][query head][D] and [kv head][query head][2] starting at
+    // part_acc / part_ml (a global slot, or the CTA's own copy in shared memory).
+    __device__ __forceinline__ void store_state(const ItemOut &o, float *part_acc, float *part_ml) const
     {
         const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
         const int n0 = 2 * c, n1 = 2 * c + 1;
-        const size_t head0 = (o.slot * kMaxHG + o.hh) * kGroupMax;
-        float *p0 = a.part_acc + (head0 + n0) * D;
-        float *p1 = a.part_acc + (head0 + n1) * D;
+        const size_t head0 = static_cast<size_t>(o.hh) * kGroupMax;
+        float *p0 = part_acc + (head0 + n0) * D;
+        float *p1 = part_acc + (head0 + n1) * D;
 #pragma unroll
         for (int mt = 0; mt < kMt; ++mt) {
             const int d = mt * 16 + r;
@@ -581,12 +489,12 @@ struct Consumer<E, D, kPathMma, NH> {
         }
         if (r == 0) {
             if (n0 < o.gc) {
-                a.part_ml[(head0 + n0) * 2] = m0;
-                a.part_ml[(head0 + n0) * 2 + 1] = l0;
+                part_ml[(head0 + n0) * 2] = m0;
+                part_ml[(head0 + n0) * 2 + 1] = l0;
             }
             if (n1 < o.gc) {
-                a.part_ml[(head0 + n1) * 2] = m1;
-                a.part_ml[(head0 + n1) * 2 + 1] = l1;
+                part_ml[(head0 + n1) * 2] = m1;
+                part_ml[(head0 + n1) * 2 + 1] = l1;
             }
         }
     }
@@ -740,74 +648,6 @@ struct Consumer<E, D, kPathSimt, NH> {
         }
     }
 
-    // As Consumer<E, D, kPathMma>::merge_solo: same order and arithmetic as merge_pieces_global.
-    __device__ __forceinline__ void merge_solo(const DecodeArgs &a, const ItemOut &o, int item, int first_cta,
-                                               int last_cta)
-    {
-        const int lane = threadIdx.x & 31;
-        const int self = static_cast<int>(blockIdx.x);
-        const size_t hbase = static_cast<size_t>(o.hh) * kGroupMax;
-#pragma unroll
-        for (int n = 0; n < NH; ++n) {
-            float M = -INFINITY, L = 0.f;
-            float O[C];
-#pragma unroll
-            for (int e = 0; e < C; ++e)
-                O[e] = 0.f;
-            for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
-                float mv[kMergeBatch], lv[kMergeBatch];
-#pragma unroll
-                for (int j = 0; j < kMergeBatch; ++j) {
-                    const int cc = c0 + j;
-                    if (cc > last_cta) {
-                        mv[j] = -INFINITY;
-                        lv[j] = 0.f;
-                    } else if (cc == self) {
-                        mv[j] = m[n];
-                        lv[j] = l[n];
-                    } else {
-                        const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase + n;
-                        mv[j] = __ldcg(a.part_ml + h * 2);
-                        lv[j] = __ldcg(a.part_ml + h * 2 + 1);
-                    }
-                }
-                float Mb = M;
-#pragma unroll
-                for (int j = 0; j < kMergeBatch; ++j)
-                    Mb = fmaxf(Mb, mv[j]);
-                const float sc = rescale(M, Mb);
-                L *= sc;
-#pragma unroll
-                for (int e = 0; e < C; ++e)
-                    O[e] *= sc;
-#pragma unroll
-                for (int j = 0; j < kMergeBatch; ++j) {
-                    const int cc = c0 + j;
-                    const float w = rescale(mv[j], Mb);
-                    L = fmaf(w, lv[j], L);
-                    if (cc > last_cta)
-                        continue;
-                    if (cc == self) {
-#pragma unroll
-                        for (int e = 0; e < C; ++e)
-                            O[e] = fmaf(w, acc[n][e], O[e]);
-                    } else {
-                        const size_t h = (static_cast<size_t>(cc) + item) * (kMaxHG * kGroupMax) + hbase + n;
-#pragma unroll
-                        for (int e = 0; e < C; ++e)
-                            O[e] = fmaf(w, __ldcg(a.part_acc + h * D + lane * C + e), O[e]);
-                    }
-                }
-                M = Mb;
-            }
-#pragma unroll
-            for (int e = 0; e < C; ++e)
-                acc[n][e] = O[e];
-            m[n] = M;
-            l[n] = L;
-        }
-    }
-
     __device__ __forceinline__ void store_final(const DecodeArgs &a, const ItemOut &o) const
     {
         const int lane = threadIdx.x & 31;
@@ -823,46 +663,49 @@ struct Consumer<E, D, kPathSimt, NH> {
         }
     }
 
-    __device__ __forceinline__ void store_partial(const DecodeArgs &a, const ItemOut &o) const
+    __device__ __forceinline__ void store_state(const ItemOut &o, float *part_acc, float *part_ml) const
     {
         const int lane = threadIdx.x & 31;
-        const size_t head0 = (o.slot * kMaxHG + o.hh) * kGroupMax;
+        const size_t head0 = static_cast<size_t>(o.hh) * kGroupMax;
 #pragma unroll
         for (int n = 0; n < NH; ++n) {
             if (n < o.gc) {
-                float *dst = a.part_acc + (head0 + n) * D + lane * C;
+                float *dst = part_acc + (head0 + n) * D + lane * C;
 #pragma unroll
                 for (int e = 0; e < C; ++e)
                     dst[e] = acc[n][e];
                 if (lane == 0) {
-                    a.part_ml[(head0 + n) * 2] = m[n];
-                    a.part_ml[(head0 + n) * 2 + 1] = l[n];
+                    part_ml[(head0 + n) * 2] = m[n];
+                    part_ml[(head0 + n) * 2 + 1] = l[n];
                 }
             }
         }
     }
 };
 
-// Log-sum-exp merge of the split-K pieces of one item, read from global memory.
-// The item's pieces sit in slots first_cta + item .. last_cta + item. Each
-// thread merges two groups of four output columns at a time, and all loads
-// for up to four pieces are issued before any is used, so a merge costs
-// about one memory round trip per four pieces.
+// Log-sum-exp merge of the split-K pieces of one item. The item's pieces sit in
+// slots first_cta + item .. last_cta + item of the workspace, except that piece
+// `own_cta` (if own_acc is not null) is read from the caller's shared-memory
+// copy in the same layout. Each thread merges NC groups of four output columns
+// at a time, and all loads for up to four pieces are issued before any is used,
+// so a merge costs about one memory round trip per four pieces. The order of
+// the arithmetic depends only on the pieces, not on which CTA merges.
 template <class E, int D>
 __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int item, int first_cta, int last_cta,
-                                                    int b, int k, int tid, int nthreads)
+                                                    int b, int k, int tid, int nthreads, int own_cta = -1,
+                                                    const float *own_acc = nullptr, const float *own_ml = nullptr)
 {
     constexpr int D4 = D / 4;
+    constexpr int NC = 2;
     const int hg = k / a.hchunks, hc = k - hg * a.hchunks;
     const int gc = min(kGroupMax, a.group - hc * kGroupMax);
     const int per_head = gc * D4;
     const int total = a.hg * per_head;
-    for (int base = tid; base < total; base += 2 * nthreads) {
-        size_t head[2];
-        int col[2];
-        bool ok[2];
+    for (int base = tid; base < total; base += NC * nthreads) {
+        int head[NC], col[NC];
+        bool ok[NC];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
+        for (int e = 0; e < NC; ++e) {
             const int idx = base + e * nthreads;
             ok[e] = idx < total;
             const int i2 = ok[e] ? idx : base;
@@ -870,32 +713,44 @@ __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int ite
             const int rem = i2 - hh * per_head;
             const int n = rem / D4;
             col[e] = (rem - n * D4) * 4;
-            head[e] = static_cast<size_t>(hh) * kGroupMax + n;  // within a slot
+            head[e] = hh * kGroupMax + n;  // within a slot
         }
-        float M[2] = {-INFINITY, -INFINITY}, L[2] = {0.f, 0.f};
-        float4 O[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+        float M[NC], L[NC];
+        float4 O[NC];
+#pragma unroll
+        for (int e = 0; e < NC; ++e) {
+            M[e] = -INFINITY;
+            L[e] = 0.f;
+            O[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
-            float mv[2][kMergeBatch], lv[2][kMergeBatch];
-            float4 ov[2][kMergeBatch];
+            float mv[NC][kMergeBatch], lv[NC][kMergeBatch];
+            float4 ov[NC][kMergeBatch];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
+            for (int j = 0; j < kMergeBatch; ++j) {
+                const int c = c0 + j;
+                const bool own = c == own_cta && own_acc != nullptr;
+                const size_t slot = (static_cast<size_t>(c) + item) * (kMaxHG * kGroupMax);
 #pragma unroll
-                for (int j = 0; j < kMergeBatch; ++j) {
-                    const int c = c0 + j;
-                    if (c <= last_cta) {
-                        const size_t h = (static_cast<size_t>(c) + item) * (kMaxHG * kGroupMax) + head[e];
-                        mv[e][j] = __ldcg(a.part_ml + h * 2);
-                        lv[e][j] = __ldcg(a.part_ml + h * 2 + 1);
-                        ov[e][j] = __ldcg(reinterpret_cast<const float4 *>(a.part_acc + h * D + col[e]));
-                    } else {
+                for (int e = 0; e < NC; ++e) {
+                    if (c > last_cta || !ok[e]) {
                         mv[e][j] = -INFINITY;
                         lv[e][j] = 0.f;
                         ov[e][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    } else if (own) {
+                        mv[e][j] = own_ml[head[e] * 2];
+                        lv[e][j] = own_ml[head[e] * 2 + 1];
+                        ov[e][j] = *reinterpret_cast<const float4 *>(own_acc + head[e] * D + col[e]);
+                    } else {
+                        const size_t h = slot + head[e];
+                        mv[e][j] = __ldcg(a.part_ml + h * 2);
+                        lv[e][j] = __ldcg(a.part_ml + h * 2 + 1);
+                        ov[e][j] = __ldcg(reinterpret_cast<const float4 *>(a.part_acc + h * D + col[e]));
                     }
                 }
             }
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
+            for (int e = 0; e < NC; ++e) {
                 float Mb = M[e];
 #pragma unroll
                 for (int j = 0; j < kMergeBatch; ++j)
@@ -919,10 +774,10 @@ __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int ite
             }
         }
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
+        for (int e = 0; e < NC; ++e) {
             if (!ok[e])
                 continue;
-            const int hh = static_cast<int>(head[e] / kGroupMax), n = static_cast<int>(head[e] % kGroupMax);
+            const int hh = head[e] / kGroupMax, n = head[e] % kGroupMax;
             const int h = (hg * a.hg + hh) * a.group + hc * kGroupMax + n;
             const float inv = 1.f / L[e];
             uint2 packed;
@@ -1340,18 +1195,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // stores its partial and counts itself in; the CTA that completes the count
         // merges from global memory -- checked at that CTA's next epilogue.
         const bool solo = misc[kMiscSolo] != 0;
+        float *own_acc = scratch;                                   // the solo merge's copy of this piece
+        float *own_ml = scratch + kMaxHG * kGroupMax * D;
         if (stream == 0) {
             if (single) {
                 st.store_final(a, o);
             } else if (solo) {
-                st.merge_solo(a, o, item, first_cta, last_cta);
-                st.store_final(a, o);
+                st.store_state(o, own_acc, own_ml);
             } else {
-                st.store_partial(a, o);
+                const size_t slot0 = o.slot * (kMaxHG * kGroupMax);
+                st.store_state(o, a.part_acc + slot0 * D, a.part_ml + slot0 * 2);
             }
         }
-        if (!single && a.fused && solo && tid == 0)
-            a.counters[item] = 0;
+        if (!single && solo) {
+            // every other piece is done: merge them with this one (read from shared memory)
+            named_barrier(1, kConsumerThreads);
+            merge_pieces_global<E, D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads,
+                                      static_cast<int>(blockIdx.x), own_acc, own_ml);
+            if (tid == 0)
+                a.counters[item] = 0;
+        }
         named_barrier(1, kConsumerThreads);  // this piece's partial is written; the scratch is free
         if (!single && a.fused && !solo) {
             if (!final_piece) {
