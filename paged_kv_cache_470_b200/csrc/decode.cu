@@ -1113,8 +1113,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         const int first_cta = cur.pos / chunk;
         const int last_cta = (cur.pos + cur.n - 1) / chunk;
         const bool single = first_cta == last_cta;
-        // pieces of this item already finished elsewhere: read by thread 0 when it
-        // starts its last unit of the piece, used at the epilogue
+        // Pieces of this item already finished elsewhere, read by the first lane of
+        // a stream that does not take the item's last unit (the checker) when it
+        // starts its own last unit, and judged when it has finished it: its wait
+        // for the count and the acquire fence overlap the last unit's work.
+        const int checker_stream = ((u + run - 1) % NS + 1) % NS;
+        const bool checker = stream == checker_stream && hh == 0 && lane == 0;
         int seen = -1;
 
         if (PATH == kPathSimt) {
@@ -1150,7 +1154,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 }
                 break;
             }
-            if (tid == 0 && !single && a.fused && i + NS >= run)
+            if (checker && !single && a.fused && i + NS >= run)
                 seen = ld_relaxed_gpu(a.counters + item);
             const uint32_t kb = ring + s * a.stage_bytes + hh * kHeadTileBytes;
             const int valid = min(kBlockTokens, cur.ctx - (cur.off + i) * kBlockTokens);
@@ -1162,17 +1166,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (lane == 0)
                 mbar_arrive(&empty[s]);
         }
-        st.finish();
-        const bool final_piece = u + run == count;
-        if (tid == 0) {
+        if (checker) {
             bool solo_now = false;
             if (!single && a.fused) {
+                if (seen < 0)  // the checker's stream had no unit of this item
+                    seen = ld_relaxed_gpu(a.counters + item);
                 solo_now = seen == last_cta - first_cta;
                 if (solo_now)
                     fence_acquire_gpu();  // the other pieces' partials, before anyone reads them
             }
             misc[kMiscSolo] = solo_now ? 1 : 0;
         }
+        st.finish();
+        const bool final_piece = u + run == count;
 
         // ---- merge the streams pairwise: stream s + step hands over to stream s ----
         if (PATH == kPathSimt || NS == 1)
