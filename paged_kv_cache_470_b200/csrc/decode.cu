@@ -686,104 +686,97 @@ struct Consumer<E, D, kPathSimt, NH> {
 // Log-sum-exp merge of the split-K pieces of one item. The item's pieces sit in
 // slots first_cta + item .. last_cta + item of the workspace, except that piece
 // `own_cta` (if own_acc is not null) is read from the caller's shared-memory
-// copy in the same layout. Each thread merges NC groups of four output columns
-// at a time, and all loads for up to four pieces are issued before any is used,
-// so a merge costs about one memory round trip per four pieces. The order of
-// the arithmetic depends only on the pieces, not on which CTA merges.
+// copy in the same layout. A thread takes NC consecutive groups of four output
+// columns of one (kv head, query head) row, and issues all loads for MB pieces
+// before using any, so a merge costs about one memory round trip per MB pieces.
+// The order of the arithmetic depends only on the pieces, not on which CTA
+// merges.
 template <class E, int D>
 __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int item, int first_cta, int last_cta,
                                                     int b, int k, int tid, int nthreads, int own_cta = -1,
                                                     const float *own_acc = nullptr, const float *own_ml = nullptr)
 {
-    constexpr int D4 = D / 4;
-    constexpr int NC = 2;
+    constexpr int NC = D == 128 ? 4 : 2;          // float4 column groups per thread
+    constexpr int MB = D == 128 ? 2 : kMergeBatch;  // pieces per round of loads
+    constexpr int TPR = D / 4 / NC;               // threads per row
     const int hg = k / a.hchunks, hc = k - hg * a.hchunks;
     const int gc = min(kGroupMax, a.group - hc * kGroupMax);
-    const int per_head = gc * D4;
-    const int total = a.hg * per_head;
-    for (int base = tid; base < total; base += NC * nthreads) {
-        int head[NC], col[NC];
-        bool ok[NC];
-#pragma unroll
-        for (int e = 0; e < NC; ++e) {
-            const int idx = base + e * nthreads;
-            ok[e] = idx < total;
-            const int i2 = ok[e] ? idx : base;
-            const int hh = i2 / per_head;
-            const int rem = i2 - hh * per_head;
-            const int n = rem / D4;
-            col[e] = (rem - n * D4) * 4;
-            head[e] = hh * kGroupMax + n;  // within a slot
-        }
-        float M[NC], L[NC];
+    const int rows = a.hg * gc;
+    const int rows_per_pass = nthreads / TPR;
+    for (int row = tid / TPR; row < rows; row += rows_per_pass) {
+        if (tid >= rows_per_pass * TPR)
+            break;
+        const int hh = row / gc, n = row - hh * gc;
+        const int head = hh * kGroupMax + n;      // within a slot
+        const int col0 = (tid % TPR) * NC * 4;
+        float M = -INFINITY, L = 0.f;
         float4 O[NC];
 #pragma unroll
-        for (int e = 0; e < NC; ++e) {
-            M[e] = -INFINITY;
-            L[e] = 0.f;
+        for (int e = 0; e < NC; ++e)
             O[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        for (int c0 = first_cta; c0 <= last_cta; c0 += kMergeBatch) {
-            float mv[NC][kMergeBatch], lv[NC][kMergeBatch];
-            float4 ov[NC][kMergeBatch];
+        for (int c0 = first_cta; c0 <= last_cta; c0 += MB) {
+            float mv[MB], lv[MB];
+            float4 ov[MB][NC];
 #pragma unroll
-            for (int j = 0; j < kMergeBatch; ++j) {
+            for (int j = 0; j < MB; ++j) {
                 const int c = c0 + j;
-                const bool own = c == own_cta && own_acc != nullptr;
-                const size_t slot = (static_cast<size_t>(c) + item) * (kMaxHG * kGroupMax);
+                if (c > last_cta) {
+                    mv[j] = -INFINITY;
+                    lv[j] = 0.f;
 #pragma unroll
-                for (int e = 0; e < NC; ++e) {
-                    if (c > last_cta || !ok[e]) {
-                        mv[e][j] = -INFINITY;
-                        lv[e][j] = 0.f;
-                        ov[e][j] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    } else if (own) {
-                        mv[e][j] = own_ml[head[e] * 2];
-                        lv[e][j] = own_ml[head[e] * 2 + 1];
-                        ov[e][j] = *reinterpret_cast<const float4 *>(own_acc + head[e] * D + col[e]);
-                    } else {
-                        const size_t h = slot + head[e];
-                        mv[e][j] = __ldcg(a.part_ml + h * 2);
-                        lv[e][j] = __ldcg(a.part_ml + h * 2 + 1);
-                        ov[e][j] = __ldcg(reinterpret_cast<const float4 *>(a.part_acc + h * D + col[e]));
-                    }
+                    for (int e = 0; e < NC; ++e)
+                        ov[j][e] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else if (c == own_cta && own_acc != nullptr) {
+                    mv[j] = own_ml[head * 2];
+                    lv[j] = own_ml[head * 2 + 1];
+#pragma unroll
+                    for (int e = 0; e < NC; ++e)
+                        ov[j][e] = *reinterpret_cast<const float4 *>(own_acc + head * D + col0 + e * 4);
+                } else {
+                    const size_t h = (static_cast<size_t>(c) + item) * (kMaxHG * kGroupMax) + head;
+                    mv[j] = __ldcg(a.part_ml + h * 2);
+                    lv[j] = __ldcg(a.part_ml + h * 2 + 1);
+#pragma unroll
+                    for (int e = 0; e < NC; ++e)
+                        ov[j][e] = __ldcg(reinterpret_cast<const float4 *>(a.part_acc + h * D + col0 + e * 4));
                 }
             }
+            float Mb = M;
+#pragma unroll
+            for (int j = 0; j < MB; ++j)
+                Mb = fmaxf(Mb, mv[j]);
+            const float sc = rescale(M, Mb);
+            L *= sc;
 #pragma unroll
             for (int e = 0; e < NC; ++e) {
-                float Mb = M[e];
-#pragma unroll
-                for (int j = 0; j < kMergeBatch; ++j)
-                    Mb = fmaxf(Mb, mv[e][j]);
-                const float sc = rescale(M[e], Mb);
-                L[e] *= sc;
                 O[e].x *= sc;
                 O[e].y *= sc;
                 O[e].z *= sc;
                 O[e].w *= sc;
-#pragma unroll
-                for (int j = 0; j < kMergeBatch; ++j) {
-                    const float w = rescale(mv[e][j], Mb);
-                    L[e] = fmaf(w, lv[e][j], L[e]);
-                    O[e].x = fmaf(w, ov[e][j].x, O[e].x);
-                    O[e].y = fmaf(w, ov[e][j].y, O[e].y);
-                    O[e].z = fmaf(w, ov[e][j].z, O[e].z);
-                    O[e].w = fmaf(w, ov[e][j].w, O[e].w);
-                }
-                M[e] = Mb;
             }
+#pragma unroll
+            for (int j = 0; j < MB; ++j) {
+                const float w = rescale(mv[j], Mb);
+                L = fmaf(w, lv[j], L);
+#pragma unroll
+                for (int e = 0; e < NC; ++e) {
+                    O[e].x = fmaf(w, ov[j][e].x, O[e].x);
+                    O[e].y = fmaf(w, ov[j][e].y, O[e].y);
+                    O[e].z = fmaf(w, ov[j][e].z, O[e].z);
+                    O[e].w = fmaf(w, ov[j][e].w, O[e].w);
+                }
+            }
+            M = Mb;
         }
+        const int h = (hg * a.hg + hh) * a.group + hc * kGroupMax + n;
+        const float inv = 1.f / L;
+        uint16_t *dst = a.out + (static_cast<size_t>(b) * a.Hq + h) * D + col0;
 #pragma unroll
         for (int e = 0; e < NC; ++e) {
-            if (!ok[e])
-                continue;
-            const int hh = head[e] / kGroupMax, n = head[e] % kGroupMax;
-            const int h = (hg * a.hg + hh) * a.group + hc * kGroupMax + n;
-            const float inv = 1.f / L[e];
             uint2 packed;
             packed.x = E::pack(O[e].x * inv, O[e].y * inv);
             packed.y = E::pack(O[e].z * inv, O[e].w * inv);
-            *reinterpret_cast<uint2 *>(a.out + (static_cast<size_t>(b) * a.Hq + h) * D + col[e]) = packed;
+            *reinterpret_cast<uint2 *>(dst + e * 4) = packed;
         }
     }
 }
