@@ -235,6 +235,10 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
  *                     group and query-head chunk) adds this many more for its
  *                     fixed cost; CTAs take equal ranges of positions.
  *                     0 auto, -1 none, 1..64 that many.
+ * Kernels are launched with programmatic dependent launch. q, k_new, v_new,
+ * the caches, the workspace and out are touched only after the previous kernel
+ * in the stream has completed; block_tables and context_lens are read before
+ * that, so the kernel launched just before a decode call must not write them.
  * Returns KV_ERR_ARG for an unknown key or value.
  */
 #define KV_OPT_COMPUTE 1

@@ -59,6 +59,7 @@ constexpr int kProducerWarp = kConsumerWarps;
 constexpr int kHelperWarp = kConsumerWarps + 1;   // counts finished split pieces off the consumers' path
 constexpr int kThreads = kConsumerThreads + 64;
 constexpr int kPieceQueue = 4;                    // consumer -> helper queue of finished split pieces
+constexpr int kBarConsumers = 1;                  // named barrier of the consumer warps
 constexpr int kGroupMax = 8;            // query heads per kv head per work item
 constexpr int kMaxHG = 4;               // kv heads per work unit
 constexpr int kHeadTileBytes = 2048;    // one kv head: 16 rows x 64 elements, 128B-swizzled
@@ -977,8 +978,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (warp == kProducerWarp) {
         // ---------------- producer: block ids -> TMA loads ----------------
         // The first batch of block ids is read before waiting on the previous
-        // grid (no kernel of this library writes the tables); the cache itself
-        // is only touched after the wait.
+        // grid (the tables must not come from the kernel launched just before);
+        // the cache is only touched after the wait.
         int blk_first = load_block_ids(a, cur0, min(32, min(cur0.n - cur0.off, count)), lane);
         grid_dependency_wait();
         grid_launch_dependents();
@@ -1086,9 +1087,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     Consumer<E, D, PATH, NH> st;
     float *q_s = scratch + hh * kGroupMax * G::kQStride;                         // CUDA-core path only
     float *p_s = scratch + kMaxHG * kGroupMax * G::kQStride + warp * 16 * kGroupMax;
-    st.prefetch_q(a, item_out(a, cur0, hh));  // q is never written by this library: no wait needed
     grid_dependency_wait();
     grid_launch_dependents();
+    // q, like the new token rows, may come from the previous kernel: load after the wait
+    st.prefetch_q(a, item_out(a, cur0, hh));
     // the new token rows (fused append) are loaded after the wait: the caller may
     // have produced them in the previous kernel
     AppendRow ar_next = load_append_row<D>(a, cur0, (cur0.k / a.hchunks) * a.hg + hh,
@@ -1125,7 +1127,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const float v = (n < o.gc) ? E::to_f32(a.q[(static_cast<size_t>(cur.b) * a.Hq + h) * D + d]) : 0.f;
                 scratch[(h2 * kGroupMax + n) * G::kQStride + d + ((d >= D / 2) ? 4 : 0)] = v;
             }
-            named_barrier(1, kConsumerThreads);
+            named_barrier(kBarConsumers, kConsumerThreads);
         }
         st.begin_item(a, o, q_s);
         const AppendRow ar = ar_next;
@@ -1175,7 +1177,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
         // ---- merge the streams pairwise: stream s + step hands over to stream s ----
         if (PATH == kPathSimt || NS == 1)
-            named_barrier(1, kConsumerThreads);  // the scratch also holds q_s / p_s
+            named_barrier(kBarConsumers, kConsumerThreads);  // the scratch also holds q_s / p_s
         for (int step = 1; step < NS; step <<= 1) {
             const bool giver = (stream % (2 * step)) == step;
             const bool taker = (stream % (2 * step)) == 0 && stream + step < NS;
@@ -1183,10 +1185,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int slot_taker = ((stream + step) / (2 * step)) * a.hg + hh;
             if (giver)
                 st.save(scratch + slot_giver * Consumer<E, D, PATH, NH>::kRegs * 32);
-            named_barrier(1, kConsumerThreads);
+            named_barrier(kBarConsumers, kConsumerThreads);
             if (taker)
                 st.merge(scratch + slot_taker * Consumer<E, D, PATH, NH>::kRegs * 32);
-            named_barrier(1, kConsumerThreads);
+            named_barrier(kBarConsumers, kConsumerThreads);
         }
 
         // Split items: if every other piece was already done when this one started,
@@ -1208,13 +1210,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         }
         if (!single && solo) {
             // every other piece is done: merge them with this one (read from shared memory)
-            named_barrier(1, kConsumerThreads);
+            named_barrier(kBarConsumers, kConsumerThreads);
             merge_pieces_global<E, D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads,
                                       static_cast<int>(blockIdx.x), own_acc, own_ml);
             if (tid == 0)
                 a.counters[item] = 0;
         }
-        named_barrier(1, kConsumerThreads);  // this piece's partial is written; the scratch is free
+        named_barrier(kBarConsumers, kConsumerThreads);  // this piece's partial is written; the scratch is free
         if (!single && a.fused && !solo) {
             if (!final_piece) {
                 // hand the count to the helper warp and go on streaming
@@ -1240,7 +1242,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     const bool last = atom_add_acq_rel_gpu(a.counters + item, 1) == last_cta - first_cta;
                     misc[kMiscLast] = last ? 1 : 0;
                 }
-                named_barrier(1, kConsumerThreads);
+                named_barrier(kBarConsumers, kConsumerThreads);
                 if (misc[kMiscLast]) {
                     merge_pieces_global<E, D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads);
                     if (tid == 0)

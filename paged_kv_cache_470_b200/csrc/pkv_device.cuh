@@ -21,8 +21,8 @@ __device__ __forceinline__ uint32_t smem_addr(const void *p)
 
 // ---- programmatic dependent launch -------------------------------------
 // Wait until the previous grid in the stream has completed and its writes are
-// visible. Everything before this call may only read data that no kernel of
-// this library writes (tables, lengths, q).
+// visible. Everything before this call may only read data that the previous
+// kernel does not write (the block tables and lengths).
 __device__ __forceinline__ void grid_dependency_wait()
 {
     asm volatile("griddepcontrol.wait;" ::: "memory");

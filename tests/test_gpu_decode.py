@@ -88,6 +88,25 @@ def test_item_cost_changes_only_the_split(pkv, oracle_mod, cuda_device, cid, cos
     run_and_check(pkv, oracle_mod, case, what=f"config {cid} shape, item cost {cost}")
 
 
+@pytest.mark.parametrize("grid", [0, 5])
+@pytest.mark.parametrize("cid", [2, 3])
+def test_back_to_back_layers(pkv, oracle_mod, cuda_device, cid, grid):
+    """Fused launches of several layers back to back on one stream and one workspace, no
+    synchronisation between them: each launch's prologue overlaps the previous launch."""
+    pkv.set_option(pkv.KV_OPT_GRID, grid)
+    cfg = workloads.small_config(cid, batch=7, ctx_lo=1, ctx_hi=1300, W=96, n_layers=4)
+    case = Case(cfg, cuda_device, n_layers=4)
+    hosts = [case.host_inputs(layer) for layer in range(4)]
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    outs = [gpu_step(pkv, case, layer, ws, fused=True) for layer in range(4)]
+    torch.cuda.synchronize()
+    for layer in range(4):
+        k2, v2, ref = oracle_step(oracle_mod, case, layer, hosts[layer])
+        assert np.array_equal(bf16_bits_np(case.k[layer]), k2)
+        compare(outs[layer], ref, f"back to back, config {cid} shape, layer {layer}")
+    assert pkv.read_status(ws) == 0
+
+
 @pytest.mark.parametrize("hg", [1, 2, 4])
 def test_forced_head_groups(pkv, oracle_mod, cuda_device, hg):
     """Work units of 1, 2 or 4 kv heads give the same answers."""
