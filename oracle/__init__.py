@@ -21,6 +21,12 @@ Contents, each citing the passage it follows:
 * :func:`kv_cache_append` -- the byte-exact scatter of new tokens into their
   block slots, slot = block * 16 + offset ("Module 23: Serving", section 23.4:
   blocks are allocated as the sequence grows).
+* :func:`paged_attention_prefill` -- a chunk of new query tokens per
+  sequence attending causally over the paged cache ("Module 23: Serving",
+  section 23.2, Prefill and Decode; "Designing an LLM serving system",
+  section "Scheduling: when prefill meets decode": chunked prefill). A query
+  at position p sees tokens 0..p, so it is a decode step over a context of
+  p + 1 tokens: the oracle is written as exactly that.
 * :func:`sequence_tokens` -- the logical token rows of one sequence, read
   through its block table (step 1 of the attention definition above).
 * :func:`copy_blocks`, :func:`gather_blocks`, :func:`scatter_blocks` --
@@ -181,6 +187,39 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
 
 def _is_fp16(x) -> bool:
     return not isinstance(x, np.ndarray) and str(x.dtype) == "torch.float16"
+
+
+def paged_attention_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start, scale: float,
+                            dtype: str = "bf16"):
+    """Reference chunked-prefill attention in float64.
+
+    q [T,Hq,D] holds, for sequence b, query_start[b+1] - query_start[b] = n_b
+    new tokens (rows query_start[b] ..), at positions c_b - n_b .. c_b - 1 of
+    its context (c_b = context_lens[b], the chunk included and already in the
+    cache). Token i of the chunk attends to cache positions 0 .. c_b - n_b + i.
+    Returns out [T,Hq,D] float64.
+    """
+    unpack = fp16_bits if dtype == "fp16" else bf16_bits
+    qb = unpack(q)
+    tables = np.asarray(block_tables, dtype=np.int32)
+    lens = np.asarray(context_lens, dtype=np.int64)
+    qs = np.asarray(query_start, dtype=np.int64)
+    B = tables.shape[0]
+    if qs.shape != (B + 1,) or qs[0] != 0 or qs[-1] != qb.shape[0] or (np.diff(qs) < 0).any():
+        raise ValueError("query_start must be [B+1], starting at 0, non-decreasing, ending at T")
+    rows, ctx = [], []
+    for b in range(B):
+        n = int(qs[b + 1] - qs[b])
+        if n > lens[b]:
+            raise ValueError("a chunk longer than its context")
+        for i in range(n):
+            rows.append(b)
+            ctx.append(int(lens[b]) - n + i + 1)   # the query's own position, plus one
+    if not rows:
+        return np.zeros(qb.shape, dtype=np.float64)
+    per_query_tables = np.ascontiguousarray(tables[np.array(rows)])
+    return paged_attention_decode(qb, k_cache, v_cache, per_query_tables, np.array(ctx, np.int32), scale,
+                                  dtype=dtype)
 
 
 def kv_cache_append(k_cache, v_cache, k_new, v_new, slot_mapping):

@@ -336,6 +336,60 @@ def test_fp16_decode_matches_dense_attention(oracle_mod):
 
 
 # ---------------------------------------------------------------------------
+# chunked prefill ("Module 23: Serving", 23.2; "Designing an LLM serving system",
+# Scheduling: when prefill meets decode)
+# ---------------------------------------------------------------------------
+def dense_causal_reference(q, K, V, lens, nq, qs, Hq, Hkv, scale):
+    """torch SDPA in float64 with an explicit boolean mask: query i of sequence b sees tokens < c - n + i + 1."""
+    g = Hq // Hkv
+    outs = []
+    for b, c in enumerate(lens):
+        n = nq[b]
+        if n == 0:
+            continue
+        qb = q[qs[b]:qs[b + 1]].to(torch.float64).permute(1, 0, 2)
+        kb = K[b].to(torch.float64).permute(1, 0, 2).repeat_interleave(g, 0)
+        vb = V[b].to(torch.float64).permute(1, 0, 2).repeat_interleave(g, 0)
+        mask = torch.zeros(n, c, dtype=torch.bool)
+        for i in range(n):
+            mask[i, :c - n + i + 1] = True
+        outs.append(F.scaled_dot_product_attention(qb, kb, vb, attn_mask=mask, scale=scale).permute(1, 0, 2))
+    return torch.cat(outs).numpy()
+
+
+@pytest.mark.parametrize("Hq,Hkv,D", [(4, 2, 8), (6, 6, 16), (8, 1, 8)])
+def test_prefill_matches_dense_causal_attention(oracle_mod, Hq, Hkv, D):
+    lens = [5, 20, 33, 16, 40]
+    nq = [5, 7, 1, 0, 40]            # whole prompts, a chunk, one token (a decode step), none, whole
+    g = torch.Generator().manual_seed(Hq * 100 + D)
+    K = [bf16_round(torch.randn(c, Hkv, D, generator=g)) for c in lens]
+    V = [bf16_round(torch.randn(c, Hkv, D, generator=g)) for c in lens]
+    qs = np.concatenate([[0], np.cumsum(nq)]).astype(np.int32)
+    q = bf16_round(torch.randn(int(qs[-1]), Hq, D, generator=g))
+    nb = sum(-(-c // 16) for c in lens) + 4
+    kp, vp, tab = paginate(K, V, lens, Hkv, D, nb, 3, 5)
+    scale = 1.0 / math.sqrt(D)
+    out = oracle_mod.paged_attention_prefill(bits(q), kp, vp, tab, np.array(lens, np.int32), qs, scale)
+    ref = dense_causal_reference(q, K, V, lens, nq, qs, Hq, Hkv, scale)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-12)
+    # the last query of a chunk sees the whole context: it equals the decode step at that length
+    dec = oracle_mod.paged_attention_decode(bits(q[qs[2] - 1:qs[2]]), kp, vp, tab[1:2], np.array([20], np.int32), scale)
+    np.testing.assert_array_equal(out[qs[2] - 1], dec[0])
+
+
+def test_prefill_rejects_bad_chunks(oracle_mod):
+    lens = [4]
+    kp = np.zeros((2, 16, 1, 8), np.uint16)
+    tab = np.array([[0, 1]], np.int32)
+    with pytest.raises(ValueError):   # a chunk longer than its context
+        oracle_mod.paged_attention_prefill(np.zeros((5, 1, 8), np.uint16), kp, kp, tab, np.array(lens, np.int32),
+                                           np.array([0, 5]), 1.0)
+    with pytest.raises(ValueError):   # offsets that do not cover q
+        oracle_mod.paged_attention_prefill(np.zeros((3, 1, 8), np.uint16), kp, kp, tab, np.array(lens, np.int32),
+                                           np.array([0, 2]), 1.0)
+
+
+# ---------------------------------------------------------------------------
 # reading through the table, and whole-block moves
 # ---------------------------------------------------------------------------
 def test_sequence_tokens_recovers_the_dense_sequence(oracle_mod):
