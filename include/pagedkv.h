@@ -216,6 +216,37 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
                                                 int num_blocks, int Hq, int Hkv, int D,
                                                 float scale, int dtype, kv_stream_t stream);
 
+/* ------------------------------------------------------------------------ */
+/* Chunked prefill over the paged cache                                      */
+/* ------------------------------------------------------------------------ */
+/*
+ * For each sequence b, the n_b = query_start[b+1] - query_start[b] rows
+ * q[query_start[b] ..] are the queries of the last n_b tokens of its context
+ * (context_lens[b] = c_b tokens, this chunk included: append its K/V first with
+ * kv_cache_append). Chunk token i sits at position p = c_b - n_b + i and
+ * attends causally to positions 0..p:
+ *   out[query_start[b] + i][h] = sum_{t <= p} softmax_t(scale * <q[.][h], K_t>) V_t
+ * with kv head h / (Hq / Hkv) and K_t, V_t read through block_tables as for the
+ * decode. ("Module 23: Serving", section 23.2, Prefill and Decode; "Designing an
+ * LLM serving system", section "Scheduling: when prefill meets decode":
+ * chunked prefill.) n_b = c_b is a whole prompt; n_b = 1 is a decode step.
+ *
+ * q, out: [T][Hq][D] device, T = query_start[B]; query_start: [B+1] device
+ * int32, non-decreasing from 0; max_query_len >= every n_b (it sizes the
+ * grid). Tensor cores (mma.sync), fp32 accumulation, the probabilities rounded
+ * to the element type before they multiply V. No workspace. Data errors are
+ * OR-ed into *error_flag (device int32, may be NULL): KV_STATUS_BAD_CONTEXT
+ * when n_b > c_b, c_b > 16 * max_blocks_per_seq or n_b > max_query_len (that
+ * sequence's rows are not written), KV_STATUS_BAD_BLOCK_ID for ids outside the
+ * pool (block 0 is read instead). B <= 65535, Hkv <= 65535.
+ */
+KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k_cache,
+                                         const void *v_cache, const int32_t *block_tables,
+                                         int max_blocks_per_seq, const int32_t *context_lens,
+                                         const int32_t *query_start, int B, int max_query_len,
+                                         int num_blocks, int Hq, int Hkv, int D, float scale,
+                                         int dtype, int32_t *error_flag, kv_stream_t stream);
+
 /*
  * Process-wide tuning switches (defaults are the tuned choices).
  *   KV_OPT_COMPUTE:   0 auto, 1 tensor cores (mma.sync, 16-bit inputs), 2 CUDA cores

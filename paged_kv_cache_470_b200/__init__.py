@@ -42,6 +42,8 @@ _sig = {
     "paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
                                             _P]),
     "paged_attention_read_status": (_I, [_P, _P, _I, _P]),
+    "paged_attention_prefill": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P,
+                                     _P]),
     "kv_decode_set_option": (_I, [_I, _I]),
     "kv_decode_get_option": (_I, [_I]),
     "kv_pool_create": (_I, [_I, ctypes.POINTER(ctypes.c_void_p)]),
@@ -169,6 +171,27 @@ def paged_attention_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: tor
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
+    return out
+
+
+def paged_attention_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                            block_tables: torch.Tensor, context_lens: torch.Tensor, query_start: torch.Tensor,
+                            max_query_len: int, scale: float, error_flag: torch.Tensor | None = None,
+                            stream=None) -> torch.Tensor:
+    """Chunked prefill: rows q[query_start[b]:query_start[b+1]] are the last tokens of sequence b's context;
+    each attends causally over the paged cache. q/out [T,Hq,D], query_start [B+1] int32."""
+    T, Hq, D = q.shape
+    num_blocks, _, Hkv, Dk = k_cache.shape
+    B = block_tables.shape[0]
+    if Dk != D or tuple(out.shape) != (T, Hq, D) or query_start.numel() != B + 1 or context_lens.numel() != B:
+        raise ValueError("shape mismatch")
+    dt, code = k_cache.dtype, _cache_dtype(k_cache)
+    ef = _dev(error_flag, "error_flag", torch.int32) if error_flag is not None else None
+    _check("paged_attention_prefill", _lib.paged_attention_prefill(
+        _dev(out, "out", dt), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), _dev(query_start, "query_start", torch.int32), B,
+        int(max_query_len), num_blocks, Hq, Hkv, D, float(scale), code, ef, _stream_handle(stream)))
     return out
 
 

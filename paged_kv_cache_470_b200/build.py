@@ -20,7 +20,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpagedkv.so")
-SOURCES = ["append.cu", "decode.cu", "blocks.cu", "pool.cpp"]
+SOURCES = ["append.cu", "decode.cu", "prefill.cu", "blocks.cu", "pool.cpp"]
 HEADERS = ["pkv_device.cuh"]
 
 NVCC_FLAGS = [

@@ -45,6 +45,7 @@
 // 23.1).
 #include "pkv_device.cuh"
 #include "pagedkv.h"
+#include "tma_host.h"
 
 #include <cuda_runtime.h>
 
@@ -1392,46 +1393,6 @@ bool make_layout(int B, int Hq, int Hkv, int D, int sms, Layout *L)
     return true;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn()
-{
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-// View one cache tensor [num_blocks][16][Hkv][D] as a 4-D map whose dimensions
-// are (column, row, kv head, block) -- rows inside heads, so each head's 16
-// rows land as one contiguous 128B-swizzled 2 KB tile -- with a box of
-// 64 columns x 16 rows x HG heads x 1 block.
-bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv, int D, int hg, int dtype)
-{
-    EncodeTiledFn enc = encode_fn();
-    if (!enc)
-        return false;
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), 16, static_cast<cuuint64_t>(Hkv),
-                                static_cast<cuuint64_t>(num_blocks)};
-    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(Hkv) * D * 2, static_cast<cuuint64_t>(D) * 2,
-                                   static_cast<cuuint64_t>(16) * Hkv * D * 2};
-    const cuuint32_t box[4] = {64, 16, static_cast<cuuint32_t>(hg), 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUtensorMapDataType dt =
-        dtype == KV_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    return enc(tm, dt, 4, const_cast<void *>(cache), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 using DecodeFn = void (*)(const CUtensorMap, const CUtensorMap, const DecodeArgs);
 
 template <class E>
@@ -1584,8 +1545,8 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
         return KV_ERR_ARG;
 
     CUtensorMap tmK, tmV;
-    if (!make_cache_map(&tmK, k_cache, num_blocks, Hkv, D, hg, dtype) ||
-        !make_cache_map(&tmV, v_cache, num_blocks, Hkv, D, hg, dtype))
+    if (!pkv_host::make_cache_map(&tmK, k_cache, num_blocks, Hkv, D, hg, dtype) ||
+        !pkv_host::make_cache_map(&tmV, v_cache, num_blocks, Hkv, D, hg, dtype))
         return KV_ERR_CUDA;
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);

@@ -118,6 +118,17 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *tm,
         : "memory");
 }
 
+// The same without an L2 cache hint (default eviction priority).
+__device__ __forceinline__ void tma_load_4d_nohint(uint32_t dst, const CUtensorMap *tm, int x, int y, int z, int w,
+                                                   uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_addr(bar))
+        : "memory");
+}
+
 // ---- warp-level tensor-core pieces ---------------------------------------
 __device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr)
 {

@@ -1,0 +1,434 @@
+// paged_attention_prefill: chunked-prefill attention over a paged KV cache, for
+// sm_100a.
+//
+// What is computed ("Module 23: Serving", section 23.2, Prefill and Decode;
+// "Designing an LLM serving system", section "Scheduling: when prefill meets
+// decode": a long prompt is split into chunks processed between decode steps):
+// sequence b has c_b tokens in the cache, the last n_b of which are this
+// chunk's (already appended). Chunk token i sits at position p = c_b - n_b + i
+// and attends causally to cache positions 0..p, with query head h reading kv
+// head h / (Hq / Hkv):
+//     out[i][h] = sum_{t <= p} softmax_t(scale * <q[i][h], K_t>) V_t.
+//
+// Work decomposition. The query rows of one (sequence, kv head) are the chunk's
+// tokens times the group's query heads, token-major; a CTA takes 64 of them
+// (4 warps x 16 rows: the group's heads share every K/V tile) and reads the
+// sequence's KV blocks up to the last position among its rows. CTAs with
+// later rows (more KV) are launched first.
+//
+// Pipeline. Warp 4 is the producer: it reads block ids and issues TMA loads of
+// 4 KV blocks (64 tokens) per stage into a ring of 3 stages, guarded by
+// mbarriers with bounded waits. Warps 0-3 compute with tensor cores
+// (mma.sync.m16n8k16, 16-bit inputs, fp32 accumulate): per 16-token block
+// S[16 rows x 16 tokens] = Q K^T, the causal mask, an fp32 online softmax in
+// base 2, then O[16 x D] += P V with P rounded to the element type.
+#include "pkv_device.cuh"
+#include "pagedkv.h"
+#include "tma_host.h"
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <mutex>
+
+namespace pkv {
+namespace prefill {
+
+constexpr int kWarps = 4;                    // compute warps, 16 query rows each
+constexpr int kRows = kWarps * 16;           // query rows per CTA
+constexpr int kThreads = (kWarps + 1) * 32;  // + the producer warp
+constexpr int kBlocksPerStage = 4;           // KV blocks (64 tokens) per stage
+constexpr int kStages = 3;
+constexpr unsigned kFullMask = 0xffffffffu;
+
+template <int D>
+struct PGeo {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int kTiles = D / 64;                               // 64-column boxes per block
+    static constexpr int kBlockBytes = kTiles * 2048;                   // one block of one head, K or V
+    static constexpr int kStageBytes = 2 * kBlocksPerStage * kBlockBytes;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    static constexpr int kOffBar = kRingBytes;
+    static constexpr int kSmemBytes = kOffBar + 2 * kStages * 8 + 16 + 1024;  // + room to align the base
+};
+
+struct PrefillArgs {
+    uint16_t *out;              // [T][Hq][D]
+    const uint16_t *q;          // [T][Hq][D]
+    const int32_t *block_tables;
+    const int32_t *context_lens;
+    const int32_t *query_start;  // [B + 1]
+    int32_t *status;             // may be null
+    int B, W, Hq, Hkv, group, num_blocks, max_tiles, max_query_len;
+    float scale_log2;
+};
+
+__device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
+
+__device__ __forceinline__ void flag(const PrefillArgs &a, int bits)
+{
+    if (a.status)
+        atomicOr(a.status, bits);
+}
+
+template <class E, int D>
+__global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                           const __grid_constant__ CUtensorMap tmV,
+                                                           const PrefillArgs a)
+{
+    using G = PGeo<D>;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    const uint32_t ring = (raw_s + 1023u) & ~1023u;
+    unsigned char *base = smem_raw + (ring - raw_s);
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + G::kOffBar);
+    uint64_t *empty = full + kStages;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + kStages);
+    volatile int *zero_flag = abort_flag + 1;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.z, j = blockIdx.y;
+    const int tile = a.max_tiles - 1 - static_cast<int>(blockIdx.x);  // later rows (more KV) first
+    const int g = a.group;
+
+    // lengths and offsets: read before the grid dependency wait (the kernel
+    // launched just before must not write them)
+    const int q0 = __ldg(a.query_start + b);
+    const int n = __ldg(a.query_start + b + 1) - q0;
+    const int c = __ldg(a.context_lens + b);
+    if (n <= 0)
+        return;
+    if (n > c || c > a.W * kBlockTokens || n > a.max_query_len) {
+        if (tid == 0 && j == 0 && tile == a.max_tiles - 1)
+            flag(a, KV_STATUS_BAD_CONTEXT);
+        return;
+    }
+    const int rows_total = n * g;
+    const int row0 = tile * kRows;
+    if (row0 >= rows_total)
+        return;
+    const int p0 = c - n;  // position of the chunk's first token
+    const int last_row = min(row0 + kRows, rows_total) - 1;
+    const int kv_len = p0 + last_row / g + 1;  // tokens this CTA reads
+    const int nblk = (kv_len + kBlockTokens - 1) / kBlockTokens;
+    const int nst = (nblk + kBlocksPerStage - 1) / kBlocksPerStage;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kWarps);
+        }
+        mbar_fence_init();
+        *abort_flag = 0;
+        *zero_flag = 0;
+    }
+    __syncthreads();
+
+    if (warp == kWarps) {
+        // ---------------- producer: block ids -> TMA loads ----------------
+        if (lane == 0) {
+            tma_prefetch_descriptor(&tmK);
+            tma_prefetch_descriptor(&tmV);
+        }
+        grid_dependency_wait();  // the cache may come from the kernel before (an append)
+        grid_launch_dependents();
+        const int32_t *row = a.block_tables + static_cast<size_t>(b) * a.W;
+        int issued = 0;
+        for (int st = 0; st < nst; ++st) {
+            const int s = st % kStages;
+            const int kb0 = st * kBlocksPerStage;
+            const int nb = min(kBlocksPerStage, nblk - kb0);
+            int blk = 0;
+            if (lane < nb) {
+                blk = __ldg(row + kb0 + lane);
+                if (blk < 0 || blk >= a.num_blocks) {
+                    flag(a, KV_STATUS_BAD_BLOCK_ID);
+                    blk = 0;  // never read outside the pool
+                }
+            }
+            int ok = 1;
+            if (lane == 0) {
+                ok = mbar_wait_bounded(&empty[s], ((st / kStages) & 1) ^ 1, abort_flag);
+                if (ok)
+                    mbar_arrive_expect_tx(&full[s], nb * 2 * G::kBlockBytes);
+                else {
+                    *abort_flag = 1;
+                    flag(a, KV_STATUS_WAIT_TIMEOUT);
+                }
+            }
+            ok = __shfl_sync(kFullMask, ok, 0);
+            if (!ok)
+                break;
+            __syncwarp();
+            if (lane < nb) {
+                const uint32_t kdst = ring + s * G::kStageBytes + lane * G::kBlockBytes;
+                const uint32_t vdst = kdst + kBlocksPerStage * G::kBlockBytes;
+#pragma unroll
+                for (int t = 0; t < G::kTiles; ++t)
+                    tma_load_4d_nohint(kdst + t * 2048, &tmK, t * 64, 0, j, blk, &full[s]);
+#pragma unroll
+                for (int t = 0; t < G::kTiles; ++t)
+                    tma_load_4d_nohint(vdst + t * 2048, &tmV, t * 64, 0, j, blk, &full[s]);
+            }
+            issued = st + 1;
+        }
+        // No load may land after this CTA exits: wait (bounded) for the last ones.
+        if (lane == 0)
+            for (int st = max(0, issued - kStages); st < issued; ++st)
+                mbar_wait_bounded(&full[st % kStages], (st / kStages) & 1, zero_flag);
+        return;
+    }
+
+    // -------------------- compute warps 0..3 --------------------
+    grid_dependency_wait();  // q may come from the kernel before
+    grid_launch_dependents();
+    constexpr int kK = D / 16;  // k-steps of Q K^T, and pairs of 8-column tiles of O
+    const int r = lane >> 2, cq = lane & 3, mi = lane >> 3, rr = lane & 7;
+    const int wrow0 = row0 + warp * 16;
+    const int rowA_raw = wrow0 + r, rowB_raw = rowA_raw + 8;
+    const bool okA = rowA_raw < rows_total, okB = rowB_raw < rows_total;
+    const int rowA = min(rowA_raw, rows_total - 1), rowB = min(rowB_raw, rows_total - 1);
+    const int tokA = rowA / g, hA = rowA - tokA * g;
+    const int tokB = rowB / g, hB = rowB - tokB * g;
+    const int posA = p0 + tokA, posB = p0 + tokB;
+    const int wlast = min(wrow0 + 15, rows_total - 1);
+    const int wmin_pos = p0 + min(wrow0, rows_total - 1) / g, wmax_pos = p0 + wlast / g;
+
+    // Q as the A operand: rows A (a0, a2) and B (a1, a3)
+    uint32_t qf[kK][4];
+    {
+        const uint32_t *qa = reinterpret_cast<const uint32_t *>(
+            a.q + (static_cast<size_t>(q0 + tokA) * a.Hq + j * g + hA) * D);
+        const uint32_t *qb = reinterpret_cast<const uint32_t *>(
+            a.q + (static_cast<size_t>(q0 + tokB) * a.Hq + j * g + hB) * D);
+#pragma unroll
+        for (int kk = 0; kk < kK; ++kk) {
+            qf[kk][0] = okA ? __ldg(qa + kk * 8 + cq) : 0u;
+            qf[kk][1] = okB ? __ldg(qb + kk * 8 + cq) : 0u;
+            qf[kk][2] = okA ? __ldg(qa + kk * 8 + 4 + cq) : 0u;
+            qf[kk][3] = okB ? __ldg(qb + kk * 8 + 4 + cq) : 0u;
+        }
+    }
+    float o[2 * kK][4];
+#pragma unroll
+    for (int dt = 0; dt < 2 * kK; ++dt)
+        o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+    float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
+    const float sl2 = a.scale_log2;
+    const int last_blk = (c - 1) / kBlockTokens;  // the sequence's last block, maybe partly filled
+
+    for (int st = 0; st < nst; ++st) {
+        const int s = st % kStages;
+        if (!mbar_wait_bounded(&full[s], (st / kStages) & 1, abort_flag)) {
+            if (lane == 0) {
+                *abort_flag = 1;
+                flag(a, KV_STATUS_WAIT_TIMEOUT);
+            }
+            break;
+        }
+        const int kb0 = st * kBlocksPerStage;
+        const int nb = min(kBlocksPerStage, nblk - kb0);
+        const uint32_t kst = ring + s * G::kStageBytes;
+        const uint32_t vst = kst + kBlocksPerStage * G::kBlockBytes;
+        for (int bi = 0; bi < nb; ++bi) {
+            const int tok0 = (kb0 + bi) * kBlockTokens;
+            if (tok0 > wmax_pos)
+                break;  // after every row of this warp
+            const uint32_t kb = kst + bi * G::kBlockBytes, vb = vst + bi * G::kBlockBytes;
+            // S = Q K^T: 16 rows x 16 tokens
+            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < kK; ++kk) {
+                uint32_t bf[4];
+                ldmatrix_x4(bf, kb + (kk >> 2) * 2048 + swz(((mi >> 1) << 3) + rr, ((kk & 3) << 1) + (mi & 1)));
+                E::mma(sc[0], qf[kk], bf[0], bf[1]);
+                E::mma(sc[1], qf[kk], bf[2], bf[3]);
+            }
+            const bool need_mask = tok0 + kBlockTokens - 1 > wmin_pos;
+            float v[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int t = tok0 + nt * 8 + 2 * cq + (e & 1);
+                    const int pos = e < 2 ? posA : posB;
+                    v[nt][e] = (need_mask && t > pos) ? -INFINITY : sc[nt][e] * sl2;
+                }
+            float bmA = fmaxf(fmaxf(v[0][0], v[0][1]), fmaxf(v[1][0], v[1][1]));
+            float bmB = fmaxf(fmaxf(v[0][2], v[0][3]), fmaxf(v[1][2], v[1][3]));
+            bmA = fmaxf(bmA, __shfl_xor_sync(kFullMask, bmA, 1));
+            bmA = fmaxf(bmA, __shfl_xor_sync(kFullMask, bmA, 2));
+            bmB = fmaxf(bmB, __shfl_xor_sync(kFullMask, bmB, 1));
+            bmB = fmaxf(bmB, __shfl_xor_sync(kFullMask, bmB, 2));
+            const float nmA = fmaxf(mA, bmA), nmB = fmaxf(mB, bmB);  // finite: token 0 is in every row's range
+            const float alA = exp2f(mA - nmA), alB = exp2f(mB - nmB);
+            mA = nmA;
+            mB = nmB;
+            float p[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                p[nt][0] = exp2f(v[nt][0] - nmA);
+                p[nt][1] = exp2f(v[nt][1] - nmA);
+                p[nt][2] = exp2f(v[nt][2] - nmB);
+                p[nt][3] = exp2f(v[nt][3] - nmB);
+            }
+            lA = lA * alA + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+            lB = lB * alB + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
+            // rows of the sequence's last block past the context hold whatever the pool
+            // holds: their V halves are zeroed in the fragments so 0 * V stays 0
+            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // for tokens 2cq, 2cq+1 and 8+2cq, 9+2cq
+            if (kb0 + bi == last_blk) {
+                const int valid = c - tok0;  // 1..16
+                keep_lo = (2 * cq < valid ? 0x0000ffffu : 0u) | (2 * cq + 1 < valid ? 0xffff0000u : 0u);
+                keep_hi = (2 * cq + 8 < valid ? 0x0000ffffu : 0u) | (2 * cq + 9 < valid ? 0xffff0000u : 0u);
+            }
+            uint32_t pa[4];
+            pa[0] = E::pack(p[0][0], p[0][1]);
+            pa[1] = E::pack(p[0][2], p[0][3]);
+            pa[2] = E::pack(p[1][0], p[1][1]);
+            pa[3] = E::pack(p[1][2], p[1][3]);
+            // O += P V: pairs of 8-column tiles
+#pragma unroll
+            for (int dp = 0; dp < kK; ++dp) {
+                o[2 * dp][0] *= alA;
+                o[2 * dp][1] *= alA;
+                o[2 * dp][2] *= alB;
+                o[2 * dp][3] *= alB;
+                o[2 * dp + 1][0] *= alA;
+                o[2 * dp + 1][1] *= alA;
+                o[2 * dp + 1][2] *= alB;
+                o[2 * dp + 1][3] *= alB;
+                uint32_t vf[4];
+                ldmatrix_x4_trans(vf, vb + (dp >> 2) * 2048 + swz(((mi & 1) << 3) + rr, ((dp & 3) << 1) + (mi >> 1)));
+                vf[0] &= keep_lo;
+                vf[1] &= keep_hi;
+                vf[2] &= keep_lo;
+                vf[3] &= keep_hi;
+                E::mma(o[2 * dp], pa, vf[0], vf[1]);
+                E::mma(o[2 * dp + 1], pa, vf[2], vf[3]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(&empty[s]);
+    }
+
+    // normalise and store this lane's two rows
+    lA += __shfl_xor_sync(kFullMask, lA, 1);
+    lA += __shfl_xor_sync(kFullMask, lA, 2);
+    lB += __shfl_xor_sync(kFullMask, lB, 1);
+    lB += __shfl_xor_sync(kFullMask, lB, 2);
+    const float iA = 1.f / lA, iB = 1.f / lB;
+    uint32_t *outA = reinterpret_cast<uint32_t *>(a.out + (static_cast<size_t>(q0 + tokA) * a.Hq + j * g + hA) * D);
+    uint32_t *outB = reinterpret_cast<uint32_t *>(a.out + (static_cast<size_t>(q0 + tokB) * a.Hq + j * g + hB) * D);
+#pragma unroll
+    for (int dt = 0; dt < 2 * kK; ++dt) {
+        if (okA)
+            outA[dt * 4 + cq] = E::pack(o[dt][0] * iA, o[dt][1] * iA);
+        if (okB)
+            outB[dt * 4 + cq] = E::pack(o[dt][2] * iB, o[dt][3] * iB);
+    }
+}
+
+}  // namespace prefill
+}  // namespace pkv
+
+namespace {
+
+using PrefillFn = void (*)(const CUtensorMap, const CUtensorMap, const pkv::prefill::PrefillArgs);
+
+PrefillFn pick_prefill(int dtype, int D, int *smem)
+{
+    using namespace pkv;
+    using namespace pkv::prefill;
+    *smem = D == 64 ? PGeo<64>::kSmemBytes : PGeo<128>::kSmemBytes;
+    if (dtype == KV_DTYPE_FP16)
+        return D == 64 ? prefill_kernel<ElemF16, 64> : prefill_kernel<ElemF16, 128>;
+    return D == 64 ? prefill_kernel<ElemBf16, 64> : prefill_kernel<ElemBf16, 128>;
+}
+
+bool prepare_prefill(PrefillFn fn, int smem, int dev)
+{
+    struct Entry {
+        const void *fn;
+        int dev;
+    };
+    static std::mutex mu;
+    static Entry done[16];
+    static int used = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < used; ++i)
+        if (done[i].fn == reinterpret_cast<const void *>(fn) && done[i].dev == dev)
+            return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return false;
+    if (used < 16)
+        done[used++] = Entry{reinterpret_cast<const void *>(fn), dev};
+    return true;
+}
+
+bool misaligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+}  // namespace
+
+extern "C" kv_status paged_attention_prefill(void *out, const void *q, const void *k_cache, const void *v_cache,
+                                             const int32_t *block_tables, int max_blocks_per_seq,
+                                             const int32_t *context_lens, const int32_t *query_start, int B,
+                                             int max_query_len, int num_blocks, int Hq, int Hkv, int D, float scale,
+                                             int dtype, int32_t *error_flag, kv_stream_t stream)
+{
+    using namespace pkv::prefill;
+    if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_FP16) || B < 0 || B > 65535 || max_query_len < 0 ||
+        max_blocks_per_seq < 1 || num_blocks < 1 || Hq < 1 || Hkv < 1 || Hkv > 65535 || Hq % Hkv != 0 ||
+        (D != 64 && D != 128))
+        return KV_ERR_ARG;
+    if (B == 0 || max_query_len == 0)
+        return KV_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start)
+        return KV_ERR_ARG;
+    if (misaligned16(out) || misaligned16(q) || misaligned16(k_cache) || misaligned16(v_cache))
+        return KV_ERR_ARG;
+    const int group = Hq / Hkv;
+    const long long tiles = (static_cast<long long>(max_query_len) * group + kRows - 1) / kRows;
+    if (tiles > (1ll << 31) - 1)
+        return KV_ERR_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return KV_ERR_CUDA;
+    int smem = 0;
+    PrefillFn fn = pick_prefill(dtype, D, &smem);
+    if (!prepare_prefill(fn, smem, dev))
+        return KV_ERR_CUDA;
+    CUtensorMap tmK, tmV;
+    if (!pkv_host::make_cache_map(&tmK, k_cache, num_blocks, Hkv, D, 1, dtype) ||
+        !pkv_host::make_cache_map(&tmV, v_cache, num_blocks, Hkv, D, 1, dtype))
+        return KV_ERR_CUDA;
+    PrefillArgs a;
+    a.out = static_cast<uint16_t *>(out);
+    a.q = static_cast<const uint16_t *>(q);
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.query_start = query_start;
+    a.status = error_flag;
+    a.B = B;
+    a.W = max_blocks_per_seq;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.group = group;
+    a.num_blocks = num_blocks;
+    a.max_tiles = static_cast<int>(tiles);
+    a.max_query_len = max_query_len;
+    a.scale_log2 = scale * 1.4426950408889634f;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, tmK, tmV, a) == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}

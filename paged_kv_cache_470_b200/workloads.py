@@ -218,3 +218,91 @@ def make_step_inputs(cfg: DecodeConfig, gen: torch.Generator, device, n_layers=N
 def small_config(cid: int = 1, **overrides) -> DecodeConfig:
     """A copy of one workload with some fields changed (edge-case and CPU-sized tests)."""
     return replace(CONFIGS[cid], **overrides)
+
+
+# ---------------------------------------------------------------------------
+# Chunked prefill ("Module 23: Serving", section 23.2; "Designing an LLM serving
+# system", section "Scheduling: when prefill meets decode"): each sequence adds a
+# chunk of new tokens on top of what it already holds in the cache.
+# ---------------------------------------------------------------------------
+@dataclass(frozen=True)
+class PrefillConfig:
+    name: str
+    Hq: int
+    Hkv: int
+    D: int
+    batch: int
+    chunk: int                    # new tokens per sequence
+    prior_lo: int                 # tokens already cached before the chunk: U[prior_lo, prior_hi]
+    prior_hi: int
+    W: int
+    seed: int = 4700
+    elem: str = "bf16"
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.float16 if self.elem == "fp16" else torch.bfloat16
+
+
+PREFILL_CONFIGS = {
+    "llama3_8b": PrefillConfig("chunked prefill, LLaMA-3-8B shape (Hq=32, Hkv=8, D=128): 16 sequences, "
+                               "512-token chunks on U[0,3584] cached tokens, one layer", 32, 8, 128, 16, 512, 0,
+                               3584, 256),
+    "0p5b": PrefillConfig("chunked prefill, 0.5B GQA shape (Hq=20, Hkv=4, D=64): 16 sequences, "
+                          "512-token chunks on U[0,3584] cached tokens, one layer", 20, 4, 64, 16, 512, 0, 3584, 256,
+                          seed=4701),
+}
+
+
+@dataclass
+class PrefillLayout:
+    num_blocks: int
+    context_lens: torch.Tensor    # [B] int32, chunk included
+    chunk_lens: torch.Tensor      # [B] int32
+    query_start: torch.Tensor     # [B+1] int32
+    block_tables: torch.Tensor    # [B, W] int32, -1 past each sequence's blocks
+
+    def slot_mapping(self) -> torch.Tensor:
+        """int64 slot of every chunk token, in q's row order (for kv_cache_append)."""
+        out = []
+        for b in range(self.block_tables.shape[0]):
+            c, n = int(self.context_lens[b]), int(self.chunk_lens[b])
+            for p in range(c - n, c):
+                out.append(int(self.block_tables[b, p // BLOCK_TOKENS]) * BLOCK_TOKENS + p % BLOCK_TOKENS)
+        return torch.tensor(out, dtype=torch.int64)
+
+
+def draw_prefill_layout(cfg: PrefillConfig, chunk_lens=None, prior_lens=None, seed=None) -> PrefillLayout:
+    """Chunk and prior lengths, and the sequences' blocks scattered over a shuffled pool."""
+    gen = cpu_generator(cfg.seed if seed is None else seed)
+    B = cfg.batch
+    if prior_lens is None:
+        prior_lens = torch.randint(cfg.prior_lo, cfg.prior_hi + 1, (B,), generator=gen).tolist()
+    if chunk_lens is None:
+        chunk_lens = [cfg.chunk] * B
+    lens = [int(p) + int(n) for p, n in zip(prior_lens, chunk_lens)]
+    need = sum(-(-c // BLOCK_TOKENS) for c in lens)
+    num_blocks = max(1, int(need * 1.08) + 16)
+    perm = torch.randperm(num_blocks, generator=gen).tolist()
+    tables = torch.full((B, cfg.W), -1, dtype=torch.int32)
+    cur = 0
+    for b, c in enumerate(lens):
+        nb = -(-c // BLOCK_TOKENS)
+        if nb > cfg.W:
+            raise ValueError("context longer than the table")
+        tables[b, :nb] = torch.tensor(perm[cur:cur + nb], dtype=torch.int32)
+        cur += nb
+    qs = [0]
+    for n in chunk_lens:
+        qs.append(qs[-1] + int(n))
+    return PrefillLayout(num_blocks, torch.tensor(lens, dtype=torch.int32),
+                         torch.tensor([int(n) for n in chunk_lens], dtype=torch.int32),
+                         torch.tensor(qs, dtype=torch.int32), tables)

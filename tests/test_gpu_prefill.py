@@ -1,0 +1,114 @@
+"""GPU parity of chunked-prefill attention (paged_attention_prefill) against the
+oracle, which states a query at position p as a decode over p + 1 tokens:
+within |gpu - ref| <= 5e-3 + 1e-2 |ref| elementwise. The chunk's K/V are
+appended with kv_cache_append first, and that append is checked bit-exactly.
+"""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_470_b200 import workloads
+from gpu_cases import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+class PrefillCase:
+    def __init__(self, cfg, device, chunk_lens=None, prior_lens=None, seed=None):
+        self.cfg = cfg
+        self.layout = workloads.draw_prefill_layout(cfg, chunk_lens=chunk_lens, prior_lens=prior_lens, seed=seed)
+        gen = workloads.device_generator(cfg.seed if seed is None else seed, device)
+        dt = cfg.torch_dtype
+        self.k, self.v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device, dt)
+        T = int(self.layout.query_start[-1])
+        self.q = workloads.random_bf16((T, cfg.Hq, cfg.D), gen, device, dt)
+        self.k_new = workloads.random_bf16((T, cfg.Hkv, cfg.D), gen, device, dt)
+        self.v_new = workloads.random_bf16((T, cfg.Hkv, cfg.D), gen, device, dt)
+        self.tables = self.layout.block_tables.to(device)
+        self.lens = self.layout.context_lens.to(device)
+        self.qs = self.layout.query_start.to(device)
+        self.slots = self.layout.slot_mapping().to(device)
+        self.max_q = int(self.layout.chunk_lens.max()) if self.layout.chunk_lens.numel() else 0
+
+
+def run_case(pkv, oracle_mod, case, what, rows=None):
+    cfg = case.cfg
+    k_host, v_host = case.k.cpu(), case.v.cpu()
+    flag = torch.zeros(1, dtype=torch.int32, device=case.q.device)
+    pkv.kv_cache_append(case.k_new, case.v_new, case.k, case.v, case.slots, flag)
+    out = torch.full_like(case.q, float("nan"))
+    pkv.paged_attention_prefill(out, case.q, case.k, case.v, case.tables, case.lens, case.qs, case.max_q, cfg.scale,
+                                flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) == 0
+    k2, v2 = oracle_mod.kv_cache_append(k_host, v_host, case.k_new.cpu(), case.v_new.cpu(),
+                                        case.layout.slot_mapping().numpy())
+    assert np.array_equal(bits(case.k), k2) and np.array_equal(bits(case.v), v2), f"{what}: append not bit-exact"
+    seqs = range(cfg.batch) if rows is None else rows
+    qs = case.layout.query_start.numpy()
+    for b in seqs:
+        lo, hi = int(qs[b]), int(qs[b + 1])
+        if hi == lo:
+            continue
+        ref = oracle_mod.paged_attention_prefill(bits(case.q[lo:hi]), k2, v2, case.layout.block_tables.numpy()[b:b + 1],
+                                                 case.layout.context_lens.numpy()[b:b + 1], np.array([0, hi - lo]),
+                                                 cfg.scale, dtype=cfg.elem)
+        compare(out[lo:hi], ref, f"{what}, sequence {b}")
+    return out
+
+
+@pytest.mark.parametrize("elem", ["bf16", "fp16"])
+@pytest.mark.parametrize("Hq,Hkv,D", [(20, 4, 64), (32, 8, 128), (8, 8, 128), (12, 1, 64), (16, 2, 128), (6, 6, 64)])
+def test_prefill_chunks(pkv, oracle_mod, cuda_device, Hq, Hkv, D, elem):
+    """Whole prompts, chunks over a cached prefix, single tokens and empty chunks; lengths at and
+    around block edges."""
+    chunk = [37, 1, 16, 100, 0, 64, 17, 5]
+    prior = [0, 250, 15, 33, 40, 0, 111, 1]
+    cfg = workloads.PrefillConfig("test", Hq, Hkv, D, len(chunk), 0, 0, 0, 16, seed=Hq * 7 + D, elem=elem)
+    case = PrefillCase(cfg, cuda_device, chunk_lens=chunk, prior_lens=prior)
+    run_case(pkv, oracle_mod, case, f"prefill {Hq}/{Hkv} D{D} {elem}")
+
+
+def test_single_token_chunk_matches_the_decode(pkv, cuda_device):
+    """A one-token chunk is a decode step: both kernels agree to within rounding."""
+    cfg = workloads.PrefillConfig("test", 32, 8, 128, 4, 1, 100, 700, 64, seed=3)
+    case = PrefillCase(cfg, cuda_device)
+    pkv.kv_cache_append(case.k_new, case.v_new, case.k, case.v, case.slots)
+    out_p = torch.empty_like(case.q)
+    pkv.paged_attention_prefill(out_p, case.q, case.k, case.v, case.tables, case.lens, case.qs, 1, cfg.scale)
+    out_d = torch.empty_like(case.q)
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    pkv.paged_attention_decode(out_d, case.q, case.k, case.v, case.tables, case.lens, cfg.scale, ws)
+    torch.cuda.synchronize()
+    d = (out_p.float() - out_d.float()).abs()
+    assert float(d.max()) <= 2e-2, float(d.max())
+
+
+def test_full_size_prefill_workload(pkv, oracle_mod, cuda_device):
+    """The bench's prefill workload (LLaMA-3-8B shape), three of its sequences against the oracle."""
+    cfg = workloads.PREFILL_CONFIGS["llama3_8b"]
+    case = PrefillCase(cfg, cuda_device)
+    run_case(pkv, oracle_mod, case, "full-size prefill", rows=[0, 7, 15])
+
+
+def test_bad_chunks_are_flagged(pkv, cuda_device):
+    cfg = workloads.PrefillConfig("test", 8, 2, 64, 3, 10, 20, 40, 8, seed=5)
+    case = PrefillCase(cfg, cuda_device)
+    out = torch.zeros_like(case.q)
+    flag = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    lens = case.lens.clone()
+    lens[1] = 5                                   # shorter than its 10-token chunk
+    pkv.paged_attention_prefill(out, case.q, case.k, case.v, case.tables, lens, case.qs, case.max_q, cfg.scale, flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) & pkv.KV_STATUS_BAD_CONTEXT
+    assert not out[10:20].any()                   # that sequence's rows are not written
+    flag.zero_()
+    tables = case.tables.clone()
+    tables[0, 0] = 10 ** 6                        # outside the pool
+    pkv.paged_attention_prefill(out, case.q, case.k, case.v, tables, case.lens, case.qs, case.max_q, cfg.scale, flag)
+    torch.cuda.synchronize()
+    assert int(flag.item()) & pkv.KV_STATUS_BAD_BLOCK_ID
