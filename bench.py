@@ -47,6 +47,7 @@ from paged_kv_cache_470_b200 import workloads  # noqa: E402  (no CUDA library ne
 
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_470_b200", "csrc", "decode.cu")
 
@@ -85,6 +86,15 @@ def measured_peak():
             return float(json.load(f)["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor throughput of this machine's B200s (a kernel timed alone: the burst figure)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured cuBLAS bf16 GEMM (burst)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def profiled_traffic(cfg):
@@ -378,6 +388,51 @@ def block_moves_measure(wl, peak, reps=10):
     return res
 
 
+def prefill_measure(pkv, device, elem, reps=20, keys=("llama3_8b", "0p5b")):
+    """The chunked-prefill workloads: one layer's paged_attention_prefill each, timed with CUDA events.
+    Algorithmic flops = 4 * Hq * D per (query, visible token) pair (Q K^T and P V, a multiply-add = 2)."""
+    from dataclasses import replace
+    peak, kind = measured_tensor_peak()
+    res = {}
+    for key in keys:
+        cfg = replace(workloads.PREFILL_CONFIGS[key], elem=elem)
+        layout = workloads.draw_prefill_layout(cfg)
+        gen = workloads.device_generator(cfg.seed, device)
+        k, v = workloads.make_layer_cache(layout.num_blocks, cfg.Hkv, cfg.D, gen, device, cfg.torch_dtype)
+        T = int(layout.query_start[-1])
+        q = workloads.random_bf16((T, cfg.Hq, cfg.D), gen, device, cfg.torch_dtype)
+        out = torch.empty_like(q)
+        tables, lens, qs = (layout.block_tables.to(device), layout.context_lens.to(device),
+                            layout.query_start.to(device))
+        flag = torch.zeros(1, dtype=torch.int32, device=device)
+        pairs = sum(sum(int(c) - int(n) + i + 1 for i in range(int(n)))
+                    for c, n in zip(layout.context_lens.tolist(), layout.chunk_lens.tolist()))
+        flops = 4.0 * cfg.Hq * cfg.D * pairs
+        stream = torch.cuda.current_stream()
+
+        def one():
+            pkv.paged_attention_prefill(out, q, k, v, tables, lens, qs, cfg.chunk, cfg.scale, flag, stream=stream)
+        for _ in range(3):
+            one()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            one()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        tf = flops / (ms * 1e-3) / 1e12
+        res[key] = {"workload": cfg.name, "bound": "tensor", "achieved": round(tf, 1), "unit": "TFLOP/s",
+                    "peak": peak, "peak_kind": kind, "frac": round(tf / peak, 4), "ms": round(ms, 4),
+                    "flops_per_launch": flops, "status": int(flag.item()),
+                    "arithmetic": f"mma.sync m16n8k16 {elem} in, fp32 accumulate",
+                    "timing": f"CUDA events, mean of {reps} back-to-back launches after 3 warm-up launches; "
+                              f"KV {2 * k.numel() * k.element_size() / 1e6:.0f} MB + q "
+                              f"{q.numel() * q.element_size() / 1e6:.0f} MB per launch (L2 126 MB)"}
+        del k, v, q, out
+    return res
+
+
 def e2e_measure(wl, steps, warmup, world):
     """The same step through the C ABI with host buffers: H2D of the step's inputs, D2H of its outputs."""
     cfg = wl.cfg
@@ -471,6 +526,10 @@ def run_ours(args, world, rank, local):
         pkv.set_option(pkv.KV_OPT_ITEM_COST, args.item_cost)
     if args.profile_step:
         return run_profile_step(args, cfg, device)
+    if args.profile_prefill:
+        r = prefill_measure(pkv, device, cfg.elem, reps=args.steps, keys=(args.profile_prefill,))
+        print(json.dumps(r), flush=True)
+        return
     wl = Workload(cfg, device, rank)
     wl.fused = not args.separate_append
     lens = [int(c) for c in wl.layout.context_lens]
@@ -514,6 +573,7 @@ def run_ours(args, world, rank, local):
 
     e2e_ms, h2d, d2h = e2e_measure(wl, max(args.steps // 4, 3), args.warmup, world)
     moves = block_moves_measure(wl, peak)
+    prefill = prefill_measure(pkv, device, cfg.elem)
     e2e_ms = dist_max(e2e_ms, world)
 
     cpu = None
@@ -571,6 +631,7 @@ def run_ours(args, world, rank, local):
         "device_status": status,
         "cpu_baseline": cpu,
         "block_moves": moves,
+        "prefill": prefill,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -620,6 +681,8 @@ def main(argv=None):
     ap.add_argument("--reference-budget", type=float, default=120.0)
     ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling a smaller case)")
     ap.add_argument("--profile-step", action="store_true", help="only replay the step graph (for ncu)")
+    ap.add_argument("--profile-prefill", choices=sorted(workloads.PREFILL_CONFIGS), default=None,
+                    help="only run the chunked-prefill workload: 3 warm-up and --steps timed launches (for ncu)")
     ap.add_argument("--grid", type=int, default=0, help="decode CTAs per launch (0: one per SM)")
     ap.add_argument("--combine-kernel", action="store_true", help="split-K merge in a separate kernel")
     ap.add_argument("--head-group", type=int, default=0, help="kv heads per work unit (0: auto)")

@@ -19,9 +19,10 @@
 // Pipeline. Warp 4 is the producer: it reads block ids and issues TMA loads of
 // 4 KV blocks (64 tokens) per stage into a ring of 3 stages, guarded by
 // mbarriers with bounded waits. Warps 0-3 compute with tensor cores
-// (mma.sync.m16n8k16, 16-bit inputs, fp32 accumulate): per 16-token block
-// S[16 rows x 16 tokens] = Q K^T, the causal mask, an fp32 online softmax in
-// base 2, then O[16 x D] += P V with P rounded to the element type.
+// (mma.sync.m16n8k16, 16-bit inputs, fp32 accumulate): per stage
+// S[16 rows x 64 tokens] = Q K^T, the causal mask, an fp32 online softmax in
+// base 2 (one rescale of O per stage), then O[16 x D] += P V with P rounded to
+// the element type.
 #include "pkv_device.cuh"
 #include "pagedkv.h"
 #include "tma_host.h"
@@ -72,11 +73,12 @@ __device__ __forceinline__ void flag(const PrefillArgs &a, int bits)
 }
 
 template <class E, int D>
-__global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_constant__ CUtensorMap tmK,
                                                            const __grid_constant__ CUtensorMap tmV,
                                                            const PrefillArgs a)
 {
     using G = PGeo<D>;
+    constexpr int kBPI = D == 128 ? 2 : 4;  // KV blocks per softmax pass
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
     const uint32_t ring = (raw_s + 1023u) & ~1023u;
@@ -227,35 +229,57 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
             break;
         }
         const int kb0 = st * kBlocksPerStage;
-        const int nb = min(kBlocksPerStage, nblk - kb0);
-        const uint32_t kst = ring + s * G::kStageBytes;
-        const uint32_t vst = kst + kBlocksPerStage * G::kBlockBytes;
-        for (int bi = 0; bi < nb; ++bi) {
-            const int tok0 = (kb0 + bi) * kBlockTokens;
-            if (tok0 > wmax_pos)
-                break;  // after every row of this warp
-            const uint32_t kb = kst + bi * G::kBlockBytes, vb = vst + bi * G::kBlockBytes;
-            // S = Q K^T: 16 rows x 16 tokens
-            float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        const int tok_s = kb0 * kBlockTokens;
+        // blocks of this stage that some row of this warp can see (the rest are after all of them)
+        const int nbw = wmax_pos < tok_s ? 0
+                                         : min(min(kBlocksPerStage, nblk - kb0), (wmax_pos - tok_s) / kBlockTokens + 1);
+        const uint32_t kst0 = ring + s * G::kStageBytes;
+        const uint32_t vst0 = kst0 + kBlocksPerStage * G::kBlockBytes;
+#pragma unroll 1
+        for (int grp = 0; grp < nbw; grp += kBPI) {
+            // blocks grp .. grp + kBPI - 1 of the stage, kept to kBPI per pass to bound registers
+            const uint32_t kst = kst0 + grp * G::kBlockBytes, vst = vst0 + grp * G::kBlockBytes;
+            const int nbg = min(kBPI, nbw - grp);
+            const int tok_g = tok_s + grp * kBlockTokens;
+            const int kbg = kb0 + grp;
+            // S = Q K^T: 16 rows x up to 16 * kBPI tokens, as [block][8-token tile][4]
+            float sc[kBPI][2][4];
+#pragma unroll
+            for (int bi = 0; bi < kBPI; ++bi)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    sc[bi][nt][0] = sc[bi][nt][1] = sc[bi][nt][2] = sc[bi][nt][3] = 0.f;
 #pragma unroll
             for (int kk = 0; kk < kK; ++kk) {
-                uint32_t bf[4];
-                ldmatrix_x4(bf, kb + (kk >> 2) * 2048 + swz(((mi >> 1) << 3) + rr, ((kk & 3) << 1) + (mi & 1)));
-                E::mma(sc[0], qf[kk], bf[0], bf[1]);
-                E::mma(sc[1], qf[kk], bf[2], bf[3]);
-            }
-            const bool need_mask = tok0 + kBlockTokens - 1 > wmin_pos;
-            float v[2][4];
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int t = tok0 + nt * 8 + 2 * cq + (e & 1);
-                    const int pos = e < 2 ? posA : posB;
-                    v[nt][e] = (need_mask && t > pos) ? -INFINITY : sc[nt][e] * sl2;
+                for (int bi = 0; bi < kBPI; ++bi) {
+                    if (bi < nbg) {
+                        uint32_t bf[4];
+                        ldmatrix_x4(bf, kst + bi * G::kBlockBytes + (kk >> 2) * 2048 +
+                                            swz(((mi >> 1) << 3) + rr, ((kk & 3) << 1) + (mi & 1)));
+                        E::mma(sc[bi][0], qf[kk], bf[0], bf[1]);
+                        E::mma(sc[bi][1], qf[kk], bf[2], bf[3]);
+                    }
                 }
-            float bmA = fmaxf(fmaxf(v[0][0], v[0][1]), fmaxf(v[1][0], v[1][1]));
-            float bmB = fmaxf(fmaxf(v[0][2], v[0][3]), fmaxf(v[1][2], v[1][3]));
+            }
+            const bool need_mask = tok_g + nbg * kBlockTokens - 1 > wmin_pos;
+            float bmA = -INFINITY, bmB = -INFINITY;
+#pragma unroll
+            for (int bi = 0; bi < kBPI; ++bi)
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int t = tok_g + bi * kBlockTokens + nt * 8 + 2 * cq + (e & 1);
+                        const int pos = e < 2 ? posA : posB;
+                        const bool vis = bi < nbg && (!need_mask || t <= pos);
+                        const float x = vis ? sc[bi][nt][e] * sl2 : -INFINITY;
+                        sc[bi][nt][e] = x;
+                        if (e < 2)
+                            bmA = fmaxf(bmA, x);
+                        else
+                            bmB = fmaxf(bmB, x);
+                    }
             bmA = fmaxf(bmA, __shfl_xor_sync(kFullMask, bmA, 1));
             bmA = fmaxf(bmA, __shfl_xor_sync(kFullMask, bmA, 2));
             bmB = fmaxf(bmB, __shfl_xor_sync(kFullMask, bmB, 1));
@@ -264,48 +288,58 @@ __global__ void __launch_bounds__(kThreads) prefill_kernel(const __grid_constant
             const float alA = exp2f(mA - nmA), alB = exp2f(mB - nmB);
             mA = nmA;
             mB = nmB;
-            float p[2][4];
+            float sumA = 0.f, sumB = 0.f;
 #pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-                p[nt][0] = exp2f(v[nt][0] - nmA);
-                p[nt][1] = exp2f(v[nt][1] - nmA);
-                p[nt][2] = exp2f(v[nt][2] - nmB);
-                p[nt][3] = exp2f(v[nt][3] - nmB);
-            }
-            lA = lA * alA + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-            lB = lB * alB + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-            // rows of the sequence's last block past the context hold whatever the pool
-            // holds: their V halves are zeroed in the fragments so 0 * V stays 0
-            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // for tokens 2cq, 2cq+1 and 8+2cq, 9+2cq
-            if (kb0 + bi == last_blk) {
-                const int valid = c - tok0;  // 1..16
-                keep_lo = (2 * cq < valid ? 0x0000ffffu : 0u) | (2 * cq + 1 < valid ? 0xffff0000u : 0u);
-                keep_hi = (2 * cq + 8 < valid ? 0x0000ffffu : 0u) | (2 * cq + 9 < valid ? 0xffff0000u : 0u);
-            }
-            uint32_t pa[4];
-            pa[0] = E::pack(p[0][0], p[0][1]);
-            pa[1] = E::pack(p[0][2], p[0][3]);
-            pa[2] = E::pack(p[1][0], p[1][1]);
-            pa[3] = E::pack(p[1][2], p[1][3]);
-            // O += P V: pairs of 8-column tiles
+            for (int bi = 0; bi < kBPI; ++bi)
 #pragma unroll
-            for (int dp = 0; dp < kK; ++dp) {
-                o[2 * dp][0] *= alA;
-                o[2 * dp][1] *= alA;
-                o[2 * dp][2] *= alB;
-                o[2 * dp][3] *= alB;
-                o[2 * dp + 1][0] *= alA;
-                o[2 * dp + 1][1] *= alA;
-                o[2 * dp + 1][2] *= alB;
-                o[2 * dp + 1][3] *= alB;
-                uint32_t vf[4];
-                ldmatrix_x4_trans(vf, vb + (dp >> 2) * 2048 + swz(((mi & 1) << 3) + rr, ((dp & 3) << 1) + (mi >> 1)));
-                vf[0] &= keep_lo;
-                vf[1] &= keep_hi;
-                vf[2] &= keep_lo;
-                vf[3] &= keep_hi;
-                E::mma(o[2 * dp], pa, vf[0], vf[1]);
-                E::mma(o[2 * dp + 1], pa, vf[2], vf[3]);
+                for (int nt = 0; nt < 2; ++nt) {
+                    sc[bi][nt][0] = exp2f(sc[bi][nt][0] - nmA);
+                    sc[bi][nt][1] = exp2f(sc[bi][nt][1] - nmA);
+                    sc[bi][nt][2] = exp2f(sc[bi][nt][2] - nmB);
+                    sc[bi][nt][3] = exp2f(sc[bi][nt][3] - nmB);
+                    sumA += sc[bi][nt][0] + sc[bi][nt][1];
+                    sumB += sc[bi][nt][2] + sc[bi][nt][3];
+                }
+            lA = lA * alA + sumA;
+            lB = lB * alB + sumB;
+#pragma unroll
+            for (int dt = 0; dt < 2 * kK; ++dt) {
+                o[dt][0] *= alA;
+                o[dt][1] *= alA;
+                o[dt][2] *= alB;
+                o[dt][3] *= alB;
+            }
+            // O += P V, one 16-token block (the k dimension) at a time
+#pragma unroll
+            for (int bi = 0; bi < kBPI; ++bi) {
+                if (bi < nbg) {
+                    // rows of the sequence's last block past the context hold whatever the pool
+                    // holds: their V halves are zeroed in the fragments so 0 * V stays 0
+                    uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;  // tokens 2cq, 2cq+1 / 8+2cq, 9+2cq
+                    if (kbg + bi == last_blk) {
+                        const int valid = c - (tok_g + bi * kBlockTokens);  // 1..16
+                        keep_lo = (2 * cq < valid ? 0x0000ffffu : 0u) | (2 * cq + 1 < valid ? 0xffff0000u : 0u);
+                        keep_hi = (2 * cq + 8 < valid ? 0x0000ffffu : 0u) | (2 * cq + 9 < valid ? 0xffff0000u : 0u);
+                    }
+                    uint32_t pa[4];
+                    pa[0] = E::pack(sc[bi][0][0], sc[bi][0][1]);
+                    pa[1] = E::pack(sc[bi][0][2], sc[bi][0][3]);
+                    pa[2] = E::pack(sc[bi][1][0], sc[bi][1][1]);
+                    pa[3] = E::pack(sc[bi][1][2], sc[bi][1][3]);
+                    const uint32_t vb = vst + bi * G::kBlockBytes;
+#pragma unroll
+                    for (int dp = 0; dp < kK; ++dp) {
+                        uint32_t vf[4];
+                        ldmatrix_x4_trans(vf, vb + (dp >> 2) * 2048 +
+                                                  swz(((mi & 1) << 3) + rr, ((dp & 3) << 1) + (mi >> 1)));
+                        vf[0] &= keep_lo;
+                        vf[1] &= keep_hi;
+                        vf[2] &= keep_lo;
+                        vf[3] &= keep_hi;
+                        E::mma(o[2 * dp], pa, vf[0], vf[1]);
+                        E::mma(o[2 * dp + 1], pa, vf[2], vf[3]);
+                    }
+                }
             }
         }
         __syncwarp();
