@@ -252,19 +252,23 @@ class Workload:
         self.lens.copy_(self.layout.context_lens)
         self.slots.copy_(self.layout.slot_mapping())
 
-    def step(self, stream=None):
-        """Every layer: append this step's token and attend (one fused launch, or two kernels)."""
+    def layer(self, layer, stream=None):
+        """One layer: append this step's token and attend (one fused launch, or two kernels)."""
         pkv, cfg = self.pkv, self.cfg
-        for layer in range(cfg.n_layers):
-            if self.fused:
-                pkv.paged_attention_decode_append(self.out[layer], self.q[layer], self.k_new[layer],
-                                                  self.v_new[layer], self.k[layer], self.v[layer], self.slots,
-                                                  self.tables, self.lens, cfg.scale, self.ws, stream=stream)
-            else:
-                pkv.kv_cache_append(self.k_new[layer], self.v_new[layer], self.k[layer], self.v[layer], self.slots,
-                                    stream=stream)
-                pkv.paged_attention_decode(self.out[layer], self.q[layer], self.k[layer], self.v[layer],
-                                           self.tables, self.lens, cfg.scale, self.ws, stream=stream)
+        if self.fused:
+            pkv.paged_attention_decode_append(self.out[layer], self.q[layer], self.k_new[layer],
+                                              self.v_new[layer], self.k[layer], self.v[layer], self.slots,
+                                              self.tables, self.lens, cfg.scale, self.ws, stream=stream)
+        else:
+            pkv.kv_cache_append(self.k_new[layer], self.v_new[layer], self.k[layer], self.v[layer], self.slots,
+                                stream=stream)
+            pkv.paged_attention_decode(self.out[layer], self.q[layer], self.k[layer], self.v[layer],
+                                       self.tables, self.lens, cfg.scale, self.ws, stream=stream)
+
+    def step(self, stream=None):
+        """Every layer, in order."""
+        for layer in range(self.cfg.n_layers):
+            self.layer(layer, stream)
 
 
 def capture(fn):
@@ -433,23 +437,77 @@ def prefill_measure(pkv, device, elem, reps=20, keys=("llama3_8b", "0p5b")):
     return res
 
 
-def e2e_measure(wl, steps, warmup, world):
-    """The same step through the C ABI with host buffers: H2D of the step's inputs, D2H of its outputs."""
+def gpu_local_cpus(device_index: int):
+    """The host CPUs nearest the GPU (NVML's CPU affinity), or None."""
+    try:
+        import pynvml
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+        words = pynvml.nvmlDeviceGetCpuAffinity(h, (os.cpu_count() + 63) // 64)
+        cpus = {w * 64 + bit for w, mask in enumerate(words) for bit in range(64) if (int(mask) >> bit) & 1}
+        cpus &= os.sched_getaffinity(0)
+        return cpus or None
+    except Exception:
+        return None
+
+
+def pinned_near(tensors, device_index: int):
+    """Pinned host copies of the tensors, first touched from the CPUs nearest the GPU (NUMA-local pages)."""
+    old = os.sched_getaffinity(0)
+    near = gpu_local_cpus(device_index)
+    try:
+        if near:
+            os.sched_setaffinity(0, near)
+        return [t.cpu().pin_memory() for t in tensors]
+    finally:
+        if near:
+            os.sched_setaffinity(0, old)
+
+
+def e2e_measure(wl, steps, warmup, world, chunks=4):
+    """The same step through the C ABI with host buffers: every step copies its inputs from pinned host
+    memory and its outputs back. The copies run on two side streams, pipelined with the layers: the tables,
+    lengths and slots, then q, k_new and v_new in `chunks` groups of layers, each ahead of its first launch;
+    each layer's output is copied back while later layers run -- as a serving loop would. One CUDA graph.
+    The host buffers are pinned pages on the GPU's NUMA node."""
     cfg = wl.cfg
-    host_in = {name: t.cpu().pin_memory() for name, t in
-               (("q", wl.q), ("k_new", wl.k_new), ("v_new", wl.v_new), ("tables", wl.tables),
-                ("lens", wl.lens), ("slots", wl.slots))}
-    dev_in = {"q": wl.q, "k_new": wl.k_new, "v_new": wl.v_new, "tables": wl.tables, "lens": wl.lens,
-              "slots": wl.slots}
-    host_out = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    L = cfg.n_layers
+    dev_index = wl.q.device.index or 0
+    step_in = {"tables": wl.tables, "lens": wl.lens, "slots": wl.slots}
+    layer_in = {"q": wl.q, "k_new": wl.k_new, "v_new": wl.v_new}
+    names = list(step_in) + list(layer_in)
+    pinned = pinned_near([step_in.get(k, layer_in.get(k)) for k in names] + [wl.out], dev_index)
+    host = dict(zip(names, pinned[:-1]))
+    host_out = pinned[-1]
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = host_out.numel() * host_out.element_size()
+    h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+    per = -(-L // chunks)
+    ev_in = [torch.cuda.Event() for _ in range(chunks)]
+    ev_done = [torch.cuda.Event() for _ in range(L)]
 
     def one():
-        for name, t in host_in.items():
-            dev_in[name].copy_(t, non_blocking=True)
-        wl.step()
-        host_out.copy_(wl.out, non_blocking=True)
+        main = torch.cuda.current_stream()
+        h2d_stream.wait_stream(main)
+        d2h_stream.wait_stream(main)
+        with torch.cuda.stream(h2d_stream):
+            for k in step_in:
+                step_in[k].copy_(host[k], non_blocking=True)
+            for c in range(chunks):
+                lo, hi = c * per, min(L, (c + 1) * per)
+                for k in layer_in:
+                    layer_in[k][lo:hi].copy_(host[k][lo:hi], non_blocking=True)
+                ev_in[c].record(h2d_stream)
+        for layer in range(L):
+            if layer % per == 0:
+                main.wait_event(ev_in[layer // per])
+            wl.layer(layer)
+            ev_done[layer].record(main)
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(ev_done[layer])
+                host_out[layer].copy_(wl.out[layer], non_blocking=True)
+        main.wait_stream(h2d_stream)
+        main.wait_stream(d2h_stream)
 
     g = capture(one)
     for _ in range(warmup):
@@ -624,7 +682,9 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "api": ("paged_attention_decode_append" if wl.fused else "kv_cache_append + paged_attention_decode")
-                       + " per layer, captured in a CUDA graph with the copies"},
+                       + " per layer; inputs copied host-to-device on a side stream in 4 groups of layers ahead "
+                         "of their launches, each layer's output copied back on another behind it, all in one "
+                         "CUDA graph; pinned host buffers on the GPU's NUMA node"},
         "gpu_launches": ((1 if wl.fused else 2) + (pkv.get_option(pkv.KV_OPT_COMBINE) == 1))
                         * cfg.n_layers * args.steps,
         "clocks": clk.summary(),
