@@ -266,6 +266,8 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     group and query-head chunk) adds this many more for its
  *                     fixed cost; CTAs take equal ranges of positions.
  *                     0 auto, -1 none, 1..64 that many.
+ *   KV_OPT_PREFILL_PATH: paged_attention_prefill on 0 auto (tcgen05), 1
+ *                     tcgen05.mma with tensor-memory accumulators, 2 mma.sync.
  * Kernels are launched with programmatic dependent launch. q, k_new, v_new,
  * the caches, the workspace and out are touched only after the previous kernel
  * in the stream has completed; block_tables and context_lens are read before
@@ -279,6 +281,7 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
 #define KV_OPT_PRODUCER_LANES 5
 #define KV_OPT_HEAD_GROUP 6
 #define KV_OPT_ITEM_COST 7
+#define KV_OPT_PREFILL_PATH 8
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

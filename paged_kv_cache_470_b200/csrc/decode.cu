@@ -1326,6 +1326,7 @@ std::atomic<int> g_opt_min_chunk{0};
 std::atomic<int> g_opt_prod_lanes{0};
 std::atomic<int> g_opt_head_group{0};
 std::atomic<int> g_opt_item_cost{0};
+std::atomic<int> g_opt_prefill_path{0};
 constexpr int kDefaultMinChunk = 4;
 
 // Work positions charged per work item (its fixed cost, in units of one work
@@ -1753,6 +1754,11 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_item_cost.store(value);
         return KV_OK;
+    case KV_OPT_PREFILL_PATH:
+        if (value < 0 || value > 2)
+            return KV_ERR_ARG;
+        g_opt_prefill_path.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -1775,7 +1781,12 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_head_group.load();
     case KV_OPT_ITEM_COST:
         return g_opt_item_cost.load();
+    case KV_OPT_PREFILL_PATH:
+        return g_opt_prefill_path.load();
     default:
         return -1;
     }
 }
+
+// The prefill path switch (read by prefill.cu).
+int pkv_prefill_path() { return g_opt_prefill_path.load(); }

@@ -364,12 +364,391 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
     }
 }
 
+// ===========================================================================
+// tcgen05 path. The same computation on the 5th-generation tensor cores: a CTA
+// takes 128 query rows; S = Q K^T (M=128, N=64 tokens) and O += P V
+// (M=128, N=D) are each a few tcgen05.mma issued by one thread, accumulating in
+// tensor memory (S: 64 columns, O: D columns). Warps 0-3 own one row per
+// thread: they read the row of S from tensor memory, run the online softmax
+// (all in the thread: no shuffles) and write the row of P to shared memory.
+// O is rescaled lazily: only when a row's maximum grows by more than 2^8,
+// which keeps P <= 256; the final division by the row sum makes the result
+// the same as with a rescale at every step.
+// Warp 4 issues the TMA tile loads, warp 5 allocates tensor memory and issues
+// the MMAs. Shared memory, 1024-byte aligned: Q [D/64][128 rows][128 B],
+// K/V stages [K tiles D/64][64 tokens][128 B] then V likewise, P [128][128 B],
+// all 128B-swizzled (the MMA descriptors say so).
+// ===========================================================================
+namespace tc {
+
+constexpr int kRows = 128;
+constexpr int kThreads = 192;
+constexpr int kStages = 2;
+constexpr int kTok = 64;               // KV tokens per tile (4 blocks)
+constexpr float kRescaleLog2 = 8.f;    // rescale O when a row maximum grows by more than 2^8
+
+template <int D>
+struct TGeo {
+    static constexpr int kTiles = D / 64;
+    static constexpr int kQBytes = kTiles * kRows * 128;
+    static constexpr int kKVTileBytes = kTok * 128;              // one 64-column tile of 64 tokens
+    static constexpr int kStageBytes = 2 * kTiles * kKVTileBytes;
+    static constexpr int kPBytes = kRows * 128;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffKV = kOffQ + kQBytes;
+    static constexpr int kOffP = kOffKV + kStages * kStageBytes;
+    static constexpr int kOffBar = kOffP + kPBytes;
+    static constexpr int kSmemBytes = kOffBar + 128 + 1024;
+    static constexpr int kTmemCols = D == 128 ? 256 : 128;     // S at column 0, O at kOCol
+    static constexpr int kOCol = D == 128 ? 128 : 64;
+};
+
+template <class E, int D>
+__global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                              const __grid_constant__ CUtensorMap tmV,
+                                                              const PrefillArgs a)
+{
+    using G = TGeo<D>;
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
+    unsigned char *base = smem_raw + (base_s - raw_s);
+    const uint32_t sQ = base_s + G::kOffQ, sKV = base_s + G::kOffKV, sP = base_s + G::kOffP;
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + G::kOffBar);
+    uint64_t *empty = full + kStages;
+    uint64_t *s_full = empty + kStages;
+    uint64_t *p_full = s_full + 1;
+    uint64_t *pv_done = p_full + 1;
+    uint64_t *q_ready = pv_done + 1;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_ready + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *zero_flag = abort_flag + 1;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int b = blockIdx.z, j = blockIdx.y;
+    const int tile = a.max_tiles - 1 - static_cast<int>(blockIdx.x);
+    const int g = a.group;
+    const int q0 = __ldg(a.query_start + b);
+    const int n = __ldg(a.query_start + b + 1) - q0;
+    const int c = __ldg(a.context_lens + b);
+    if (n <= 0)
+        return;
+    if (n > c || c > a.W * kBlockTokens || n > a.max_query_len) {
+        if (tid == 0 && j == 0 && tile == a.max_tiles - 1)
+            flag(a, KV_STATUS_BAD_CONTEXT);
+        return;
+    }
+    const int rows_total = n * g;
+    const int row0 = tile * kRows;
+    if (row0 >= rows_total)
+        return;
+    const int p0 = c - n;
+    const int last_row = min(row0 + kRows, rows_total) - 1;
+    const int kv_len = p0 + last_row / g + 1;
+    const int nblk = (kv_len + kBlockTokens - 1) / kBlockTokens;
+    const int ntiles = (kv_len + kTok - 1) / kTok;
+    constexpr int fmt = E::kDtype == KV_DTYPE_BF16 ? 1 : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(p_full, kRows);
+        mbar_init(pv_done, 1);
+        mbar_init(q_ready, kRows);
+        mbar_fence_init();
+        *abort_flag = 0;
+        *zero_flag = 0;
+    }
+    if (warp == 5)
+        tmem_alloc(tmem_slot, G::kTmemCols);
+    tcgen05_before_sync();
+    __syncthreads();
+    tcgen05_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ---------------- producer: block ids -> TMA loads ----------------
+        if (lane == 0) {
+            tma_prefetch_descriptor(&tmK);
+            tma_prefetch_descriptor(&tmV);
+        }
+        grid_dependency_wait();
+        grid_launch_dependents();
+        const int32_t *trow = a.block_tables + static_cast<size_t>(b) * a.W;
+        int issued = 0;
+        for (int jt = 0; jt < ntiles; ++jt) {
+            const int s = jt % kStages;
+            const int kb0 = jt * (kTok / kBlockTokens);
+            const int nb = min(kTok / kBlockTokens, nblk - kb0);
+            int blk = 0;
+            if (lane < nb) {
+                blk = __ldg(trow + kb0 + lane);
+                if (blk < 0 || blk >= a.num_blocks) {
+                    flag(a, KV_STATUS_BAD_BLOCK_ID);
+                    blk = 0;
+                }
+            }
+            int ok = 1;
+            if (lane == 0) {
+                ok = mbar_wait_bounded(&empty[s], ((jt / kStages) & 1) ^ 1, abort_flag);
+                if (ok)
+                    mbar_arrive_expect_tx(&full[s], nb * 2 * G::kTiles * 2048);
+                else {
+                    *abort_flag = 1;
+                    flag(a, KV_STATUS_WAIT_TIMEOUT);
+                }
+            }
+            ok = __shfl_sync(kFullMask, ok, 0);
+            if (!ok)
+                break;
+            __syncwarp();
+            if (lane < nb) {
+                const uint32_t kdst = sKV + s * G::kStageBytes + lane * 2048;
+                const uint32_t vdst = kdst + G::kTiles * G::kKVTileBytes;
+#pragma unroll
+                for (int t = 0; t < G::kTiles; ++t)
+                    tma_load_4d_nohint(kdst + t * G::kKVTileBytes, &tmK, t * 64, 0, j, blk, &full[s]);
+#pragma unroll
+                for (int t = 0; t < G::kTiles; ++t)
+                    tma_load_4d_nohint(vdst + t * G::kKVTileBytes, &tmV, t * 64, 0, j, blk, &full[s]);
+            }
+            issued = jt + 1;
+        }
+        if (lane == 0)
+            for (int jt = max(0, issued - kStages); jt < issued; ++jt)
+                mbar_wait_bounded(&full[jt % kStages], (jt / kStages) & 1, zero_flag);
+    } else if (warp == 5) {
+        // ---------------- MMA issuer (one thread) ----------------
+        grid_dependency_wait();
+        grid_launch_dependents();
+        if (lane == 0) {
+            const uint32_t idesc_s = umma_idesc_f16(kRows, kTok, fmt, 0, 0);
+            const uint32_t idesc_o = umma_idesc_f16(kRows, D, fmt, 0, 1);
+            bool ok = mbar_wait_bounded(q_ready, 0, abort_flag);
+            tcgen05_after_sync();
+            int done = 0;  // tiles whose PV was issued
+            for (int jt = 0; jt < ntiles && ok; ++jt) {
+                const int s = jt % kStages;
+                const uint32_t kst = sKV + s * G::kStageBytes;
+                const uint32_t vst = kst + G::kTiles * G::kKVTileBytes;
+                if (!mbar_wait_bounded(&full[s], (jt / kStages) & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tcgen05_after_sync();
+                // S = Q K^T
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32;  // 16 elements along the 128-byte row
+                    const uint64_t ad = umma_desc_sw128(sQ + (kk >> 2) * (kRows * 128) + koff, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(kst + (kk >> 2) * G::kKVTileBytes + koff, 16, 1024);
+                    umma_f16(tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(s_full);
+                if (!mbar_wait_bounded(p_full, jt & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tcgen05_after_sync();
+                // O += P V
+#pragma unroll
+                for (int kk = 0; kk < kTok / 16; ++kk) {
+                    const uint64_t ad = umma_desc_sw128(sP + kk * 32, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(vst + kk * 2048, G::kKVTileBytes, 1024);
+                    umma_f16(tmem + G::kOCol, ad, bd, idesc_o, (jt > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(pv_done);
+                umma_commit(&empty[s]);
+                done = jt + 1;
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                flag(a, KV_STATUS_WAIT_TIMEOUT);
+            }
+            // the MMAs in flight finish before tensor memory is released (below)
+            if (done > 0)
+                mbar_wait_bounded(pv_done, (done - 1) & 1, zero_flag);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- softmax: one query row per thread ----------------
+        grid_dependency_wait();  // q may come from the kernel before
+        grid_launch_dependents();
+        const int r = tid;  // 0..127: TMEM lane and row of the tile
+        const int row = row0 + r;
+        const bool ok = row < rows_total;
+        const int rowc = min(row, rows_total - 1);
+        const int tok = rowc / g, h = rowc - tok * g;
+        const int pos = p0 + tok;
+        {
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D);
+#pragma unroll
+            for (int ch = 0; ch < D / 8; ++ch) {
+                const uint4 v = ok ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t dst = sQ + (ch >> 3) * (kRows * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
+                             "r"(v.w)
+                             : "memory");
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(q_ready);
+        }
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const float sl2 = a.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
+        bool good = true;
+        for (int jt = 0; jt < ntiles; ++jt) {
+            // tcgen05.ld/st are warp-wide: a warp takes every branch below as one
+            if (!__all_sync(kFullMask, mbar_wait_bounded(s_full, jt & 1, abort_flag))) {
+                good = false;
+                break;
+            }
+            tcgen05_after_sync();
+            float x[kTok];
+            {
+                uint32_t v[16];
+#pragma unroll
+                for (int q4 = 0; q4 < kTok / 16; ++q4) {
+                    tmem_ld16(lane_base + q4 * 16, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        x[q4 * 16 + i] = __uint_as_float(v[i]);
+                }
+            }
+            const int tok0 = jt * kTok;
+            float xmax = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kTok; ++i) {
+                x[i] = (tok0 + i <= pos) ? x[i] * sl2 : -INFINITY;
+                xmax = fmaxf(xmax, x[i]);
+            }
+            bool rescale = false;
+            float alpha = 1.f;
+            if (xmax > m_used + kRescaleLog2) {  // always true on the first tile (m_used = -inf)
+                alpha = exp2f(m_used - xmax);
+                rescale = jt > 0;
+                m_used = xmax;
+                l *= alpha;
+            }
+            if (jt > 0) {
+                // PV of the previous tile is done: P may be rewritten and O rescaled
+                if (!__all_sync(kFullMask, mbar_wait_bounded(pv_done, (jt - 1) & 1, abort_flag))) {
+                    good = false;
+                    break;
+                }
+                tcgen05_after_sync();
+            }
+            if (!rescale)
+                alpha = 1.f;  // lanes that keep their scale rewrite their row unchanged
+            if (__any_sync(kFullMask, rescale)) {
+                uint32_t v[16];
+#pragma unroll 1
+                for (int q4 = 0; q4 < D / 16; ++q4) {
+                    tmem_ld16(lane_base + G::kOCol + q4 * 16, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                    tmem_st16(lane_base + G::kOCol + q4 * 16, v);
+                }
+                tmem_wait_st();
+            }
+            float psum = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < kTok / 8; ++ch) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float pa = exp2f(x[ch * 8 + 2 * e] - m_used), pb = exp2f(x[ch * 8 + 2 * e + 1] - m_used);
+                    psum += pa + pb;
+                    w[e] = E::pack(pa, pb);
+                }
+                const uint32_t dst = sP + r * 128 + ((ch ^ (r & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                             "r"(w[3])
+                             : "memory");
+            }
+            l += psum;
+            // tokens of this tile at or past the context hold whatever the stage holds: zero those V rows
+            const int vrow0 = c - tok0;
+            if (vrow0 < kTok) {
+                const uint32_t vst = sKV + (jt % kStages) * G::kStageBytes + G::kTiles * G::kKVTileBytes;
+                const int cnt = (kTok - vrow0) * G::kTiles * 8;
+                for (int idx = r; idx < cnt; idx += kRows) {
+                    const int rr = vrow0 + idx / (G::kTiles * 8);
+                    const int rem = idx % (G::kTiles * 8);
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(vst + (rem >> 3) * G::kKVTileBytes +
+                                                                               rr * 128 + ((rem & 7) << 4)),
+                                 "r"(0)
+                                 : "memory");
+                }
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tcgen05_before_sync();
+            mbar_arrive(p_full);
+        }
+        // epilogue: O / l
+        if (__all_sync(kFullMask, good && mbar_wait_bounded(pv_done, (ntiles - 1) & 1, abort_flag))) {
+            tcgen05_after_sync();
+            const float inv = 1.f / l;
+            uint16_t *dst = a.out + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D;
+            uint32_t v[16];
+#pragma unroll 1
+            for (int q4 = 0; q4 < D / 16; ++q4) {
+                tmem_ld16(lane_base + G::kOCol + q4 * 16, v);
+                tmem_wait_ld();
+                uint4 o0, o1;
+                o0.x = E::pack(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
+                o0.y = E::pack(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv);
+                o0.z = E::pack(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv);
+                o0.w = E::pack(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv);
+                o1.x = E::pack(__uint_as_float(v[8]) * inv, __uint_as_float(v[9]) * inv);
+                o1.y = E::pack(__uint_as_float(v[10]) * inv, __uint_as_float(v[11]) * inv);
+                o1.z = E::pack(__uint_as_float(v[12]) * inv, __uint_as_float(v[13]) * inv);
+                o1.w = E::pack(__uint_as_float(v[14]) * inv, __uint_as_float(v[15]) * inv);
+                if (ok) {
+                    reinterpret_cast<uint4 *>(dst + q4 * 16)[0] = o0;
+                    reinterpret_cast<uint4 *>(dst + q4 * 16)[1] = o1;
+                }
+            }
+        } else if (lane == 0) {
+            *abort_flag = 1;
+            flag(a, KV_STATUS_WAIT_TIMEOUT);
+        }
+    }
+    // every thread is past its last tensor-memory access; release it
+    tcgen05_before_sync();
+    __syncthreads();
+    if (warp == 5) {
+        tcgen05_after_sync();
+        tmem_dealloc(tmem, G::kTmemCols);
+    }
+}
+
+}  // namespace tc
 }  // namespace prefill
 }  // namespace pkv
+
+// KV_OPT_PREFILL_PATH, kept with the other switches in decode.cu
+int pkv_prefill_path();
 
 namespace {
 
 using PrefillFn = void (*)(const CUtensorMap, const CUtensorMap, const pkv::prefill::PrefillArgs);
+
+PrefillFn pick_prefill_tc(int dtype, int D, int *smem)
+{
+    using namespace pkv;
+    using namespace pkv::prefill::tc;
+    *smem = D == 64 ? TGeo<64>::kSmemBytes : TGeo<128>::kSmemBytes;
+    if (dtype == KV_DTYPE_FP16)
+        return D == 64 ? prefill_tc_kernel<ElemF16, 64> : prefill_tc_kernel<ElemF16, 128>;
+    return D == 64 ? prefill_tc_kernel<ElemBf16, 64> : prefill_tc_kernel<ElemBf16, 128>;
+}
 
 PrefillFn pick_prefill(int dtype, int D, int *smem)
 {
@@ -423,14 +802,16 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
     if (misaligned16(out) || misaligned16(q) || misaligned16(k_cache) || misaligned16(v_cache))
         return KV_ERR_ARG;
     const int group = Hq / Hkv;
-    const long long tiles = (static_cast<long long>(max_query_len) * group + kRows - 1) / kRows;
+    const bool use_tc = pkv_prefill_path() != 2;  // tcgen05 unless the mma.sync path is asked for
+    const int rows_per_cta = use_tc ? tc::kRows : kRows;
+    const long long tiles = (static_cast<long long>(max_query_len) * group + rows_per_cta - 1) / rows_per_cta;
     if (tiles > (1ll << 31) - 1)
         return KV_ERR_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return KV_ERR_CUDA;
     int smem = 0;
-    PrefillFn fn = pick_prefill(dtype, D, &smem);
+    PrefillFn fn = use_tc ? pick_prefill_tc(dtype, D, &smem) : pick_prefill(dtype, D, &smem);
     if (!prepare_prefill(fn, smem, dev))
         return KV_ERR_CUDA;
     CUtensorMap tmK, tmV;
@@ -456,7 +837,7 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(use_tc ? tc::kThreads : kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];

@@ -12,6 +12,14 @@ from gpu_cases import compare
 
 pytestmark = pytest.mark.gpu
 
+PREFILL_PATHS = {"tcgen05": 1, "mma_sync": 2}
+
+
+@pytest.fixture(autouse=True)
+def _default_path(pkv):
+    yield
+    pkv.set_option(pkv.KV_OPT_PREFILL_PATH, 0)
+
 
 def bits(t: torch.Tensor) -> np.ndarray:
     return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
@@ -61,16 +69,18 @@ def run_case(pkv, oracle_mod, case, what, rows=None):
     return out
 
 
+@pytest.mark.parametrize("path", sorted(PREFILL_PATHS))
 @pytest.mark.parametrize("elem", ["bf16", "fp16"])
 @pytest.mark.parametrize("Hq,Hkv,D", [(20, 4, 64), (32, 8, 128), (8, 8, 128), (12, 1, 64), (16, 2, 128), (6, 6, 64)])
-def test_prefill_chunks(pkv, oracle_mod, cuda_device, Hq, Hkv, D, elem):
+def test_prefill_chunks(pkv, oracle_mod, cuda_device, Hq, Hkv, D, elem, path):
     """Whole prompts, chunks over a cached prefix, single tokens and empty chunks; lengths at and
     around block edges."""
+    pkv.set_option(pkv.KV_OPT_PREFILL_PATH, PREFILL_PATHS[path])
     chunk = [37, 1, 16, 100, 0, 64, 17, 5]
     prior = [0, 250, 15, 33, 40, 0, 111, 1]
     cfg = workloads.PrefillConfig("test", Hq, Hkv, D, len(chunk), 0, 0, 0, 16, seed=Hq * 7 + D, elem=elem)
     case = PrefillCase(cfg, cuda_device, chunk_lens=chunk, prior_lens=prior)
-    run_case(pkv, oracle_mod, case, f"prefill {Hq}/{Hkv} D{D} {elem}")
+    run_case(pkv, oracle_mod, case, f"prefill {Hq}/{Hkv} D{D} {elem} {path}")
 
 
 def test_single_token_chunk_matches_the_decode(pkv, cuda_device):
@@ -88,14 +98,18 @@ def test_single_token_chunk_matches_the_decode(pkv, cuda_device):
     assert float(d.max()) <= 2e-2, float(d.max())
 
 
-def test_full_size_prefill_workload(pkv, oracle_mod, cuda_device):
+@pytest.mark.parametrize("path", sorted(PREFILL_PATHS))
+def test_full_size_prefill_workload(pkv, oracle_mod, cuda_device, path):
     """The bench's prefill workload (LLaMA-3-8B shape), three of its sequences against the oracle."""
+    pkv.set_option(pkv.KV_OPT_PREFILL_PATH, PREFILL_PATHS[path])
     cfg = workloads.PREFILL_CONFIGS["llama3_8b"]
     case = PrefillCase(cfg, cuda_device)
-    run_case(pkv, oracle_mod, case, "full-size prefill", rows=[0, 7, 15])
+    run_case(pkv, oracle_mod, case, f"full-size prefill {path}", rows=[0, 7, 15])
 
 
-def test_bad_chunks_are_flagged(pkv, cuda_device):
+@pytest.mark.parametrize("path", sorted(PREFILL_PATHS))
+def test_bad_chunks_are_flagged(pkv, cuda_device, path):
+    pkv.set_option(pkv.KV_OPT_PREFILL_PATH, PREFILL_PATHS[path])
     cfg = workloads.PrefillConfig("test", 8, 2, 64, 3, 10, 20, 40, 8, seed=5)
     case = PrefillCase(cfg, cuda_device)
     out = torch.zeros_like(case.q)
