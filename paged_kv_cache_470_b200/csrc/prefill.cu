@@ -398,7 +398,9 @@ struct TGeo {
     static constexpr int kOffKV = kOffQ + kQBytes;
     static constexpr int kOffP = kOffKV + kStages * kStageBytes;
     static constexpr int kOffBar = kOffP + kPBytes;
-    static constexpr int kSmemBytes = kOffBar + 128 + 1024;
+    // no slack for aligning the base: the buffer is declared 1024-byte aligned (checked at run time),
+    // which lets two CTAs share an SM at D = 128
+    static constexpr int kSmemBytes = kOffBar + 128;
     static constexpr int kTmemCols = D == 128 ? 256 : 128;     // S at column 0, O at kOCol
     static constexpr int kOCol = D == 128 ? 128 : 64;
 };
@@ -409,10 +411,14 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                                                               const PrefillArgs a)
 {
     using G = TGeo<D>;
-    extern __shared__ unsigned char smem_raw[];
-    const uint32_t raw_s = smem_addr(smem_raw);
-    const uint32_t base_s = (raw_s + 1023u) & ~1023u;
-    unsigned char *base = smem_raw + (base_s - raw_s);
+    extern __shared__ __align__(1024) unsigned char smem_tc[];
+    const uint32_t base_s = smem_addr(smem_tc);
+    unsigned char *base = smem_tc;
+    if (base_s & 1023u) {  // the swizzle atoms need 1024-byte alignment
+        if (threadIdx.x == 0)
+            flag(a, KV_STATUS_BAD_CONTEXT);
+        return;
+    }
     const uint32_t sQ = base_s + G::kOffQ, sKV = base_s + G::kOffKV, sP = base_s + G::kOffP;
     uint64_t *full = reinterpret_cast<uint64_t *>(base + G::kOffBar);
     uint64_t *empty = full + kStages;
