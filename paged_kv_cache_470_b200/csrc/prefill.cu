@@ -368,16 +368,18 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
 // tcgen05 path. The same computation on the 5th-generation tensor cores: a CTA
 // takes 128 query rows; S = Q K^T (M=128, N=64 tokens) and O += P V
 // (M=128, N=D) are each a few tcgen05.mma issued by one thread, accumulating in
-// tensor memory (S: 64 columns, O: D columns). Warps 0-3 own one row per
-// thread: they read the row of S from tensor memory, run the online softmax
-// (all in the thread: no shuffles) and write the row of P to shared memory.
-// O is rescaled lazily: only when a row's maximum grows by more than 2^8,
-// which keeps P <= 256; the final division by the row sum makes the result
-// the same as with a rescale at every step.
-// Warp 4 issues the TMA tile loads, warp 5 allocates tensor memory and issues
-// the MMAs. Shared memory, 1024-byte aligned: Q [D/64][128 rows][128 B],
-// K/V stages [K tiles D/64][64 tokens][128 B] then V likewise, P [128][128 B],
-// all 128B-swizzled (the MMA descriptors say so).
+// tensor memory. S is double-buffered (columns 0-63 and 64-127): the MMAs of
+// the next tile's S run while warps 0-3 turn this tile's S into P. Those warps
+// own one row per thread: they read the row of S from tensor memory, run the
+// online softmax (all in the thread: no shuffles) and write the row of P, as
+// 16-bit pairs, over the first half of the same S buffer, where the P V MMA
+// takes its A operand from. O (columns 128..) is rescaled lazily: only when a
+// row's maximum grows by more than 2^8, which keeps P <= 256; the final
+// division by the row sum makes the result the same as with a rescale at every
+// step. Warp 4 issues the TMA tile loads, warp 5 allocates tensor memory and
+// issues the MMAs. Shared memory, 1024-byte aligned: Q [D/64][128 rows][128 B],
+// then K/V stages [K tiles D/64][64 tokens][128 B] and V likewise, all
+// 128B-swizzled (the MMA descriptors say so).
 // ===========================================================================
 namespace tc {
 
@@ -393,16 +395,16 @@ struct TGeo {
     static constexpr int kQBytes = kTiles * kRows * 128;
     static constexpr int kKVTileBytes = kTok * 128;              // one 64-column tile of 64 tokens
     static constexpr int kStageBytes = 2 * kTiles * kKVTileBytes;
-    static constexpr int kPBytes = kRows * 128;
     static constexpr int kOffQ = 0;
     static constexpr int kOffKV = kOffQ + kQBytes;
-    static constexpr int kOffP = kOffKV + kStages * kStageBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
+    static constexpr int kOffBar = kOffKV + kStages * kStageBytes;
     // no slack for aligning the base: the buffer is declared 1024-byte aligned (checked at run time),
     // which lets two CTAs share an SM at D = 128
-    static constexpr int kSmemBytes = kOffBar + 128;
-    static constexpr int kTmemCols = D == 128 ? 256 : 128;     // S at column 0, O at kOCol
-    static constexpr int kOCol = D == 128 ? 128 : 64;
+    // at most two CTAs per SM: two of them use all 512 tensor-memory columns (an allocation beyond
+    // that would wait for a CTA to finish), so D = 64 asks for more shared memory than it uses
+    static constexpr int kSmemBytes = kOffBar + 128 < 80 * 1024 ? 80 * 1024 : kOffBar + 128;
+    static constexpr int kTmemCols = 256;                       // S/P buffers at 0 and 64, O at kOCol
+    static constexpr int kOCol = 128;
 };
 
 template <class E, int D>
@@ -419,11 +421,11 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             flag(a, KV_STATUS_BAD_CONTEXT);
         return;
     }
-    const uint32_t sQ = base_s + G::kOffQ, sKV = base_s + G::kOffKV, sP = base_s + G::kOffP;
+    const uint32_t sQ = base_s + G::kOffQ, sKV = base_s + G::kOffKV;
     uint64_t *full = reinterpret_cast<uint64_t *>(base + G::kOffBar);
     uint64_t *empty = full + kStages;
-    uint64_t *s_full = empty + kStages;
-    uint64_t *p_full = s_full + 1;
+    uint64_t *s_full = empty + kStages;  // [2]: one per S buffer
+    uint64_t *p_full = s_full + 2;
     uint64_t *pv_done = p_full + 1;
     uint64_t *q_ready = pv_done + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_ready + 1);
@@ -460,7 +462,8 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(s_full, 1);
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
         mbar_init(p_full, kRows);
         mbar_init(pv_done, 1);
         mbar_init(q_ready, kRows);
@@ -535,36 +538,51 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             const uint32_t idesc_o = umma_idesc_f16(kRows, D, fmt, 0, 1);
             bool ok = mbar_wait_bounded(q_ready, 0, abort_flag);
             tcgen05_after_sync();
-            int done = 0;  // tiles whose PV was issued
-            for (int jt = 0; jt < ntiles && ok; ++jt) {
+            // S = Q K^T for tile jt into S buffer jt & 1
+            auto issue_s = [&](int jt) -> bool {
                 const int s = jt % kStages;
-                const uint32_t kst = sKV + s * G::kStageBytes;
-                const uint32_t vst = kst + G::kTiles * G::kKVTileBytes;
-                if (!mbar_wait_bounded(&full[s], (jt / kStages) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+                if (!mbar_wait_bounded(&full[s], (jt / kStages) & 1, abort_flag))
+                    return false;
                 tcgen05_after_sync();
-                // S = Q K^T
+                const uint32_t kst = sKV + s * G::kStageBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk & 3) * 32;  // 16 elements along the 128-byte row
                     const uint64_t ad = umma_desc_sw128(sQ + (kk >> 2) * (kRows * 128) + koff, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(kst + (kk >> 2) * G::kKVTileBytes + koff, 16, 1024);
-                    umma_f16(tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    umma_f16(tmem + (jt & 1) * kTok, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(s_full);
+                umma_commit(&s_full[jt & 1]);
+                return true;
+            };
+            int done = 0;  // tiles whose PV was issued
+            if (ok && ntiles > 0)
+                ok = issue_s(0);
+            for (int jt = 0; jt < ntiles && ok; ++jt) {
+                const int s = jt % kStages;
+                const uint32_t vst = sKV + s * G::kStageBytes + G::kTiles * G::kKVTileBytes;
+                if (jt + 1 < ntiles) {
+                    // the next S goes into the buffer that P of tile jt-1 used: wait for that PV
+                    if (jt >= 1 && !mbar_wait_bounded(pv_done, (jt - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!issue_s(jt + 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
                 if (!mbar_wait_bounded(p_full, jt & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tcgen05_after_sync();
-                // O += P V
+                // O += P V, P (16-bit pairs) in the first 32 columns of S buffer jt & 1
 #pragma unroll
                 for (int kk = 0; kk < kTok / 16; ++kk) {
-                    const uint64_t ad = umma_desc_sw128(sP + kk * 32, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(vst + kk * 2048, G::kKVTileBytes, 1024);
-                    umma_f16(tmem + G::kOCol, ad, bd, idesc_o, (jt > 0 || kk > 0) ? 1u : 0u);
+                    umma_f16_tmem_a(tmem + G::kOCol, tmem + (jt & 1) * kTok + kk * 8, bd, idesc_o,
+                                    (jt > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(pv_done);
                 umma_commit(&empty[s]);
@@ -608,17 +626,18 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
         bool good = true;
         for (int jt = 0; jt < ntiles; ++jt) {
             // tcgen05.ld/st are warp-wide: a warp takes every branch below as one
-            if (!__all_sync(kFullMask, mbar_wait_bounded(s_full, jt & 1, abort_flag))) {
+            if (!__all_sync(kFullMask, mbar_wait_bounded(&s_full[jt & 1], (jt >> 1) & 1, abort_flag))) {
                 good = false;
                 break;
             }
             tcgen05_after_sync();
+            const uint32_t sbuf = lane_base + (jt & 1) * kTok;
             float x[kTok];
             {
                 uint32_t v[16];
 #pragma unroll
                 for (int q4 = 0; q4 < kTok / 16; ++q4) {
-                    tmem_ld16(lane_base + q4 * 16, v);
+                    tmem_ld16(sbuf + q4 * 16, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
@@ -640,17 +659,15 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 m_used = xmax;
                 l *= alpha;
             }
-            if (jt > 0) {
-                // PV of the previous tile is done: P may be rewritten and O rescaled
+            if (!rescale)
+                alpha = 1.f;  // lanes that keep their scale rewrite their row unchanged
+            if (__any_sync(kFullMask, rescale)) {
+                // O is rescaled once the previous tile's PV has finished with it
                 if (!__all_sync(kFullMask, mbar_wait_bounded(pv_done, (jt - 1) & 1, abort_flag))) {
                     good = false;
                     break;
                 }
                 tcgen05_after_sync();
-            }
-            if (!rescale)
-                alpha = 1.f;  // lanes that keep their scale rewrite their row unchanged
-            if (__any_sync(kFullMask, rescale)) {
                 uint32_t v[16];
 #pragma unroll 1
                 for (int q4 = 0; q4 < D / 16; ++q4) {
@@ -665,19 +682,17 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             }
             float psum = 0.f;
 #pragma unroll
-            for (int ch = 0; ch < kTok / 8; ++ch) {
-                uint32_t w[4];
+            for (int half = 0; half < 2; ++half) {
+                uint32_t w[16];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float pa = exp2f(x[ch * 8 + 2 * e] - m_used), pb = exp2f(x[ch * 8 + 2 * e + 1] - m_used);
+                for (int e = 0; e < 16; ++e) {
+                    const float pa = exp2f(x[half * 32 + 2 * e] - m_used), pb = exp2f(x[half * 32 + 2 * e + 1] - m_used);
                     psum += pa + pb;
                     w[e] = E::pack(pa, pb);
                 }
-                const uint32_t dst = sP + r * 128 + ((ch ^ (r & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(w[0]), "r"(w[1]), "r"(w[2]),
-                             "r"(w[3])
-                             : "memory");
+                tmem_st16(sbuf + half * 16, w);
             }
+            tmem_wait_st();
             l += psum;
             // tokens of this tile at or past the context hold whatever the stage holds: zero those V rows
             const int vrow0 = c - tok0;
