@@ -238,7 +238,7 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
  * OR-ed into *error_flag (device int32, may be NULL): KV_STATUS_BAD_CONTEXT
  * when n_b > c_b, c_b > 16 * max_blocks_per_seq or n_b > max_query_len (that
  * sequence's rows are not written), KV_STATUS_BAD_BLOCK_ID for ids outside the
- * pool (block 0 is read instead). B <= 65535, Hkv <= 65535.
+ * pool (block 0 is read instead). B <= 65535, Hkv <= 65535, scale > 0.
  */
 KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,

@@ -389,6 +389,15 @@ constexpr int kStages = 2;
 constexpr int kTok = 64;               // KV tokens per tile (4 blocks)
 constexpr float kRescaleLog2 = 8.f;    // rescale O when a row maximum grows by more than 2^8
 
+// 2^x by the special-function unit's approximate base-2 exponential (results
+// below 2^-126, and 2^-inf, are 0).
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <int D>
 struct TGeo {
     static constexpr int kTiles = D / 64;
@@ -645,16 +654,22 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 }
             }
             const int tok0 = jt * kTok;
-            float xmax = -INFINITY;
+            // raw scores: tokens after this row's position are -inf (scale > 0, so the maximum of
+            // the raw scores scales to the maximum of the scaled ones)
+            if (tok0 + kTok - 1 > pos) {
 #pragma unroll
-            for (int i = 0; i < kTok; ++i) {
-                x[i] = (tok0 + i <= pos) ? x[i] * sl2 : -INFINITY;
-                xmax = fmaxf(xmax, x[i]);
+                for (int i = 0; i < kTok; ++i)
+                    x[i] = (tok0 + i <= pos) ? x[i] : -INFINITY;
             }
+            float rmax = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kTok; ++i)
+                rmax = fmaxf(rmax, x[i]);
+            const float xmax = rmax * sl2;
             bool rescale = false;
             float alpha = 1.f;
             if (xmax > m_used + kRescaleLog2) {  // always true on the first tile (m_used = -inf)
-                alpha = exp2f(m_used - xmax);
+                alpha = ex2_approx(m_used - xmax);
                 rescale = jt > 0;
                 m_used = xmax;
                 l *= alpha;
@@ -686,7 +701,8 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float pa = exp2f(x[half * 32 + 2 * e] - m_used), pb = exp2f(x[half * 32 + 2 * e + 1] - m_used);
+                    const float pa = ex2_approx(fmaf(x[half * 32 + 2 * e], sl2, -m_used));
+                    const float pb = ex2_approx(fmaf(x[half * 32 + 2 * e + 1], sl2, -m_used));
                     psum += pa + pb;
                     w[e] = E::pack(pa, pb);
                 }
@@ -823,6 +839,8 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
     if (misaligned16(out) || misaligned16(q) || misaligned16(k_cache) || misaligned16(v_cache))
         return KV_ERR_ARG;
     const int group = Hq / Hkv;
+    if (!(scale > 0.f))
+        return KV_ERR_ARG;
     const bool use_tc = pkv_prefill_path() != 2;  // tcgen05 unless the mma.sync path is asked for
     const int rows_per_cta = use_tc ? tc::kRows : kRows;
     const long long tiles = (static_cast<long long>(max_query_len) * group + rows_per_cta - 1) / rows_per_cta;
