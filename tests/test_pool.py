@@ -293,3 +293,28 @@ def test_copy_on_write_errors_leave_state_unchanged(pkv):
     with pytest.raises(pkv.KVError) as e:
         p.append_slots_cow(bad, lens[:1].clone(), slots[:1].clone())
     assert e.value.status == pkv.KV_ERR_STATE and p.num_free() == 1
+
+
+# ---------------------------------------------------------------------------
+# chunked-prefill layouts (host side of the prefill workloads)
+# ---------------------------------------------------------------------------
+def test_prefill_layout_places_each_chunk_at_the_end_of_its_context(oracle_mod):
+    from paged_kv_cache_470_b200 import workloads
+    cfg = workloads.PrefillConfig("t", 8, 2, 64, 5, 0, 0, 0, 16)
+    chunk, prior = [37, 1, 16, 0, 40], [0, 250, 15, 33, 7]
+    lay = workloads.draw_prefill_layout(cfg, chunk_lens=chunk, prior_lens=prior, seed=9)
+    assert lay.context_lens.tolist() == [c + p for c, p in zip(chunk, prior)]
+    assert lay.query_start.tolist() == [0, 37, 38, 54, 54, 94]
+    slots = lay.slot_mapping().tolist()
+    assert len(slots) == sum(chunk) and len(set(slots)) == len(slots)
+    k = 0
+    for b in range(5):
+        c = int(lay.context_lens[b])
+        nblk = oracle_mod.blocks_needed(c)
+        row = lay.block_tables[b]
+        assert (row[:nblk] >= 0).all() and (row[nblk:] == -1).all()
+        for pos in range(c - chunk[b], c):      # the chunk is the last chunk[b] positions
+            assert slots[k] == int(row[pos // 16]) * 16 + pos % 16
+            k += 1
+    used = [int(x) for x in lay.block_tables.flatten().tolist() if x >= 0]
+    assert len(set(used)) == len(used) and max(used) < lay.num_blocks
