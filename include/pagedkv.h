@@ -268,6 +268,13 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     0 auto, -1 none, 1..64 that many.
  *   KV_OPT_PREFILL_PATH: paged_attention_prefill on 0 auto (tcgen05), 1
  *                     tcgen05.mma with tensor-memory accumulators, 2 mma.sync.
+ *   KV_OPT_TEST_DROP_LOAD: test hook for the timeout path, 0 (default) off;
+ *                     n > 0: in the decode kernels' CTA 0 the tile load of
+ *                     work unit n - 1 is never issued, so the wait for it runs
+ *                     out (after about a second): the call completes with
+ *                     KV_STATUS_WAIT_TIMEOUT in the status word and its output
+ *                     is not valid; the context stays usable (re-initialise
+ *                     the workspace, as after any timed-out call).
  * Kernels are launched with programmatic dependent launch. q, k_new, v_new,
  * the caches, the workspace and out are touched only after the previous kernel
  * in the stream has completed; block_tables and context_lens are read before
@@ -282,6 +289,7 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
 #define KV_OPT_HEAD_GROUP 6
 #define KV_OPT_ITEM_COST 7
 #define KV_OPT_PREFILL_PATH 8
+#define KV_OPT_TEST_DROP_LOAD 9
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

@@ -114,6 +114,7 @@ struct DecodeArgs {
     int prod_lanes;      // producer lanes issuing TMA
     int min_chunk;
     int item_cost;       // work positions charged per work item on top of its units
+    int drop_unit;       // test hook: CTA 0 never loads its unit with this index (-1: none)
     int fused;
     float scale_log2;    // scale * log2(e)
     // fused append (append != 0): this step's token of sequence b is k_new/v_new[b],
@@ -1011,7 +1012,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         const int uu = u + bi + i;
                         const int s = uu % S;
                         ok = mbar_wait_bounded(&empty[s], ((uu / S) & 1) ^ 1, abort_flag);
-                        if (ok) {
+                        if (ok && uu == a.drop_unit && blockIdx.x == 0) {
+                            // test hook: this stage is never filled, so its consumers' wait runs out
+                        } else if (ok) {
                             mbar_arrive_expect_tx(&full[s], a.stage_bytes);
                             const uint32_t dst = ring + s * a.stage_bytes;
 #pragma unroll
@@ -1327,6 +1330,7 @@ std::atomic<int> g_opt_prod_lanes{0};
 std::atomic<int> g_opt_head_group{0};
 std::atomic<int> g_opt_item_cost{0};
 std::atomic<int> g_opt_prefill_path{0};
+std::atomic<int> g_opt_drop_load{0};
 constexpr int kDefaultMinChunk = 4;
 
 // Work positions charged per work item (its fixed cost, in units of one work
@@ -1577,6 +1581,7 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     const int mc = g_opt_min_chunk.load();
     a.min_chunk = mc > 0 ? mc : kDefaultMinChunk;
     a.item_cost = cost;
+    a.drop_unit = g_opt_drop_load.load() - 1;
     const int combine_mode = g_opt_combine.load();
     a.fused = combine_mode == 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;
@@ -1759,6 +1764,11 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_prefill_path.store(value);
         return KV_OK;
+    case KV_OPT_TEST_DROP_LOAD:
+        if (value < 0)
+            return KV_ERR_ARG;
+        g_opt_drop_load.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -1783,6 +1793,8 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_item_cost.load();
     case KV_OPT_PREFILL_PATH:
         return g_opt_prefill_path.load();
+    case KV_OPT_TEST_DROP_LOAD:
+        return g_opt_drop_load.load();
     default:
         return -1;
     }
