@@ -262,6 +262,31 @@ def kv_cache_scatter_blocks(caches, inp: torch.Tensor, block_ids: torch.Tensor,
         _cache_dtype(caches[0]), ef, _stream_handle(stream)))
 
 
+def paged_attention_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                   block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                                   stream=None) -> torch.Tensor:
+    """paged_attention_decode with the library's own fixed scratch instead of a caller workspace.
+
+    Calls that can overlap on the GPU share that scratch: serialise them (one stream, or events)."""
+    B, Hq, D = q.shape
+    num_blocks, _, Hkv, Dk = k_cache.shape
+    if Dk != D or tuple(out.shape) != (B, Hq, D) or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("shape mismatch")
+    dt, code = k_cache.dtype, _cache_dtype(k_cache)
+    _check("paged_attention_decode_noalloc", _lib.paged_attention_decode_noalloc(
+        _dev(out, "out", dt), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
+        _stream_handle(stream)))
+    return out
+
+
+def workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    """Zero a workspace on the stream (before first use, and after a call reported KV_STATUS_WAIT_TIMEOUT)."""
+    _check("paged_attention_workspace_init", _lib.paged_attention_workspace_init(
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
+
+
 def read_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
     """Synchronise the stream and return (optionally clearing) the device status word."""
     v = ctypes.c_int32(0)

@@ -33,7 +33,7 @@ def test_wait_runs_out_and_the_context_survives(pkv, oracle_mod, cuda_device, fu
     assert 0.5 < waited < 30.0, waited
     # the context is usable: with the workspace re-initialised (a timed-out call may leave split-K
     # counts behind), a clean call on fresh inputs matches the oracle
-    ws.zero_()
+    pkv.workspace_init(ws)
     case2 = Case(cfg, cuda_device, seed=cfg.seed + 1)
     host2 = case2.host_inputs(0)
     out = gpu_step(pkv, case2, 0, ws, fused=fused)
