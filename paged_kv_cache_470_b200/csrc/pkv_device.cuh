@@ -304,7 +304,7 @@ struct ElemF16 {
     }
 };
 
-// Named barrier over the first `threads` threads of the CTA (id 0 is __syncthreads).
+// Named barrier `id` (0 is __syncthreads's): it completes when `threads` threads, whole warps, have arrived.
 __device__ __forceinline__ void named_barrier(int id, int threads)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

@@ -377,15 +377,18 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
 // row's maximum grows by more than 2^8, which keeps P <= 256; the final
 // division by the row sum makes the result the same as with a rescale at every
 // step. Warp 4 issues the TMA tile loads, warp 5 allocates tensor memory and
-// issues the MMAs. Shared memory, 1024-byte aligned: Q [D/64][128 rows][128 B],
-// then K/V stages [K tiles D/64][64 tokens][128 B] and V likewise, all
-// 128B-swizzled (the MMA descriptors say so).
+// issues the MMAs. K and V have rings of their own: a K stage is free once S of
+// its tile is done, so the loads of K for tile j+2 start while tile j's softmax
+// and P V still run (the producer issues K two tiles ahead of V, which is also
+// the order in which stages come free); with one ring for both, every S waited
+// a whole load latency after the P V before it. Shared memory, 1024-byte aligned:
+// Q [D/64][128 rows][128 B], then the K stages [D/64][64 tokens][128 B], then
+// the V stages likewise, all 128B-swizzled (the MMA descriptors say so).
 // ===========================================================================
 namespace tc {
 
 constexpr int kRows = 128;
 constexpr int kThreads = 192;
-constexpr int kStages = 2;
 constexpr int kTok = 64;               // KV tokens per tile (4 blocks)
 constexpr float kRescaleLog2 = 8.f;    // rescale O when a row maximum grows by more than 2^8
 
@@ -403,15 +406,23 @@ struct TGeo {
     static constexpr int kTiles = D / 64;
     static constexpr int kQBytes = kTiles * kRows * 128;
     static constexpr int kKVTileBytes = kTok * 128;              // one 64-column tile of 64 tokens
-    static constexpr int kStageBytes = 2 * kTiles * kKVTileBytes;
+    static constexpr int kStageBytes = kTiles * kKVTileBytes;     // K (or V) of one tile
+    // tiles of K and of V in flight (two each measured faster than three or four of K, and than
+    // four of each at D = 64)
+    static constexpr int kStagesK = 2;
+    static constexpr int kStagesV = 2;
     static constexpr int kOffQ = 0;
-    static constexpr int kOffKV = kOffQ + kQBytes;
-    static constexpr int kOffBar = kOffKV + kStages * kStageBytes;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kStagesK * kStageBytes;
+    static constexpr int kOffBar = kOffV + kStagesV * kStageBytes;
     // no slack for aligning the base: the buffer is declared 1024-byte aligned (checked at run time),
     // which lets two CTAs share an SM at D = 128
     // at most two CTAs per SM: two of them use all 512 tensor-memory columns (an allocation beyond
     // that would wait for a CTA to finish), so D = 64 asks for more shared memory than it uses
-    static constexpr int kSmemBytes = kOffBar + 128 < 80 * 1024 ? 80 * 1024 : kOffBar + 128;
+    // mbarriers (full and empty per K and V stage, two S buffers, P, P V, Q), the TMEM address and two flags
+    static constexpr int kBarBytes = 256;
+    static_assert((2 * kStagesK + 2 * kStagesV + 5) * 8 + 12 <= kBarBytes, "barrier area");
+    static constexpr int kSmemBytes = kOffBar + kBarBytes < 80 * 1024 ? 80 * 1024 : kOffBar + kBarBytes;
     static constexpr int kTmemCols = 256;                       // S/P buffers at 0 and 64, O at kOCol
     static constexpr int kOCol = 128;
 };
@@ -422,6 +433,7 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                                                               const PrefillArgs a)
 {
     using G = TGeo<D>;
+    constexpr int kStagesK = G::kStagesK, kStagesV = G::kStagesV;
     extern __shared__ __align__(1024) unsigned char smem_tc[];
     const uint32_t base_s = smem_addr(smem_tc);
     unsigned char *base = smem_tc;
@@ -430,10 +442,12 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             flag(a, KV_STATUS_BAD_CONTEXT);
         return;
     }
-    const uint32_t sQ = base_s + G::kOffQ, sKV = base_s + G::kOffKV;
-    uint64_t *full = reinterpret_cast<uint64_t *>(base + G::kOffBar);
-    uint64_t *empty = full + kStages;
-    uint64_t *s_full = empty + kStages;  // [2]: one per S buffer
+    const uint32_t sQ = base_s + G::kOffQ, sK = base_s + G::kOffK, sV = base_s + G::kOffV;
+    uint64_t *fullK = reinterpret_cast<uint64_t *>(base + G::kOffBar);
+    uint64_t *emptyK = fullK + kStagesK;
+    uint64_t *fullV = emptyK + kStagesK;
+    uint64_t *emptyV = fullV + kStagesV;
+    uint64_t *s_full = emptyV + kStagesV;  // [2]: one per S buffer
     uint64_t *p_full = s_full + 2;
     uint64_t *pv_done = p_full + 1;
     uint64_t *q_ready = pv_done + 1;
@@ -467,9 +481,13 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
     constexpr int fmt = E::kDtype == KV_DTYPE_BF16 ? 1 : 0;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < kStagesK; ++s) {
+            mbar_init(&fullK[s], 1);
+            mbar_init(&emptyK[s], 1);
+        }
+        for (int s = 0; s < kStagesV; ++s) {
+            mbar_init(&fullV[s], 1);
+            mbar_init(&emptyV[s], 1);
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
@@ -496,24 +514,28 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
         grid_dependency_wait();
         grid_launch_dependents();
         const int32_t *trow = a.block_tables + static_cast<size_t>(b) * a.W;
-        int issued = 0;
-        for (int jt = 0; jt < ntiles; ++jt) {
-            const int s = jt % kStages;
-            const int kb0 = jt * (kTok / kBlockTokens);
-            const int nb = min(kTok / kBlockTokens, nblk - kb0);
+        // one tile's K (which = 0) or V (which = 1): wait for its stage, then 4 blocks of TMA boxes
+        auto issue = [&](int t, int which) -> bool {
+            const int ns = which == 0 ? kStagesK : kStagesV;
+            const int s = t % ns;
+            const int nb = min(kTok / kBlockTokens, nblk - t * (kTok / kBlockTokens));
+            // the tile's block ids (read again for V: the load is under the wait for the stage)
             int blk = 0;
             if (lane < nb) {
-                blk = __ldg(trow + kb0 + lane);
+                blk = __ldg(trow + t * (kTok / kBlockTokens) + lane);
                 if (blk < 0 || blk >= a.num_blocks) {
-                    flag(a, KV_STATUS_BAD_BLOCK_ID);
+                    if (which == 0)
+                        flag(a, KV_STATUS_BAD_BLOCK_ID);
                     blk = 0;
                 }
             }
+            uint64_t *fb = which == 0 ? &fullK[s] : &fullV[s];
+            uint64_t *eb = which == 0 ? &emptyK[s] : &emptyV[s];
             int ok = 1;
             if (lane == 0) {
-                ok = mbar_wait_bounded(&empty[s], ((jt / kStages) & 1) ^ 1, abort_flag);
+                ok = mbar_wait_bounded(eb, ((t / ns) & 1) ^ 1, abort_flag);
                 if (ok)
-                    mbar_arrive_expect_tx(&full[s], nb * 2 * G::kTiles * 2048);
+                    mbar_arrive_expect_tx(fb, nb * G::kTiles * 2048);
                 else {
                     *abort_flag = 1;
                     flag(a, KV_STATUS_WAIT_TIMEOUT);
@@ -521,23 +543,37 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             }
             ok = __shfl_sync(kFullMask, ok, 0);
             if (!ok)
-                break;
+                return false;
             __syncwarp();
             if (lane < nb) {
-                const uint32_t kdst = sKV + s * G::kStageBytes + lane * 2048;
-                const uint32_t vdst = kdst + G::kTiles * G::kKVTileBytes;
+                const uint32_t dst = (which == 0 ? sK : sV) + s * G::kStageBytes + lane * 2048;
+                const CUtensorMap *tm = which == 0 ? &tmK : &tmV;
 #pragma unroll
-                for (int t = 0; t < G::kTiles; ++t)
-                    tma_load_4d_nohint(kdst + t * G::kKVTileBytes, &tmK, t * 64, 0, j, blk, &full[s]);
-#pragma unroll
-                for (int t = 0; t < G::kTiles; ++t)
-                    tma_load_4d_nohint(vdst + t * G::kKVTileBytes, &tmV, t * 64, 0, j, blk, &full[s]);
+                for (int tt = 0; tt < G::kTiles; ++tt)
+                    tma_load_4d_nohint(dst + tt * G::kKVTileBytes, tm, tt * 64, 0, j, blk, fb);
             }
-            issued = jt + 1;
+            return true;
+        };
+        // K(0) .. K(kStagesK - 1), then V(t), K(t + kStagesK) for each t: the stages come free in
+        // this order (S(t) frees K's stage, P V(t) frees V's, and the MMAs run S(t+1), P V(t), S(t+2))
+        int issuedK = 0, issuedV = 0;
+        bool go = true;
+        for (int t = 0; t < min(kStagesK, ntiles) && go; ++t)
+            if ((go = issue(t, 0)))
+                issuedK = t + 1;
+        for (int t = 0; t < ntiles && go; ++t) {
+            if ((go = issue(t, 1)))
+                issuedV = t + 1;
+            if (go && t + kStagesK < ntiles && (go = issue(t + kStagesK, 0)))
+                issuedK = t + kStagesK + 1;
         }
-        if (lane == 0)
-            for (int jt = max(0, issued - kStages); jt < issued; ++jt)
-                mbar_wait_bounded(&full[jt % kStages], (jt / kStages) & 1, zero_flag);
+        // no load may land after this CTA exits: wait (bounded) for the last ones
+        if (lane == 0) {
+            for (int t = max(0, issuedK - kStagesK); t < issuedK; ++t)
+                mbar_wait_bounded(&fullK[t % kStagesK], (t / kStagesK) & 1, zero_flag);
+            for (int t = max(0, issuedV - kStagesV); t < issuedV; ++t)
+                mbar_wait_bounded(&fullV[t % kStagesV], (t / kStagesV) & 1, zero_flag);
+        }
     } else if (warp == 5) {
         // ---------------- MMA issuer (one thread) ----------------
         grid_dependency_wait();
@@ -549,11 +585,11 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             tcgen05_after_sync();
             // S = Q K^T for tile jt into S buffer jt & 1
             auto issue_s = [&](int jt) -> bool {
-                const int s = jt % kStages;
-                if (!mbar_wait_bounded(&full[s], (jt / kStages) & 1, abort_flag))
+                const int s = jt % kStagesK;
+                if (!mbar_wait_bounded(&fullK[s], (jt / kStagesK) & 1, abort_flag))
                     return false;
                 tcgen05_after_sync();
-                const uint32_t kst = sKV + s * G::kStageBytes;
+                const uint32_t kst = sK + s * G::kStageBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t koff = (kk & 3) * 32;  // 16 elements along the 128-byte row
@@ -562,14 +598,18 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                     umma_f16(tmem + (jt & 1) * kTok, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&s_full[jt & 1]);
+                // S read this K stage: it may be refilled (only a refill waits for this arrival, and
+                // no arrival may still be on its way when the CTA exits)
+                if (jt + kStagesK < ntiles)
+                    umma_commit(&emptyK[s]);
                 return true;
             };
             int done = 0;  // tiles whose PV was issued
             if (ok && ntiles > 0)
                 ok = issue_s(0);
             for (int jt = 0; jt < ntiles && ok; ++jt) {
-                const int s = jt % kStages;
-                const uint32_t vst = sKV + s * G::kStageBytes + G::kTiles * G::kKVTileBytes;
+                const int s = jt % kStagesV;
+                const uint32_t vst = sV + s * G::kStageBytes;
                 if (jt + 1 < ntiles) {
                     // the next S goes into the buffer that P of tile jt-1 used: wait for that PV
                     if (jt >= 1 && !mbar_wait_bounded(pv_done, (jt - 1) & 1, abort_flag)) {
@@ -581,7 +621,8 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                         break;
                     }
                 }
-                if (!mbar_wait_bounded(p_full, jt & 1, abort_flag)) {
+                if (!mbar_wait_bounded(p_full, jt & 1, abort_flag) ||
+                    !mbar_wait_bounded(&fullV[s], (jt / kStagesV) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
@@ -594,7 +635,8 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                                     (jt > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(pv_done);
-                umma_commit(&empty[s]);
+                if (jt + kStagesV < ntiles)
+                    umma_commit(&emptyV[s]);
                 done = jt + 1;
             }
             if (!ok) {
@@ -710,10 +752,18 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             }
             tmem_wait_st();
             l += psum;
-            // tokens of this tile at or past the context hold whatever the stage holds: zero those V rows
-            const int vrow0 = c - tok0;
+            // rows of the CTA's last tile from its last visible token on hold whatever the pool holds
+            // (past the context) or whatever the stage held before (blocks not loaded): zero those V
+            // rows, whose P is 0, so that 0 * V stays 0 -- once V's loads have landed (S only says
+            // that K's have)
+            const int vrow0 = kv_len - tok0;
             if (vrow0 < kTok) {
-                const uint32_t vst = sKV + (jt % kStages) * G::kStageBytes + G::kTiles * G::kKVTileBytes;
+                if (!__all_sync(kFullMask, mbar_wait_bounded(&fullV[jt % kStagesV], (jt / kStagesV) & 1,
+                                                             abort_flag))) {
+                    good = false;
+                    break;
+                }
+                const uint32_t vst = sV + (jt % kStagesV) * G::kStageBytes;
                 const int cnt = (kTok - vrow0) * G::kTiles * 8;
                 for (int idx = r; idx < cnt; idx += kRows) {
                     const int rr = vrow0 + idx / (G::kTiles * 8);

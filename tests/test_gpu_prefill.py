@@ -126,3 +126,25 @@ def test_bad_chunks_are_flagged(pkv, cuda_device, path):
     pkv.paged_attention_prefill(out, case.q, case.k, case.v, tables, case.lens, case.qs, case.max_q, cfg.scale, flag)
     torch.cuda.synchronize()
     assert int(flag.item()) & pkv.KV_STATUS_BAD_BLOCK_ID
+
+
+@pytest.mark.parametrize("path", sorted(PREFILL_PATHS))
+@pytest.mark.parametrize("D", [64, 128])
+def test_stale_shared_memory_stays_out(pkv, oracle_mod, cuda_device, D, path):
+    """A launch over a cache of NaNs first leaves NaNs in every SM's tile stages; a CTA whose rows end
+    before its sequence does, and whose last tile has blocks it does not load, must not let those
+    stale rows (or the pool's rows past the context) into its output."""
+    pkv.set_option(pkv.KV_OPT_PREFILL_PATH, PREFILL_PATHS[path])
+    Hq, Hkv = (16, 4) if D == 128 else (20, 4)
+    poison = workloads.PrefillConfig("test", Hq, Hkv, D, 64, 256, 0, 1024, 80, seed=11)
+    pc = PrefillCase(poison, cuda_device)
+    pc.k.view(torch.int16).fill_(0x7fc0)            # bf16 and fp16 NaN patterns alike
+    pc.v.view(torch.int16).fill_(0x7fc0)
+    junk = torch.empty_like(pc.q)
+    pkv.paged_attention_prefill(junk, pc.q, pc.k, pc.v, pc.tables, pc.lens, pc.qs, pc.max_q, poison.scale)
+    torch.cuda.synchronize()
+    chunk = [100, 37, 130, 9]
+    prior = [33, 3, 70, 200]
+    cfg = workloads.PrefillConfig("test", Hq, Hkv, D, len(chunk), 0, 0, 0, 32, seed=12)
+    case = PrefillCase(cfg, cuda_device, chunk_lens=chunk, prior_lens=prior)
+    run_case(pkv, oracle_mod, case, f"after a NaN launch, D{D} {path}")
