@@ -275,6 +275,11 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     KV_STATUS_WAIT_TIMEOUT in the status word and its output
  *                     is not valid; the context stays usable (re-initialise
  *                     the workspace, as after any timed-out call).
+ *   KV_OPT_TEST_SLOW_SOFTMAX: test hook for the hand-offs of the tcgen05
+ *                     prefill, 0 (default) off; 1: in every CTA the first
+ *                     softmax warp waits about 30 microseconds before it hands
+ *                     over P of the first tile, so the other warps run a tile
+ *                     ahead of it. The output must not change.
  * Kernels are launched with programmatic dependent launch. q, k_new, v_new,
  * the caches, the workspace and out are touched only after the previous kernel
  * in the stream has completed; block_tables and context_lens are read before
@@ -290,6 +295,7 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
 #define KV_OPT_ITEM_COST 7
 #define KV_OPT_PREFILL_PATH 8
 #define KV_OPT_TEST_DROP_LOAD 9
+#define KV_OPT_TEST_SLOW_SOFTMAX 10
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

@@ -28,6 +28,7 @@ KV_STATUS_BAD_BLOCK_ID, KV_STATUS_BAD_CONTEXT, KV_STATUS_WAIT_TIMEOUT, KV_STATUS
 KV_OPT_COMPUTE, KV_OPT_COMBINE, KV_OPT_GRID, KV_OPT_MIN_CHUNK, KV_OPT_PRODUCER_LANES, KV_OPT_HEAD_GROUP = (
     1, 2, 3, 4, 5, 6)
 KV_OPT_ITEM_COST, KV_OPT_PREFILL_PATH, KV_OPT_TEST_DROP_LOAD = 7, 8, 9
+KV_OPT_TEST_SLOW_SOFTMAX = 10
 COMPUTE_AUTO, COMPUTE_TENSOR_CORES, COMPUTE_CUDA_CORES = 0, 1, 2
 
 _P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t

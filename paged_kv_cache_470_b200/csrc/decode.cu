@@ -1331,6 +1331,7 @@ std::atomic<int> g_opt_head_group{0};
 std::atomic<int> g_opt_item_cost{0};
 std::atomic<int> g_opt_prefill_path{0};
 std::atomic<int> g_opt_drop_load{0};
+std::atomic<int> g_opt_slow_softmax{0};
 constexpr int kDefaultMinChunk = 4;
 
 // Work positions charged per work item (its fixed cost, in units of one work
@@ -1769,6 +1770,11 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_drop_load.store(value);
         return KV_OK;
+    case KV_OPT_TEST_SLOW_SOFTMAX:
+        if (value < 0 || value > 1)
+            return KV_ERR_ARG;
+        g_opt_slow_softmax.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -1795,10 +1801,13 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_prefill_path.load();
     case KV_OPT_TEST_DROP_LOAD:
         return g_opt_drop_load.load();
+    case KV_OPT_TEST_SLOW_SOFTMAX:
+        return g_opt_slow_softmax.load();
     default:
         return -1;
     }
 }
 
-// The prefill path switch (read by prefill.cu).
+// The prefill path switch and test hook (read by prefill.cu).
 int pkv_prefill_path() { return g_opt_prefill_path.load(); }
+int pkv_prefill_slow_softmax() { return g_opt_slow_softmax.load(); }

@@ -62,6 +62,7 @@ struct PrefillArgs {
     int32_t *status;             // may be null
     int B, W, Hq, Hkv, group, num_blocks, max_tiles, max_query_len;
     float scale_log2;
+    int slow_softmax;  // test hook: the tcgen05 path's first softmax warp hands over its first P late
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
@@ -419,9 +420,10 @@ struct TGeo {
     // which lets two CTAs share an SM at D = 128
     // at most two CTAs per SM: two of them use all 512 tensor-memory columns (an allocation beyond
     // that would wait for a CTA to finish), so D = 64 asks for more shared memory than it uses
-    // mbarriers (full and empty per K and V stage, two S buffers, P, P V, Q), the TMEM address and two flags
+    // mbarriers (full and empty per K and V stage, two S buffers, two P, P V, all MMAs, Q), the TMEM
+    // address and two flags
     static constexpr int kBarBytes = 256;
-    static_assert((2 * kStagesK + 2 * kStagesV + 5) * 8 + 12 <= kBarBytes, "barrier area");
+    static_assert((2 * kStagesK + 2 * kStagesV + 7) * 8 + 12 <= kBarBytes, "barrier area");
     static constexpr int kSmemBytes = kOffBar + kBarBytes < 80 * 1024 ? 80 * 1024 : kOffBar + kBarBytes;
     static constexpr int kTmemCols = 256;                       // S/P buffers at 0 and 64, O at kOCol
     static constexpr int kOCol = 128;
@@ -448,9 +450,17 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
     uint64_t *fullV = emptyK + kStagesK;
     uint64_t *emptyV = fullV + kStagesV;
     uint64_t *s_full = emptyV + kStagesV;  // [2]: one per S buffer
+    // P of tile j is ready: one barrier per tile parity. With one, a warp that finished tile j + 1
+    // could arrive again before a slower warp had arrived for tile j, completing that phase early;
+    // with two, arriving twice on one would take a warp two tiles ahead, and S of tile j + 2 waits
+    // for the P V of tile j
     uint64_t *p_full = s_full + 2;
-    uint64_t *pv_done = p_full + 1;
-    uint64_t *q_ready = pv_done + 1;
+    uint64_t *pv_done = p_full + 2;
+    // every MMA of the CTA is done: one phase, committed once after the last P V. The epilogue cannot
+    // use pv_done: while another warp is a tile behind, pv_done can be two phases short of the last,
+    // and a parity wait cannot tell two phases apart
+    uint64_t *o_done = pv_done + 1;
+    uint64_t *q_ready = o_done + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_ready + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
     volatile int *zero_flag = abort_flag + 1;
@@ -491,8 +501,10 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
         }
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
-        mbar_init(p_full, kRows);
+        mbar_init(&p_full[0], kRows);
+        mbar_init(&p_full[1], kRows);
         mbar_init(pv_done, 1);
+        mbar_init(o_done, 1);
         mbar_init(q_ready, kRows);
         mbar_fence_init();
         *abort_flag = 0;
@@ -604,7 +616,6 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                     umma_commit(&emptyK[s]);
                 return true;
             };
-            int done = 0;  // tiles whose PV was issued
             if (ok && ntiles > 0)
                 ok = issue_s(0);
             for (int jt = 0; jt < ntiles && ok; ++jt) {
@@ -621,7 +632,7 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                         break;
                     }
                 }
-                if (!mbar_wait_bounded(p_full, jt & 1, abort_flag) ||
+                if (!mbar_wait_bounded(&p_full[jt & 1], (jt >> 1) & 1, abort_flag) ||
                     !mbar_wait_bounded(&fullV[s], (jt / kStagesV) & 1, abort_flag)) {
                     ok = false;
                     break;
@@ -637,15 +648,15 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 umma_commit(pv_done);
                 if (jt + kStagesV < ntiles)
                     umma_commit(&emptyV[s]);
-                done = jt + 1;
             }
             if (!ok) {
                 *abort_flag = 1;
                 flag(a, KV_STATUS_WAIT_TIMEOUT);
             }
-            // the MMAs in flight finish before tensor memory is released (below)
-            if (done > 0)
-                mbar_wait_bounded(pv_done, (done - 1) & 1, zero_flag);
+            // the epilogue reads O once every MMA issued here is done, and they finish before tensor
+            // memory is released (below)
+            umma_commit(o_done);
+            mbar_wait_bounded(o_done, 0, zero_flag);
         }
         __syncwarp();
     } else {
@@ -776,10 +787,16 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tcgen05_before_sync();
-            mbar_arrive(p_full);
+            if (a.slow_softmax && warp == 0 && jt == 0) {
+                // test hook: let the other warps run a tile ahead of this one (a bounded wait)
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 30000u)
+                    __nanosleep(1000);
+            }
+            mbar_arrive(&p_full[jt & 1]);
         }
         // epilogue: O / l
-        if (__all_sync(kFullMask, good && mbar_wait_bounded(pv_done, (ntiles - 1) & 1, abort_flag))) {
+        if (__all_sync(kFullMask, good && mbar_wait_bounded(o_done, 0, abort_flag))) {
             tcgen05_after_sync();
             const float inv = 1.f / l;
             uint16_t *dst = a.out + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D;
@@ -820,8 +837,9 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
 }  // namespace prefill
 }  // namespace pkv
 
-// KV_OPT_PREFILL_PATH, kept with the other switches in decode.cu
+// KV_OPT_PREFILL_PATH and KV_OPT_TEST_SLOW_SOFTMAX, kept with the other switches in decode.cu
 int pkv_prefill_path();
+int pkv_prefill_slow_softmax();
 
 namespace {
 
@@ -923,6 +941,7 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
     a.max_tiles = static_cast<int>(tiles);
     a.max_query_len = max_query_len;
     a.scale_log2 = scale * 1.4426950408889634f;
+    a.slow_softmax = pkv_prefill_slow_softmax();
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));

@@ -52,3 +52,23 @@ def test_host_argument_checks_need_no_gpu(pkv):
     assert rc == pkv.KV_ERR_ARG
     assert pkv.set_option(pkv.KV_OPT_COMPUTE, 0) is None
     assert lib.kv_decode_set_option(99, 0) == pkv.KV_ERR_ARG
+
+
+def test_option_ranges_need_no_gpu(pkv):
+    """Every switch takes its documented values, keeps them, and refuses the rest."""
+    lib = ctypes.CDLL(pkv.LIB_PATH)
+    lib.kv_decode_set_option.restype = ctypes.c_int
+    lib.kv_decode_get_option.restype = ctypes.c_int
+    cases = {pkv.KV_OPT_PREFILL_PATH: ([0, 1, 2], [-1, 3]),
+             pkv.KV_OPT_TEST_SLOW_SOFTMAX: ([0, 1], [-1, 2]),
+             pkv.KV_OPT_TEST_DROP_LOAD: ([0, 5], [-1]),
+             pkv.KV_OPT_ITEM_COST: ([-1, 0, 64], [-2, 65])}
+    for key, (good, bad) in cases.items():
+        before = lib.kv_decode_get_option(key)
+        for v in good:
+            assert lib.kv_decode_set_option(key, v) == pkv.KV_OK
+            assert lib.kv_decode_get_option(key) == v
+        for v in bad:
+            assert lib.kv_decode_set_option(key, v) == pkv.KV_ERR_ARG
+            assert lib.kv_decode_get_option(key) == good[-1]
+        assert lib.kv_decode_set_option(key, before) == pkv.KV_OK
