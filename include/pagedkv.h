@@ -233,12 +233,17 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
  *
  * q, out: [T][Hq][D] device, T = query_start[B]; query_start: [B+1] device
  * int32, non-decreasing from 0; max_query_len >= every n_b (it sizes the
- * grid). Tensor cores (mma.sync), fp32 accumulation, the probabilities rounded
+ * grid). Tensor cores (tcgen05.mma with tensor-memory accumulators; mma.sync
+ * with KV_OPT_PREFILL_PATH = 2), fp32 accumulation, the probabilities rounded
  * to the element type before they multiply V. No workspace. Data errors are
  * OR-ed into *error_flag (device int32, may be NULL): KV_STATUS_BAD_CONTEXT
  * when n_b > c_b, c_b > 16 * max_blocks_per_seq or n_b > max_query_len (that
  * sequence's rows are not written), KV_STATUS_BAD_BLOCK_ID for ids outside the
- * pool (block 0 is read instead). B <= 65535, Hkv <= 65535, scale > 0.
+ * pool (block 0 is read instead), KV_STATUS_WAIT_TIMEOUT if an internal wait
+ * gave up (~1 s; the output is not valid). B <= 65535, Hkv <= 65535, scale > 0.
+ * Launched with programmatic dependent launch: query_start and context_lens
+ * are read before the previous kernel in the stream has completed (it must not
+ * write them); q, the caches, block_tables, out and *error_flag after.
  */
 KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k_cache,
                                          const void *v_cache, const int32_t *block_tables,

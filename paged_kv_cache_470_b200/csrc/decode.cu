@@ -859,14 +859,21 @@ __device__ __forceinline__ void zero_empty_outputs(const DecodeArgs &a, int tid,
 }
 
 // Lane i (< m) reads the block id of unit cur.off + i of sequence cur.b; ids
-// outside the pool are flagged and replaced by block 0 (never read out of bounds).
-__device__ __forceinline__ int load_block_ids(const DecodeArgs &a, const Cursor &cur, int m, int lane)
+// outside the pool are replaced by block 0 (never read out of bounds) and
+// flagged: in the status word, or, for a read made before the grid dependency
+// wait (the workspace is the previous kernel's until then), in *bad, for the
+// caller to report after the wait.
+__device__ __forceinline__ int load_block_ids(const DecodeArgs &a, const Cursor &cur, int m, int lane,
+                                              int *bad = nullptr)
 {
     int blk = 0;
     if (lane < m) {
         blk = __ldg(a.block_tables + static_cast<size_t>(cur.b) * a.W + cur.off + lane);
         if (blk < 0 || blk >= a.num_blocks) {
-            atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
+            if (bad)
+                *bad = 1;
+            else
+                atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
             blk = 0;
         }
     }
@@ -982,9 +989,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // The first batch of block ids is read before waiting on the previous
         // grid (the tables must not come from the kernel launched just before);
         // the cache is only touched after the wait.
-        int blk_first = load_block_ids(a, cur0, min(32, min(cur0.n - cur0.off, count)), lane);
+        int bad_first = 0;
+        int blk_first = load_block_ids(a, cur0, min(32, min(cur0.n - cur0.off, count)), lane, &bad_first);
         grid_dependency_wait();
         grid_launch_dependents();
+        if (bad_first)
+            atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
         const uint64_t policy = l2_policy_evict_first();
         const int NL = a.prod_lanes;
         Cursor cur = cur0;

@@ -102,8 +102,10 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
     if (n <= 0)
         return;
     if (n > c || c > a.W * kBlockTokens || n > a.max_query_len) {
-        if (tid == 0 && j == 0 && tile == a.max_tiles - 1)
+        if (tid == 0 && j == 0 && tile == a.max_tiles - 1) {
+            grid_dependency_wait();  // the flag is the previous kernel's until then
             flag(a, KV_STATUS_BAD_CONTEXT);
+        }
         return;
     }
     const int rows_total = n * g;
@@ -440,8 +442,10 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
     const uint32_t base_s = smem_addr(smem_tc);
     unsigned char *base = smem_tc;
     if (base_s & 1023u) {  // the swizzle atoms need 1024-byte alignment
-        if (threadIdx.x == 0)
+        if (threadIdx.x == 0) {
+            grid_dependency_wait();  // the flag is the previous kernel's until then
             flag(a, KV_STATUS_BAD_CONTEXT);
+        }
         return;
     }
     const uint32_t sQ = base_s + G::kOffQ, sK = base_s + G::kOffK, sV = base_s + G::kOffV;
@@ -475,8 +479,10 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
     if (n <= 0)
         return;
     if (n > c || c > a.W * kBlockTokens || n > a.max_query_len) {
-        if (tid == 0 && j == 0 && tile == a.max_tiles - 1)
+        if (tid == 0 && j == 0 && tile == a.max_tiles - 1) {
+            grid_dependency_wait();  // the flag is the previous kernel's until then
             flag(a, KV_STATUS_BAD_CONTEXT);
+        }
         return;
     }
     const int rows_total = n * g;
