@@ -79,6 +79,12 @@ def layer_bytes(cfg, lens, shares_prefix=None, unique_prefix=False):
             "decode_kernel": kv + qo + tables, "total": kv + qo + tables + append}
 
 
+def prefill_pairs(context_lens, chunk_lens):
+    """(query, visible token) pairs of a chunked prefill: chunk token i of a sequence with c tokens
+    (its n-token chunk included) sits at position c - n + i and sees positions 0 .. c - n + i."""
+    return sum(sum(int(c) - int(n) + i + 1 for i in range(int(n))) for c, n in zip(context_lens, chunk_lens))
+
+
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -409,8 +415,7 @@ def prefill_measure(pkv, device, elem, reps=20, keys=("llama3_8b", "0p5b")):
         tables, lens, qs = (layout.block_tables.to(device), layout.context_lens.to(device),
                             layout.query_start.to(device))
         flag = torch.zeros(1, dtype=torch.int32, device=device)
-        pairs = sum(sum(int(c) - int(n) + i + 1 for i in range(int(n)))
-                    for c, n in zip(layout.context_lens.tolist(), layout.chunk_lens.tolist()))
+        pairs = prefill_pairs(layout.context_lens.tolist(), layout.chunk_lens.tolist())
         flops = 4.0 * cfg.Hq * cfg.D * pairs
         stream = torch.cuda.current_stream()
 
@@ -429,7 +434,9 @@ def prefill_measure(pkv, device, elem, reps=20, keys=("llama3_8b", "0p5b")):
         res[key] = {"workload": cfg.name, "bound": "tensor", "achieved": round(tf, 1), "unit": "TFLOP/s",
                     "peak": peak, "peak_kind": kind, "frac": round(tf / peak, 4), "ms": round(ms, 4),
                     "flops_per_launch": flops, "status": int(flag.item()),
-                    "arithmetic": f"mma.sync m16n8k16 {elem} in, fp32 accumulate",
+                    "arithmetic": (f"mma.sync m16n8k16 {elem} in, fp32 accumulate"
+                                   if pkv.get_option(pkv.KV_OPT_PREFILL_PATH) == 2 else
+                                   f"tcgen05.mma kind::f16 M=128 {elem} in, fp32 accumulate in tensor memory"),
                     "timing": f"CUDA events, mean of {reps} back-to-back launches after 3 warm-up launches; "
                               f"KV {2 * k.numel() * k.element_size() / 1e6:.0f} MB + q "
                               f"{q.numel() * q.element_size() / 1e6:.0f} MB per launch (L2 126 MB)"}
