@@ -72,3 +72,32 @@ def test_option_ranges_need_no_gpu(pkv):
             assert lib.kv_decode_set_option(key, v) == pkv.KV_ERR_ARG
             assert lib.kv_decode_get_option(key) == good[-1]
         assert lib.kv_decode_set_option(key, before) == pkv.KV_OK
+
+
+def test_binding_has_every_call_under_its_own_name(pkv):
+    """Every call the header declares is a Python function of the same name."""
+    for name in declared_functions():
+        assert callable(getattr(pkv, name, None)), f"{name} has no same-named binding"
+
+
+def test_pool_calls_by_their_abi_names_need_no_gpu(pkv):
+    import torch
+    pool = pkv.kv_pool_create(8)
+    ids = pkv.kv_pool_alloc(pool, 3)
+    assert pkv.kv_pool_num_free(pool) == 5 and pkv.kv_pool_num_blocks(pool) == 8
+    child = pkv.kv_pool_fork(pool, ids[:2])
+    assert child == ids[:2] and pkv.kv_pool_refcount(pool, ids[0]) == 2
+    pkv.kv_pool_incref(pool, [ids[2]])
+    pkv.kv_pool_free(pool, [ids[2], ids[2]])
+    assert pkv.kv_pool_refcount(pool, ids[2]) == 0 and pkv.kv_pool_num_free(pool) == 6
+    # one step of bookkeeping for a sequence with 16 tokens: it needs a second block
+    tables = torch.full((1, 4), -1, dtype=torch.int32)
+    tables[0, 0] = ids[1]
+    lens = torch.tensor([16], dtype=torch.int32)
+    slots = torch.zeros(1, dtype=torch.int64)
+    pkv.kv_pool_append_slots(pool, tables, lens, slots)
+    assert int(lens[0]) == 17 and int(tables[0, 1]) >= 0 and int(slots[0]) == int(tables[0, 1]) * 16
+    src, dst = pkv.kv_pool_append_slots_cow(pool, tables, lens, slots)
+    assert (src, dst) == ([], []) and int(lens[0]) == 18
+    assert pkv.kv_decode_get_option(pkv.KV_OPT_PREFILL_PATH) == pkv.get_option(pkv.KV_OPT_PREFILL_PATH)
+    pkv.kv_pool_destroy(pool)
