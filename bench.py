@@ -740,7 +740,7 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=2, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--config", type=int, default=2, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--compute", choices=["tensor", "cuda"], default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)

@@ -77,7 +77,7 @@ class DecodeConfig:
         return 470 + self.cid
 
 
-CONFIGS = {
+WORKLOADS = {
     1: DecodeConfig(1, "tiny paged decode (1 layer, Hq=20, Hkv=4, D=64, batch 4, ctx U[1,256], 128-block pool)",
                     1, 20, 4, 64, 4, "uniform", 1, 256, 16, pool_blocks=128),
     2: DecodeConfig(2, "0.5B GQA decode step (24 layers, Hq=20, Hkv=4, D=64, batch 64, ctx U[128,2048])",
@@ -217,7 +217,7 @@ def make_step_inputs(cfg: DecodeConfig, gen: torch.Generator, device, n_layers=N
 
 def small_config(cid: int = 1, **overrides) -> DecodeConfig:
     """A copy of one workload with some fields changed (edge-case and CPU-sized tests)."""
-    return replace(CONFIGS[cid], **overrides)
+    return replace(WORKLOADS[cid], **overrides)
 
 
 # ---------------------------------------------------------------------------

@@ -39,7 +39,7 @@ def walk_layout(layout):
 
 @pytest.mark.parametrize("cid", [1, 2, 5])
 def test_decode_layer_bytes_match_a_walk_of_the_tables(bench, cid):
-    cfg = workloads.CONFIGS[cid]
+    cfg = workloads.WORKLOADS[cid]
     layout = workloads.draw_layout(cfg)
     lens = layout.context_lens.tolist()
     share = layout.shares_prefix.tolist()
@@ -84,7 +84,7 @@ def test_prefill_pairs_edge_cases(bench):
 
 def test_profiled_traffic_needs_the_current_source_and_workload(bench, tmp_path, monkeypatch):
     src = hashlib.sha256(open(bench.DECODE_SRC, "rb").read()).hexdigest()[:16]
-    cfg = workloads.CONFIGS[2]
+    cfg = workloads.WORKLOADS[2]
     monkeypatch.setattr(bench, "PROFILE_DIR", str(tmp_path))
 
     def write(h, cid=2, elem="bf16"):

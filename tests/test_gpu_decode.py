@@ -49,7 +49,7 @@ def run_and_check(pkv, oracle_mod, case, layers=None, what="", fused=None):
 def test_tiny_workload(pkv, oracle_mod, cuda_device, path, combine, fused):
     pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
     pkv.set_option(pkv.KV_OPT_COMBINE, combine)
-    case = Case(workloads.CONFIGS[1], cuda_device)
+    case = Case(workloads.WORKLOADS[1], cuda_device)
     run_and_check(pkv, oracle_mod, case, what=f"tiny/{path}/combine{combine}", fused=fused)
 
 
@@ -225,7 +225,7 @@ def test_append_bit_exact_with_padding_and_bad_slots(pkv, oracle_mod, cuda_devic
 # full-size workloads, in the launch configuration the bench times
 # ---------------------------------------------------------------------------
 def _full_size(pkv, oracle_mod, cuda_device, cid, n_alloc):
-    cfg = workloads.CONFIGS[cid]
+    cfg = workloads.WORKLOADS[cid]
     case = Case(cfg, cuda_device, n_layers=n_alloc)
     layers = sorted({0, n_alloc - 1, random.Random(cid).randrange(n_alloc)})
     run_and_check(pkv, oracle_mod, case, layers=layers, what=f"config {cid}")
@@ -250,7 +250,7 @@ def test_full_size_70b_mix_with_shared_prefix(pkv, oracle_mod, cuda_device):
 def test_full_size_70b_mix_after_redraws(pkv, oracle_mod, cuda_device):
     """The 70B-style mix after two steps of re-drawing 10% of the batch through the block pool."""
     from paged_kv_cache_470_b200.batch import ContinuousBatch
-    cfg = workloads.CONFIGS[5]
+    cfg = workloads.WORKLOADS[5]
     cb = ContinuousBatch(cfg, int(workloads.draw_layout(cfg).num_blocks * 1.25))
     cb.redraw()
     cb.redraw()
