@@ -4,6 +4,8 @@ import os
 import re
 import subprocess
 
+import pytest
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "pagedkv.h")
 
@@ -101,3 +103,37 @@ def test_pool_calls_by_their_abi_names_need_no_gpu(pkv):
     assert (src, dst) == ([], []) and int(lens[0]) == 18
     assert pkv.kv_decode_get_option(pkv.KV_OPT_PREFILL_PATH) == pkv.get_option(pkv.KV_OPT_PREFILL_PATH)
     pkv.kv_pool_destroy(pool)
+
+
+C_CLIENT = r"""
+#include "pagedkv.h"
+#include <stdio.h>
+int main(void) {
+    void *pool = 0;
+    int32_t ids[3], child[2];
+    if (kv_pool_create(8, &pool) != KV_OK) return 1;
+    if (kv_pool_alloc(pool, 3, ids) != KV_OK || kv_pool_num_free(pool) != 5) return 2;
+    if (kv_pool_fork(pool, ids, 2, child) != KV_OK || kv_pool_refcount(pool, ids[0]) != 2) return 3;
+    if (kv_pool_free(pool, child, 2) != KV_OK || kv_pool_free(pool, ids, 3) != KV_OK) return 4;
+    if (kv_pool_num_free(pool) != 8 || kv_pool_alloc(pool, 9, ids) != KV_ERR_OOM) return 5;
+    kv_pool_destroy(pool);
+    if (kv_decode_set_option(99, 0) != KV_ERR_ARG) return 6;
+    printf("c client ok\n");
+    return 0;
+}
+"""
+
+
+def test_a_plain_c_program_uses_the_library(pkv, tmp_path):
+    """The boundary is a C ABI: a C99 program includes the header, links the library and calls it."""
+    import shutil
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(pkv.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                    "-L", libdir, "-lpagedkv", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "c client ok", (out.returncode, out.stdout, out.stderr)
