@@ -6,8 +6,15 @@
  *   kv_cache_append         scatter each new token's K and V rows into its slot
  *   paged_attention_decode  out = softmax(scale * q K^T) V per query head,
  *                           reading K/V through per-sequence block tables
+ *   paged_attention_decode_append   the two above in one launch
+ *   paged_attention_prefill chunked prefill: a chunk of query tokens per
+ *                           sequence, causal over the same cache
+ *   kv_cache_copy_blocks, kv_cache_gather_blocks, kv_cache_scatter_blocks
+ *                           whole-block moves over every layer's caches
+ *                           (copy-on-write, swap-out, swap-in)
  *   kv_pool_*               host bookkeeping of physical blocks: allocate,
- *                           free, and reference counts for shared prefixes
+ *                           free, reference counts for shared prefixes, fork,
+ *                           per-step slots (with copy-on-write)
  *
  * Sources for what is computed:
  *   - "Module 23: Serving", section 23.4 (Paged Attention): the cache lives in
@@ -115,7 +122,7 @@ KV_API kv_status kv_cache_append(const void *k_new, const void *v_new,
 /*
  * Bytes of device workspace paged_attention_decode needs for these sizes on
  * the current device (it depends on the device's SM count). Returns 0 for
- * invalid sizes. The workspace holds a status word, split-K partial results
+ * invalid sizes, or when no CUDA device can be queried. The workspace holds a status word, split-K partial results
  * and one counter per (sequence, kv head) work item.
  */
 KV_API size_t paged_attention_workspace_size(int B, int Hq, int Hkv, int D);
