@@ -1,13 +1,20 @@
 """Benchmark: one decode step (append + paged attention over every layer) on one or more B200s.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 4] [--impl ours|reference]
 
 A step is the whole hot path over one batch: for each layer, scatter the new
 token's K/V into its slot, then decode attention over every sequence's paged
 cache (with the split-K merge). Inputs are synthetic and seeded, shaped like
-the pages' models (see paged_kv_cache_470_b200/workloads.py); the default is
-the 0.5B GQA model's decode step (24 layers, Hq=20, Hkv=4, D=64, batch 64,
-context U[128,2048]).
+the pages' models (see paged_kv_cache_470_b200/workloads.py). The headline
+workload is the largest one that fits one GPU: the LLaMA-2-7B-shaped MHA step
+(32 layers, Hq = Hkv = 32, D = 128, batch 32, every context 4096: 64 GiB of
+KV). The other workloads are measured in the same run under `per_config`.
+
+The step runs as the library's multi-layer call (paged_attention_decode_layers
+with the append fused: one launch for all layers, inputs all present). Beside
+it, `per_layer` times the same step as one fused append + decode launch per
+layer, which is what a transformer forward pays (its layer l + 1 query comes
+from layer l's output).
 
 Reported (one JSON line on rank 0):
   value      achieved HBM GB/s = algorithmic bytes of the step / step time,
@@ -15,8 +22,10 @@ Reported (one JSON line on rank 0):
   e2e        the same metric through the C ABI with host buffers: pinned-host
              -> device copies of the step's inputs and a device -> host copy of
              its outputs inside the timed region
-  roofline   the decode kernel alone: its algorithmic bytes per launch over its
+  roofline   the step's kernel: its algorithmic bytes per launch over its
              CUDA-event duration, against the measured HBM copy bandwidth
+  per_config the other workloads, each with its own step time, roofline,
+             per-layer figures and clock record
   cpu_baseline  the float64 oracle on this host's cores, on a bounded sample
 
 With --gpus N > 1 (under torchrun) each rank runs an independent replica of
@@ -37,6 +46,7 @@ import statistics
 import sys
 import threading
 import time
+from dataclasses import replace
 
 import torch
 
@@ -103,22 +113,31 @@ def measured_tensor_peak():
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def profiled_traffic(cfg):
-    """DRAM bytes per decode launch from a committed ncu summary of this workload and element type,
-    if one matches the current kernel source (else None)."""
+def profiled_traffic(cfg, launch="layers"):
+    """DRAM bytes per launch from a committed ncu summary of this workload, element type and kind of launch
+    ("layers": the multi-layer launch, whose summary gives bytes per layer, scaled here to the workload's layer
+    count; "per_layer": one layer's launch), if one matches the current kernel source (else None)."""
     try:
         src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
         for name in sorted(os.listdir(PROFILE_DIR)):
             if not name.endswith(".txt"):
                 continue
             text = open(os.path.join(PROFILE_DIR, name)).read()
-            m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
             h = re.search(r"decode\.cu sha256\[:16\]:\s*([0-9a-f]+)", text)
             c = re.search(r"^config_id:\s*(\d+)", text, re.M)
             e = re.search(r"^elem:\s*(\w+)", text, re.M)
-            if m and h and c and e and h.group(1) == src_hash and int(c.group(1)) == cfg.cid \
-                    and e.group(1) == cfg.elem:
-                return float(m.group(1))
+            k = re.search(r"^launch:\s*(\w+)", text, re.M)
+            if not (h and c and e and k) or h.group(1) != src_hash or int(c.group(1)) != cfg.cid \
+                    or e.group(1) != cfg.elem or k.group(1) != launch:
+                continue
+            if launch == "layers":
+                m = re.search(r"dram_bytes_per_layer:\s*([0-9.eE+]+)", text)
+                if m:
+                    return float(m.group(1)) * cfg.n_layers
+            else:
+                m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+                if m:
+                    return float(m.group(1))
     except OSError:
         pass
     return None
@@ -228,6 +247,9 @@ def dist_done(world: int):
 # the GPU arm
 # ---------------------------------------------------------------------------
 class Workload:
+    """One workload resident on the GPU: every layer's K and V pools (two stacked tensors, one view per layer),
+    this step's q and new K/V rows of every layer, the tables, lengths and slots, and the outputs."""
+
     def __init__(self, cfg, device, rank=0):
         import paged_kv_cache_470_b200 as pkv
         self.pkv = pkv
@@ -238,17 +260,16 @@ class Workload:
             from paged_kv_cache_470_b200.batch import ContinuousBatch
             self.layout = ContinuousBatch(cfg, int(self.layout.num_blocks * 1.25), seed=cfg.seed + 1000 * rank)
         gen = workloads.device_generator(cfg.seed + 1000 * rank, device)
-        self.k, self.v = [], []
-        for _ in range(cfg.n_layers):
-            k, v = workloads.make_layer_cache(self.layout.num_blocks, cfg.Hkv, cfg.D, gen, device, cfg.torch_dtype)
-            self.k.append(k)
-            self.v.append(v)
+        self.k_all, self.v_all = workloads.make_stacked_caches(cfg.n_layers, self.layout.num_blocks, cfg.Hkv, cfg.D,
+                                                               gen, device, cfg.torch_dtype)
+        self.k, self.v = list(self.k_all.unbind(0)), list(self.v_all.unbind(0))
         self.q, self.k_new, self.v_new = workloads.make_step_inputs(cfg, gen, device)
         self.tables = self.layout.block_tables.to(device)
         self.lens = self.layout.context_lens.to(device)
         self.slots = self.layout.slot_mapping().to(device)
         self.out = torch.empty_like(self.q)
-        self.ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D, device)
+        self.ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D, device)                  # per-layer calls
+        self.ws_all = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D, device, cfg.n_layers)  # one launch
         self.fused = True
 
     def redraw(self):
@@ -257,6 +278,14 @@ class Workload:
         self.tables.copy_(self.layout.block_tables)
         self.lens.copy_(self.layout.context_lens)
         self.slots.copy_(self.layout.slot_mapping())
+
+    def layers_call(self, lo=0, hi=None, stream=None, ws=None):
+        """Layers lo .. hi - 1 in one launch, the append fused (paged_attention_decode_layers)."""
+        hi = self.cfg.n_layers if hi is None else hi
+        self.pkv.paged_attention_decode_layers(self.out[lo:hi], self.q[lo:hi], self.k_all[lo:hi], self.v_all[lo:hi],
+                                               self.tables, self.lens, self.cfg.scale,
+                                               self.ws_all if ws is None else ws, k_new=self.k_new[lo:hi],
+                                               v_new=self.v_new[lo:hi], slot_mapping=self.slots, stream=stream)
 
     def layer(self, layer, stream=None):
         """One layer: append this step's token and attend (one fused launch, or two kernels)."""
@@ -272,9 +301,17 @@ class Workload:
                                        self.tables, self.lens, cfg.scale, self.ws, stream=stream)
 
     def step(self, stream=None):
-        """Every layer, in order."""
+        """The step as the library runs it for inputs that are all present: every layer in one launch."""
+        self.layers_call(stream=stream)
+
+    def step_per_layer(self, stream=None):
+        """The step as a transformer forward runs it: one launch per layer, in order."""
         for layer in range(self.cfg.n_layers):
             self.layer(layer, stream)
+
+    def free(self):
+        for name in ("k_all", "v_all", "k", "v", "q", "k_new", "v_new", "out", "ws", "ws_all"):
+            setattr(self, name, None)
 
 
 def capture(fn):
@@ -327,30 +364,6 @@ def time_replays_redraw(graph, wl, steps, world):
     return total_ms / steps, total_bytes
 
 
-def decode_kernel_duration_ms(wl, reps=5):
-    """Average duration of one decode launch (with the fused append when the step uses it), by CUDA events on
-    its stream, cycling through the layers."""
-    pkv, cfg = wl.pkv, wl.cfg
-    stream = torch.cuda.current_stream()
-    evs = []
-    for _ in range(reps):
-        for layer in range(cfg.n_layers):
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            if wl.fused:  # rewriting this step's token is idempotent
-                pkv.paged_attention_decode_append(wl.out[layer], wl.q[layer], wl.k_new[layer], wl.v_new[layer],
-                                                  wl.k[layer], wl.v[layer], wl.slots, wl.tables, wl.lens,
-                                                  cfg.scale, wl.ws, stream=stream)
-            else:
-                pkv.paged_attention_decode(wl.out[layer], wl.q[layer], wl.k[layer], wl.v[layer], wl.tables,
-                                           wl.lens, cfg.scale, wl.ws, stream=stream)
-            b.record(stream)
-            evs.append((a, b))
-    torch.cuda.synchronize()
-    times = [a.elapsed_time(b) for a, b in evs]
-    return sum(times) / len(times), len(times)
-
-
 def block_moves_measure(wl, peak, reps=10):
     """Whole-block moves over every layer's K and V cache, one launch per call: swap-out staging (gather) and
     swap-in (scatter) of the blocks of a tenth of the batch's sequences, and copy-on-write copies of as many of
@@ -376,8 +389,8 @@ def block_moves_measure(wl, peak, reps=10):
     ops = {"gather": (lambda: pkv.kv_cache_gather_blocks(staged, caches, ids_d, error_flag=flag), len(ids)),
            "scatter": (lambda: pkv.kv_cache_scatter_blocks(caches, staged, ids_d, error_flag=flag), len(ids)),
            "copy": (lambda: pkv.kv_cache_copy_blocks(caches, src_d, dst_d, error_flag=flag), n_copy)}
-    res = {"blocks_swapped": len(ids), "blocks_copied": n_copy, "tensors": len(caches), "bytes_per_block": blk_bytes,
-           "timing": "CUDA events, mean of %d launches after 2 warm-up launches" % reps}
+    res = {"workload": cfg.name, "blocks_swapped": len(ids), "blocks_copied": n_copy, "tensors": len(caches),
+           "bytes_per_block": blk_bytes, "timing": "CUDA events, mean of %d launches after 2 warm-up launches" % reps}
     stream = torch.cuda.current_stream()
     for name, (fn, n) in ops.items():
         if n == 0:
@@ -473,10 +486,10 @@ def pinned_near(tensors, device_index: int):
 
 def e2e_measure(wl, steps, warmup, world, chunks=4):
     """The same step through the C ABI with host buffers: every step copies its inputs from pinned host
-    memory and its outputs back. The copies run on two side streams, pipelined with the layers: the tables,
-    lengths and slots, then q, k_new and v_new in `chunks` groups of layers, each ahead of its first launch;
-    each layer's output is copied back while later layers run -- as a serving loop would. One CUDA graph.
-    The host buffers are pinned pages on the GPU's NUMA node."""
+    memory and its outputs back. The layers go in `chunks` groups, each one multi-layer launch: the copies
+    run on two side streams, pipelined with the groups (the tables, lengths and slots, then q, k_new and v_new
+    of each group ahead of its launch; each group's output copied back while later groups run). One CUDA
+    graph. The host buffers are pinned pages on the GPU's NUMA node."""
     cfg = wl.cfg
     L = cfg.n_layers
     dev_index = wl.q.device.index or 0
@@ -489,9 +502,11 @@ def e2e_measure(wl, steps, warmup, world, chunks=4):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = host_out.numel() * host_out.element_size()
     h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+    chunks = max(1, min(chunks, L))
     per = -(-L // chunks)
-    ev_in = [torch.cuda.Event() for _ in range(chunks)]
-    ev_done = [torch.cuda.Event() for _ in range(L)]
+    groups = [(lo, min(L, lo + per)) for lo in range(0, L, per)]
+    ev_in = [torch.cuda.Event() for _ in groups]
+    ev_done = [torch.cuda.Event() for _ in groups]
 
     def one():
         main = torch.cuda.current_stream()
@@ -500,19 +515,17 @@ def e2e_measure(wl, steps, warmup, world, chunks=4):
         with torch.cuda.stream(h2d_stream):
             for k in step_in:
                 step_in[k].copy_(host[k], non_blocking=True)
-            for c in range(chunks):
-                lo, hi = c * per, min(L, (c + 1) * per)
+            for g, (lo, hi) in enumerate(groups):
                 for k in layer_in:
                     layer_in[k][lo:hi].copy_(host[k][lo:hi], non_blocking=True)
-                ev_in[c].record(h2d_stream)
-        for layer in range(L):
-            if layer % per == 0:
-                main.wait_event(ev_in[layer // per])
-            wl.layer(layer)
-            ev_done[layer].record(main)
+                ev_in[g].record(h2d_stream)
+        for g, (lo, hi) in enumerate(groups):
+            main.wait_event(ev_in[g])
+            wl.layers_call(lo, hi)
+            ev_done[g].record(main)
             with torch.cuda.stream(d2h_stream):
-                d2h_stream.wait_event(ev_done[layer])
-                host_out[layer].copy_(wl.out[layer], non_blocking=True)
+                d2h_stream.wait_event(ev_done[g])
+                host_out[lo:hi].copy_(wl.out[lo:hi], non_blocking=True)
         main.wait_stream(h2d_stream)
         main.wait_stream(d2h_stream)
 
@@ -520,28 +533,45 @@ def e2e_measure(wl, steps, warmup, world, chunks=4):
     for _ in range(warmup):
         g.replay()
     ms = time_replays(g, steps, world)
-    return ms, h2d, d2h
+    del g
+    return ms, h2d, d2h, len(groups)
 
 
 class OracleSampler:
-    """The float64 oracle on whole layers of the workload (append + attention), on this host's cores."""
+    """The float64 oracle on whole layers (append + attention) of a bounded sample of the workload, on this
+    host's cores: all sequences of one layer when that layer's KV is at most `max_layer_bytes`, else the first
+    few sequences of a batch drawn with the workload's length law, block placement and shapes."""
 
-    def __init__(self, cfg, layout):
+    def __init__(self, cfg, layout=None, max_layer_bytes=400e6):
         import oracle
-        self.oracle, self.cfg, self.layout = oracle, cfg, layout
+        self.oracle, self.cfg = oracle, cfg
+        if layout is None:
+            layout = workloads.draw_layout(cfg)
+        lens = [int(c) for c in layout.context_lens]
+        full_kv = layer_bytes(cfg, lens, layout.shares_prefix.tolist(), unique_prefix=True)["kv"]
+        if full_kv > max_layer_bytes:
+            nb = max(1, int(cfg.batch * max_layer_bytes / full_kv))
+            layout = workloads.draw_layout(replace(cfg, batch=nb, pool_blocks=0))
+            self.what = f"{nb} of the {cfg.batch} sequences (a batch of {nb} drawn with the workload's shapes and " \
+                        f"length law)"
+        else:
+            self.what = f"all {cfg.batch} sequences"
+        self.layout = layout
+        self.batch = len(layout.context_lens)
         gen = workloads.device_generator(cfg.seed, "cpu")
         self.k, self.v = workloads.make_layer_cache(layout.num_blocks, cfg.Hkv, cfg.D, gen, "cpu", cfg.torch_dtype)
-        q, kn, vn = workloads.make_step_inputs(cfg, gen, "cpu", n_layers=1)
+        sub = replace(cfg, batch=self.batch)
+        q, kn, vn = workloads.make_step_inputs(sub, gen, "cpu", n_layers=1)
         self.q, self.kn, self.vn = q[0], kn[0], vn[0]
         self.slots = layout.slot_mapping().numpy()
         self.tables = layout.block_tables.numpy()
         self.lens = layout.context_lens.numpy()
         lens = [int(c) for c in self.lens]
-        self.layer_bytes = layer_bytes(cfg, lens, layout.shares_prefix.tolist(), unique_prefix=True)["total"]
+        self.layer_bytes = layer_bytes(sub, lens, layout.shares_prefix.tolist(), unique_prefix=True)["total"]
         self.cores = oracle.num_threads()
 
     def run(self, seconds: float):
-        """Whole layers until `seconds` have passed (at least one). Returns (bytes, seconds, seq-layers)."""
+        """Whole layers until `seconds` have passed (at least one). Returns (bytes, seconds, seq-layers, layers)."""
         done_bytes, done_layers, t0 = 0, 0, time.perf_counter()
         while True:
             k2, v2 = self.oracle.kv_cache_append(self.k, self.v, self.kn, self.vn, self.slots)
@@ -551,7 +581,24 @@ class OracleSampler:
             done_layers += 1
             if time.perf_counter() - t0 >= seconds:
                 break
-        return done_bytes, time.perf_counter() - t0, done_layers * self.cfg.batch
+        return done_bytes, time.perf_counter() - t0, done_layers * self.batch, done_layers
+
+
+def config_record(cfg, layout, world):
+    """The `config` object of both arms' lines: the workload's shapes and the bytes of its first step."""
+    lens = [int(c) for c in layout.context_lens]
+    share = layout.shares_prefix.tolist()
+    lb_logical = layer_bytes(cfg, lens, share, unique_prefix=False)
+    lb_unique = layer_bytes(cfg, lens, share, unique_prefix=True)
+    return {"workload": cfg.name, "config_id": cfg.cid, "elem": cfg.elem, "layers": cfg.n_layers,
+            "batch": cfg.batch, "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "block_tokens": 16,
+            "mean_context": round(sum(lens) / len(lens), 1),
+            "kv_bytes_per_step": lb_unique["kv"] * cfg.n_layers,
+            "kv_bytes_per_step_logical": lb_logical["kv"] * cfg.n_layers,
+            "algorithmic_bytes_per_step": lb_unique["total"] * cfg.n_layers,
+            "l2": "inputs larger than L2: every step reads all layers' distinct caches "
+                  f"({lb_unique['kv'] * cfg.n_layers / 1e9:.2f} GB of KV vs 126 MB L2)",
+            "parallelism": f"replicas x{world}"}
 
 
 def run_profile_step(args, cfg, device):
@@ -559,20 +606,130 @@ def run_profile_step(args, cfg, device):
     import paged_kv_cache_470_b200 as pkv
     wl = Workload(cfg, device)
     wl.fused = not args.separate_append
-    graph = capture(wl.step)
+    graph = capture(wl.step_per_layer if args.per_layer else wl.step)
     for _ in range(args.warmup + args.steps):
         graph.replay()
     torch.cuda.synchronize()
+    ws = wl.ws if args.per_layer else wl.ws_all
     print(json.dumps({"profile_step": cfg.name, "layers": cfg.n_layers, "replays": args.warmup + args.steps,
-                      "status": pkv.read_status(wl.ws)}), flush=True)
+                      "per_layer": bool(args.per_layer), "status": pkv.read_status(ws)}), flush=True)
 
 
-def pick_config(args):
-    """The workload named by --config, with --layers and --dtype applied."""
+def pick_config(args, cid=None):
+    """The workload named by --config (or cid), with --layers and --dtype applied."""
     over = {"elem": args.dtype}
     if args.layers:
         over["n_layers"] = args.layers
-    return workloads.small_config(args.config, **over)
+    return workloads.small_config(args.config if cid is None else cid, **over)
+
+
+def timed_windows(graph, wl, steps, world, min_seconds):
+    """Time `steps` replays of the step's graph (the measurement), then repeat windows of the same length until
+    about `min_seconds` of replays have run, so that the clock sampler sees the kernels at work. Every rank runs
+    the same number of windows (the largest any rank needs). Returns (first window's ms per step, all windows'
+    ms per step, bytes per step of the first window or None)."""
+    redraw = wl.cfg.redraw_fraction > 0
+
+    def window():
+        if redraw:
+            ms, tb = time_replays_redraw(graph, wl, steps, world)
+            return ms, tb // steps
+        return time_replays(graph, steps, world), None
+
+    first, step_bytes = window()
+    more = max(0, math.ceil(min_seconds * 1e3 / max(first * steps, 1e-3)) - 1)
+    more = min(199, int(dist_max(float(more), world)))
+    windows = [first] + [window()[0] for _ in range(more)]
+    return first, windows, step_bytes
+
+
+def roofline(step_bytes, ms, launches, peak, peak_kind, traffic, how):
+    kern_ms = ms / launches
+    achieved = step_bytes / launches / (kern_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "algorithmic_bytes_per_launch": step_bytes / launches, "kernel_ms": round(kern_ms, 5),
+            "kernel_ms_how": how, "peak_kind": f"{peak_kind} HBM copy bandwidth",
+            "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)}
+
+
+def measure_config(args, cfg, device, world, rank, headline):
+    """One workload: the multi-layer step (the line's figures) and the per-layer step beside it, each a CUDA
+    graph timed over --steps replays with CUDA events; clocks sampled while they run. With `headline`, also the
+    e2e figure, the block moves and the workload object handed back for the CPU baseline."""
+    import paged_kv_cache_470_b200 as pkv
+    wl = Workload(cfg, device, rank)
+    wl.fused = not args.separate_append
+    peak, peak_kind = measured_peak()
+    cfg_rec = config_record(cfg, wl.layout, world)
+    step_bytes0 = cfg_rec["algorithmic_bytes_per_step"]
+    combine = pkv.get_option(pkv.KV_OPT_COMBINE) == 1
+    res = {}
+    for name, fn, launches in (("layers", wl.step, 1 + combine),
+                               ("per_layer", wl.step_per_layer,
+                                cfg.n_layers * ((1 if wl.fused else 2) + combine))):
+        graph = capture(fn)
+        for _ in range(args.warmup):
+            graph.replay()
+        torch.cuda.synchronize()
+        with ClockSampler(device.index or 0, period_s=0.002) as clk:
+            ms, windows, tb = timed_windows(graph, wl, args.steps, world, args.clock_window_s)
+        ms = dist_max(ms, world)
+        step_bytes = tb if tb is not None else step_bytes0
+        status = pkv.read_status(wl.ws_all if name == "layers" else wl.ws)
+        del graph
+        res[name] = {"ms": ms, "windows": windows, "step_bytes": step_bytes, "clocks": clk.summary(),
+                     "status": status, "launches": launches}
+    ml, pl = res["layers"], res["per_layer"]
+    traffic = profiled_traffic(cfg)
+    kernel_of_step = (combine == 0)
+    how_ml = ("timed step / 1 (the step is one launch of the multi-layer kernel)" if kernel_of_step else
+              "timed step / launches (decode and combine kernels)")
+    rec = {
+        "ms_per_step": round(ml["ms"], 5),
+        "value": round(ml["step_bytes"] * world / (ml["ms"] * 1e-3) / 1e9, 2),
+        "unit": "GB/s",
+        "seq_layers_per_s": round(cfg.batch * cfg.n_layers * world / (ml["ms"] * 1e-3), 1),
+        "pct_of_nominal_8TBs": round(100 * ml["step_bytes"] / (ml["ms"] * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 2),
+        "pct_of_measured_hbm": round(100 * ml["step_bytes"] / (ml["ms"] * 1e-3) / 1e9 / peak, 2),
+        "config": cfg_rec,
+        "roofline": roofline(ml["step_bytes"], ml["ms"], ml["launches"], peak, peak_kind, traffic, how_ml),
+        "windows_ms_per_step": {"n": len(ml["windows"]), "median": round(statistics.median(ml["windows"]), 5),
+                                "min": round(min(ml["windows"]), 5), "max": round(max(ml["windows"]), 5)},
+        "clocks": ml["clocks"],
+        "device_status": ml["status"],
+        "per_layer": {
+            "api": ("paged_attention_decode_append" if wl.fused else "kv_cache_append + paged_attention_decode")
+                   + " per layer, in a CUDA graph with programmatic dependent launch",
+            "ms_per_step": round(pl["ms"], 5),
+            "value": round(pl["step_bytes"] * world / (pl["ms"] * 1e-3) / 1e9, 2),
+            "pct_of_nominal_8TBs": round(100 * pl["step_bytes"] / (pl["ms"] * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 2),
+            "roofline": roofline(pl["step_bytes"], pl["ms"], pl["launches"], peak, peak_kind,
+                                 profiled_traffic(cfg, "per_layer") if wl.fused and not combine else None,
+                                 "timed step / launches per step (the step holds only these launches)"),
+            "windows_ms_per_step": {"n": len(pl["windows"]), "median": round(statistics.median(pl["windows"]), 5)},
+            "clocks": pl["clocks"],
+            "device_status": pl["status"],
+        },
+        "gpu_launches": ml["launches"] * args.steps,
+    }
+    if cfg.redraw_fraction > 0:
+        rec["timing_note"] = "10% of the batch re-drawn through the block pool before each step (untimed)"
+    if headline:
+        e2e_ms, h2d, d2h, groups = e2e_measure(wl, max(args.steps // 4, 3), args.warmup, world)
+        e2e_ms = dist_max(e2e_ms, world)
+        rec["e2e"] = {"value": round(ml["step_bytes"] * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                      "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                      "api": f"paged_attention_decode_layers over {groups} groups of layers; inputs copied "
+                             "host-to-device on a side stream ahead of each group's launch, each group's output "
+                             "copied back on another behind it, all in one CUDA graph; pinned host buffers on "
+                             "the GPU's NUMA node"}
+        rec["block_moves"] = block_moves_measure(wl, peak)
+    wl.free()
+    del wl
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_ours(args, world, rank, local):
@@ -589,115 +746,67 @@ def run_ours(args, world, rank, local):
         pkv.set_option(pkv.KV_OPT_HEAD_GROUP, args.head_group)
     if args.item_cost:
         pkv.set_option(pkv.KV_OPT_ITEM_COST, args.item_cost)
+    if args.l2_policy:
+        pkv.set_option(pkv.KV_OPT_L2_POLICY, {"first": 1, "normal": 2, "last": 3}[args.l2_policy])
     if args.profile_step:
         return run_profile_step(args, cfg, device)
     if args.profile_prefill:
         r = prefill_measure(pkv, device, cfg.elem, reps=args.steps, keys=(args.profile_prefill,))
         print(json.dumps(r), flush=True)
         return
-    wl = Workload(cfg, device, rank)
-    wl.fused = not args.separate_append
-    lens = [int(c) for c in wl.layout.context_lens]
-    share = wl.layout.shares_prefix.tolist()
-    lb_logical = layer_bytes(cfg, lens, share, unique_prefix=False)
-    lb_unique = layer_bytes(cfg, lens, share, unique_prefix=True)
-    step_bytes = lb_unique["total"] * cfg.n_layers
-
-    graph = capture(wl.step)
-    for _ in range(args.warmup):
-        graph.replay()
-    torch.cuda.synchronize()
-    redraw = cfg.redraw_fraction > 0
-    with ClockSampler(device.index or 0) as clk:
-        if redraw:
-            ms, timed_bytes = time_replays_redraw(graph, wl, args.steps, world)
-            step_bytes = timed_bytes // args.steps
-        else:
-            ms = time_replays(graph, args.steps, world)
-    ms = dist_max(ms, world)
-    status = pkv.read_status(wl.ws)
-
-    # the decode kernel alone, for the roofline (on the batch as it stands now)
-    lens = [int(c) for c in wl.layout.context_lens]
-    lb_unique = layer_bytes(cfg, lens, wl.layout.shares_prefix.tolist(), unique_prefix=True)
-    lb_logical = layer_bytes(cfg, lens, wl.layout.shares_prefix.tolist(), unique_prefix=False)
-    iso_ms, n_launch = decode_kernel_duration_ms(wl)
-    iso_ms = dist_max(iso_ms, world)
-    peak, peak_kind = measured_peak()
-    kern_bytes = lb_unique["decode_kernel"] + (lb_unique["append"] if wl.fused else 0)
-    if wl.fused and not args.combine_kernel:
-        # the timed step is nothing but n_layers launches of the decode kernel
-        kern_ms = ms / cfg.n_layers
-        kern_bytes = step_bytes / cfg.n_layers
-        kern_how = "timed step / launches per step (the step holds only this kernel)"
-    else:
-        kern_ms = iso_ms
-        kern_how = "CUDA events around single launches, layers cycled"
-    achieved = kern_bytes / (kern_ms * 1e-3) / 1e9
-    traffic = profiled_traffic(cfg)
-
-    e2e_ms, h2d, d2h = e2e_measure(wl, max(args.steps // 4, 3), args.warmup, world)
-    moves = block_moves_measure(wl, peak)
-    prefill = prefill_measure(pkv, device, cfg.elem)
-    e2e_ms = dist_max(e2e_ms, world)
+    torch.cuda.nvtx.range_push(f"workload {cfg.cid}")
+    head = measure_config(args, cfg, device, world, rank, headline=True)
+    torch.cuda.nvtx.range_pop()
+    per_config = {}
+    others = [] if args.no_per_config else [int(c) for c in args.per_config.split(",") if c.strip()]
+    for cid in others:
+        if cid == cfg.cid:
+            continue
+        torch.cuda.nvtx.range_push(f"workload {cid}")
+        per_config[str(cid)] = measure_config(args, pick_config(args, cid), device, world, rank, headline=False)
+        torch.cuda.nvtx.range_pop()
+    prefill = prefill_measure(pkv, device, cfg.elem) if not args.no_prefill else None
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        sampler = OracleSampler(cfg, wl.layout)
-        b, s, nsl = sampler.run(args.cpu_seconds)
+        sampler = OracleSampler(cfg)
+        b, s, nsl, layers = sampler.run(args.cpu_seconds)
         cpu = {"value": round(b / s / 1e9, 4), "unit": "GB/s", "cores": sampler.cores, "kind": "oracle",
                "seq_layers_per_s": round(nsl / s, 2),
-               "sample": f"{nsl // cfg.batch} layer(s) of this workload (all {cfg.batch} sequences, append + "
-                         f"attention) in float64 on the host, {s:.1f} s"}
+               "sample": f"{layers} layer(s) of this workload, each {sampler.what}, append + attention, in "
+                         f"float64 on the host, {s:.1f} s"}
 
-    value = step_bytes * world / (ms * 1e-3) / 1e9
     line = {
         "metric": "decode-attention achieved HBM GB/s (% of B200 peak); seq·layers/sec per step",
-        "value": round(value, 2),
+        "value": head["value"],
         "unit": "GB/s",
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": round(ms, 5),
+        "ms_per_step": head["ms_per_step"],
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": cfg.elem,
         "data": "synthetic",
-        "seq_layers_per_s": round(cfg.batch * cfg.n_layers * world / (ms * 1e-3), 1),
-        "pct_of_nominal_8TBs": round(100 * value / world / NOMINAL_HBM_GBS, 2),
-        "pct_of_measured_hbm": round(100 * value / world / peak, 2),
-        "config": {"workload": cfg.name, "config_id": cfg.cid, "elem": cfg.elem, "layers": cfg.n_layers, "batch": cfg.batch,
-                   "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "block_tokens": 16,
-                   "mean_context": round(sum(lens) / len(lens), 1),
-                   "kv_bytes_per_step": lb_unique["kv"] * cfg.n_layers,
-                   "kv_bytes_per_step_logical": lb_logical["kv"] * cfg.n_layers,
-                   "algorithmic_bytes_per_step": step_bytes,
-                   "l2": "inputs larger than L2: every step reads all layers' distinct caches "
-                         f"({lb_unique['kv'] * cfg.n_layers / 1e9:.2f} GB of KV vs 126 MB L2)",
-                   "timing": "CUDA-graph replay of the whole step, CUDA events, max over ranks"
-                             + ("; 10% of the batch re-drawn through the block pool before each step (untimed)"
-                                if redraw else ""),
-                   "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "algorithmic_bytes_per_launch": kern_bytes, "kernel_ms": round(kern_ms, 5),
-                     "kernel_ms_how": kern_how,
-                     "kernel_ms_single_launch": round(iso_ms, 5), "single_launches_timed": n_launch,
-                     "peak_kind": f"{peak_kind} HBM copy bandwidth",
-                     "frac_of_nominal_8TBs": round(achieved / NOMINAL_HBM_GBS, 4)},
-        "e2e": {"value": round(step_bytes * world / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
-                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "api": ("paged_attention_decode_append" if wl.fused else "kv_cache_append + paged_attention_decode")
-                       + " per layer; inputs copied host-to-device on a side stream in 4 groups of layers ahead "
-                         "of their launches, each layer's output copied back on another behind it, all in one "
-                         "CUDA graph; pinned host buffers on the GPU's NUMA node"},
-        "gpu_launches": ((1 if wl.fused else 2) + (pkv.get_option(pkv.KV_OPT_COMBINE) == 1))
-                        * cfg.n_layers * args.steps,
-        "clocks": clk.summary(),
-        "device_status": status,
+        "seq_layers_per_s": head["seq_layers_per_s"],
+        "pct_of_nominal_8TBs": head["pct_of_nominal_8TBs"],
+        "pct_of_measured_hbm": head["pct_of_measured_hbm"],
+        "config": head["config"],
+        "timing": "CUDA-graph replay of the whole step (one multi-layer launch), CUDA events, max over ranks; "
+                  "the first window of --steps replays; further windows of the same length only to give the "
+                  "clock sampler time (their spread is windows_ms_per_step)"
+                  + ("; " + head["timing_note"] if "timing_note" in head else ""),
+        "roofline": head["roofline"],
+        "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+        "windows_ms_per_step": head["windows_ms_per_step"],
+        "device_status": head["device_status"],
+        "per_layer": head["per_layer"],
+        "per_config": per_config,
         "cpu_baseline": cpu,
-        "block_moves": moves,
+        "block_moves": head["block_moves"],
         "prefill": prefill,
     }
     if rank == 0:
@@ -718,17 +827,17 @@ def run_reference(args, world, rank):
         sampler.run(0.0)
     b_all = s_all = n_all = 0
     for _ in range(args.steps):
-        b, s, n = sampler.run(per_step)
+        b, s, n, _ = sampler.run(per_step)
         b_all, s_all, n_all = b_all + b, s_all + s, n_all + n
     value = b_all / s_all / 1e9
-    sample = (f"each step: whole layers of this workload (append + attention, all {cfg.batch} sequences) "
-              f"for about {per_step:.2f} s")
+    sample = (f"each step: whole layers of this workload ({sampler.what}, append + attention) for about "
+              f"{per_step:.2f} s")
     line = {"impl": "reference", "metric": "decode-attention achieved HBM GB/s (% of B200 peak); seq·layers/sec per step",
             "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1e3 * s_all / args.steps, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "seq_layers_per_s": round(n_all / s_all, 2),
-            "config": {"workload": cfg.name, "config_id": cfg.cid, "elem": cfg.elem},
+            "config": config_record(cfg, layout, world),
             "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -738,9 +847,15 @@ def run_reference(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--config", type=int, default=2, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=4, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--per-config", default="2,3,5",
+                    help="the other workloads measured in the same run (comma-separated ids)")
+    ap.add_argument("--no-per-config", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--clock-window-s", type=float, default=0.25,
+                    help="repeat the timed window until this many seconds of replays ran (clock samples)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--compute", choices=["tensor", "cuda"], default=None)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -748,6 +863,7 @@ def main(argv=None):
     ap.add_argument("--reference-budget", type=float, default=120.0)
     ap.add_argument("--layers", type=int, default=0, help="use only this many layers (profiling a smaller case)")
     ap.add_argument("--profile-step", action="store_true", help="only replay the step graph (for ncu)")
+    ap.add_argument("--per-layer", action="store_true", help="with --profile-step: the per-layer step")
     ap.add_argument("--profile-prefill", choices=sorted(workloads.PREFILL_CONFIGS), default=None,
                     help="only run the chunked-prefill workload: 3 warm-up and --steps timed launches (for ncu)")
     ap.add_argument("--grid", type=int, default=0, help="decode CTAs per launch (0: one per SM)")
@@ -755,9 +871,11 @@ def main(argv=None):
     ap.add_argument("--head-group", type=int, default=0, help="kv heads per work unit (0: auto)")
     ap.add_argument("--item-cost", type=int, default=0,
                     help="work positions charged per work item when dividing work between CTAs (0 auto, -1 none)")
+    ap.add_argument("--l2-policy", choices=["first", "normal", "last"], default=None,
+                    help="L2 priority of the decode kernels' K/V tile loads (default: the library's)")
     ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16", help="element type of q, K, V and out")
     ap.add_argument("--separate-append", action="store_true",
-                    help="append with kv_cache_append, then paged_attention_decode (two launches per layer)")
+                    help="per-layer step: append with kv_cache_append, then paged_attention_decode")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

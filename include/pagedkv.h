@@ -7,6 +7,8 @@
  *   paged_attention_decode  out = softmax(scale * q K^T) V per query head,
  *                           reading K/V through per-sequence block tables
  *   paged_attention_decode_append   the two above in one launch
+ *   paged_attention_decode_layers   the same over several layers of one step
+ *                           in one launch
  *   paged_attention_prefill chunked prefill: a chunk of query tokens per
  *                           sequence, causal over the same cache
  *   kv_cache_copy_blocks, kv_cache_gather_blocks, kv_cache_scatter_blocks
@@ -197,6 +199,45 @@ KV_API kv_status paged_attention_decode_append(void *out, const void *q,
                                                kv_stream_t stream);
 
 /*
+ * Several layers of one decode step in one launch ("Module 23: Serving",
+ * section 23.1, equation Memory_KV: every layer keeps its own K and V for every
+ * token, so a step reads num_layers caches through the same block tables).
+ * For l in [0, num_layers) it gives the result of
+ *   paged_attention_decode_append(out + l*B*Hq*D, q + l*B*Hq*D,
+ *       k_new + l*B*Hkv*D, v_new + l*B*Hkv*D,
+ *       k_cache + l*cache_layer_stride, v_cache + l*cache_layer_stride, ...)
+ * (or of paged_attention_decode when k_new, v_new and slot_mapping are all
+ * NULL), with the same block_tables, context_lens and slot_mapping for every
+ * layer. Offsets are in elements: q and out are [num_layers][B][Hq][D], k_new
+ * and v_new [num_layers][B][Hkv][D], all contiguous; layer l's caches start
+ * cache_layer_stride elements after layer l-1's (a stacked
+ * [num_layers][num_blocks][16][Hkv][D] pool has cache_layer_stride =
+ * num_blocks*16*Hkv*D; any larger multiple of 8 up to 2^38 is accepted, the
+ * same for K and V). The work of all layers is divided between the CTAs as one
+ * sequence, so no layer waits for the previous one's split-K merges: a step
+ * whose queries are all available at once (attention of every layer from the
+ * same inputs, as a benchmark step is) pays the per-launch start-up and tail
+ * once. In a transformer forward, layer l+1's q is computed from layer l's
+ * output, so such a caller launches per layer instead.
+ * workspace_bytes >= paged_attention_workspace_size_layers(B, Hq, Hkv, D,
+ * num_layers); the other requirements, checks and the status word are those of
+ * paged_attention_decode_append (a bad slot is reported once, not per layer).
+ * num_layers >= 1; num_layers = 1 equals the single-layer calls.
+ */
+KV_API size_t paged_attention_workspace_size_layers(int B, int Hq, int Hkv, int D, int num_layers);
+KV_API kv_status paged_attention_decode_layers(void *out, const void *q,
+                                               const void *k_new, const void *v_new,
+                                               void *k_cache, void *v_cache,
+                                               size_t cache_layer_stride, int num_layers,
+                                               const int64_t *slot_mapping,
+                                               const int32_t *block_tables, int max_blocks_per_seq,
+                                               const int32_t *context_lens, int B,
+                                               int num_blocks, int Hq, int Hkv, int D,
+                                               float scale, int dtype,
+                                               void *workspace, size_t workspace_bytes,
+                                               kv_stream_t stream);
+
+/*
  * The same decode as paged_attention_decode, for callers that cannot allocate
  * device memory (for example a plugin inside a host program that owns every
  * device allocation, or code that must not trigger cudaMalloc's implicit
@@ -209,11 +250,15 @@ KV_API kv_status paged_attention_decode_append(void *out, const void *q,
  * Sizes whose scratch (paged_attention_workspace_size) exceeds the array are
  * rejected with KV_ERR_ARG. The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress, with that device current); make that
- * first call before any stream capture. Each call clears the array's status
- * word and counters on `stream` before the kernel. All calls share the one
- * array: calls that can overlap on the GPU (other streams, other threads)
- * race and give wrong results; serialise them. Device data errors are
- * guarded as in paged_attention_decode but cannot be read back here.
+ * first call before any stream capture. The address is looked up again when
+ * the device's current context has changed since; it cannot tell a context
+ * that cudaDeviceReset destroyed from a new one at the same handle, so do not
+ * call it across a cudaDeviceReset. Every check runs before anything is
+ * enqueued; a call that goes ahead clears the array's status word and counters
+ * on `stream`, then launches the kernel. All calls share the one array: calls
+ * that can overlap on the GPU (other streams, other threads) race and give
+ * wrong results; serialise them. Device data errors are guarded as in
+ * paged_attention_decode but cannot be read back here.
  */
 #define KV_NOALLOC_SCRATCH_BYTES (16u << 20)
 KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
@@ -292,6 +337,15 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     softmax warp waits about 30 microseconds before it hands
  *                     over P of the first tile, so the other warps run a tile
  *                     ahead of it. The output must not change.
+ *   KV_OPT_OUT_F32:   debug switch for checking the arithmetic, 0 (default)
+ *                     off; 1: `out` of the decode calls and of
+ *                     paged_attention_prefill holds fp32 numbers (4 bytes
+ *                     each, same shape, 16-byte aligned), the normalised
+ *                     result before any rounding to the element type. The
+ *                     other arguments keep their element type.
+ *   KV_OPT_L2_POLICY: L2 priority of the decode kernels' K/V tile loads: 0
+ *                     auto (evict first), 1 evict first, 2 evict normal,
+ *                     3 evict last.
  * Kernels are launched with programmatic dependent launch. q, k_new, v_new,
  * the caches, the workspace and out are touched only after the previous kernel
  * in the stream has completed; block_tables and context_lens are read before
@@ -308,6 +362,8 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
 #define KV_OPT_PREFILL_PATH 8
 #define KV_OPT_TEST_DROP_LOAD 9
 #define KV_OPT_TEST_SLOW_SOFTMAX 10
+#define KV_OPT_OUT_F32 11
+#define KV_OPT_L2_POLICY 12
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

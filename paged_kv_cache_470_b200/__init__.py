@@ -2,8 +2,11 @@
 
 Argument marshalling only: every step of a decode (append, attention, split-K
 merge) runs in the library's CUDA kernels, and the block pool runs in its C++
-code. PyTorch supplies device memory and the stream. There is no fallback: if
-the shared library is missing, importing this package raises ImportError.
+code. PyTorch supplies device memory and the stream. There is no fallback: the
+library is loaded by the first call that needs it (or by ``load()``), and if
+the shared library is missing that call raises ImportError. Importing the
+package alone maps no library, so that its seeded input generator
+(``workloads``) can serve code that must not load it.
 
 Build it with ``python paged_kv_cache_470_b200/build.py``.
 """
@@ -17,10 +20,6 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
 
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python paged_kv_cache_470_b200/build.py`")
-_lib = ctypes.CDLL(LIB_PATH)
-
 KV_OK, KV_ERR_ARG, KV_ERR_OOM, KV_ERR_STATE, KV_ERR_CUDA = 0, -1, -2, -3, -4
 KV_DTYPE_BF16, KV_DTYPE_FP16 = 0, 1
 BLOCK_TOKENS = 16
@@ -29,6 +28,8 @@ KV_OPT_COMPUTE, KV_OPT_COMBINE, KV_OPT_GRID, KV_OPT_MIN_CHUNK, KV_OPT_PRODUCER_L
     1, 2, 3, 4, 5, 6)
 KV_OPT_ITEM_COST, KV_OPT_PREFILL_PATH, KV_OPT_TEST_DROP_LOAD = 7, 8, 9
 KV_OPT_TEST_SLOW_SOFTMAX = 10
+KV_OPT_OUT_F32 = 11
+KV_OPT_L2_POLICY = 12
 COMPUTE_AUTO, COMPUTE_TENSOR_CORES, COMPUTE_CUDA_CORES = 0, 1, 2
 
 _P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
@@ -42,6 +43,9 @@ _sig = {
                                            _I, _P, _SZ, _P]),
     "paged_attention_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, ctypes.c_float, _I,
                                             _P]),
+    "paged_attention_workspace_size_layers": (_SZ, [_I, _I, _I, _I, _I]),
+    "paged_attention_decode_layers": (_I, [_P, _P, _P, _P, _P, _P, _SZ, _I, _P, _P, _I, _P, _I, _I, _I, _I, _I,
+                                           ctypes.c_float, _I, _P, _SZ, _P]),
     "paged_attention_read_status": (_I, [_P, _P, _I, _P]),
     "paged_attention_prefill": (_I, [_P, _P, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I, _P,
                                      _P]),
@@ -62,12 +66,33 @@ _sig = {
     "kv_cache_gather_blocks": (_I, [_P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P]),
     "kv_cache_scatter_blocks": (_I, [_P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P]),
 }
-for _name, (_res, _args) in _sig.items():
-    _f = getattr(_lib, _name)
-    _f.restype = _res
-    _f.argtypes = _args
-
 EXPORTED = tuple(_sig)
+_handle = None
+
+
+def load() -> ctypes.CDLL:
+    """The library, loaded on first use with every call's signature set; ImportError if it is missing."""
+    global _handle
+    if _handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python paged_kv_cache_470_b200/build.py`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _sig.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _handle = lib
+    return _handle
+
+
+class _Lib:
+    """Attribute access loads the library (so `_lib.call(...)` reads as a direct call)."""
+
+    def __getattr__(self, name):
+        return getattr(load(), name)
+
+
+_lib = _Lib()
 
 
 class KVError(RuntimeError):
@@ -128,9 +153,22 @@ def workspace_size(B: int, Hq: int, Hkv: int, D: int) -> int:
     return int(n)
 
 
-def make_workspace(B: int, Hq: int, Hkv: int, D: int, device=None) -> torch.Tensor:
-    """A zeroed workspace (uint8) sized for these shapes on the current device."""
-    return torch.zeros(workspace_size(B, Hq, Hkv, D), dtype=torch.uint8, device=device or "cuda")
+def workspace_size_layers(B: int, Hq: int, Hkv: int, D: int, num_layers: int) -> int:
+    n = _lib.paged_attention_workspace_size_layers(B, Hq, Hkv, D, num_layers)
+    if n == 0:
+        raise KVError("paged_attention_workspace_size_layers", KV_ERR_ARG)
+    return int(n)
+
+
+def make_workspace(B: int, Hq: int, Hkv: int, D: int, device=None, num_layers: int = 1) -> torch.Tensor:
+    """A zeroed workspace (uint8) sized for these shapes (and layers per launch) on the current device."""
+    return torch.zeros(workspace_size_layers(B, Hq, Hkv, D, num_layers), dtype=torch.uint8,
+                       device=device or "cuda")
+
+
+def _out_dtype(dt: torch.dtype) -> torch.dtype:
+    """What `out` must hold: the element type, or float32 while KV_OPT_OUT_F32 is on."""
+    return torch.float32 if get_option(KV_OPT_OUT_F32) == 1 else dt
 
 
 def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
@@ -146,7 +184,7 @@ def paged_attention_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Te
         raise ValueError("shape mismatch")
     dt, code = k_cache.dtype, _cache_dtype(k_cache)
     _check("paged_attention_decode", _lib.paged_attention_decode(
-        _dev(out, "out", dt), _dev(q, "q", dt),
+        _dev(out, "out", _out_dtype(dt)), _dev(q, "q", dt),
         _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
@@ -165,11 +203,52 @@ def paged_attention_decode_append(out: torch.Tensor, q: torch.Tensor, k_new: tor
         raise ValueError("shape mismatch")
     dt, code = k_cache.dtype, _cache_dtype(k_cache)
     _check("paged_attention_decode_append", _lib.paged_attention_decode_append(
-        _dev(out, "out", dt), _dev(q, "q", dt),
+        _dev(out, "out", _out_dtype(dt)), _dev(q, "q", dt),
         _dev(k_new, "k_new", dt), _dev(v_new, "v_new", dt),
         _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
         _dev(slot_mapping, "slot_mapping", torch.int64),
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
+        _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
+        _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
+    return out
+
+
+def paged_attention_decode_layers(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                  block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                                  workspace: torch.Tensor, k_new: torch.Tensor | None = None,
+                                  v_new: torch.Tensor | None = None, slot_mapping: torch.Tensor | None = None,
+                                  stream=None) -> torch.Tensor:
+    """Every layer of a decode step in one launch: out[l] = decode of q[l] over layer l's caches.
+
+    q, out [L,B,Hq,D] and k_new, v_new [L,B,Hkv,D] contiguous; k_cache, v_cache [L,num_blocks,16,Hkv,D] whose
+    layers may sit any equal stride apart (each layer contiguous), e.g. views of one larger pool. With k_new,
+    v_new and slot_mapping given, this step's token of every sequence is appended to every layer first (fused).
+    The workspace must be sized for L layers (make_workspace(..., num_layers=L)).
+    """
+    L, B, Hq, D = q.shape
+    Lk, num_blocks, bt, Hkv, Dk = k_cache.shape
+    if (Lk != L or Dk != D or bt != BLOCK_TOKENS or tuple(out.shape) != (L, B, Hq, D)
+            or tuple(v_cache.shape) != tuple(k_cache.shape) or block_tables.dim() != 2 or block_tables.shape[0] != B):
+        raise ValueError("shape mismatch")
+    if k_cache.stride(0) != v_cache.stride(0) or not (k_cache[0].is_contiguous() and v_cache[0].is_contiguous()):
+        raise ValueError("k_cache and v_cache must be layers of contiguous pools at one common stride")
+    if (k_new is None) != (v_new is None) or (k_new is None) != (slot_mapping is None):
+        raise ValueError("k_new, v_new and slot_mapping come together")
+    dt, code = k_cache.dtype, _cache_dtype(k_cache)
+    for name, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if not t.is_cuda or t.dtype != dt:
+            raise ValueError(f"{name} must be a CUDA {dt} tensor")
+    if k_new is not None:
+        if tuple(k_new.shape) != (L, B, Hkv, D) or tuple(v_new.shape) != (L, B, Hkv, D):
+            raise ValueError("shape mismatch")
+        kn, vn = _dev(k_new, "k_new", dt), _dev(v_new, "v_new", dt)
+        sm = _dev(slot_mapping, "slot_mapping", torch.int64)
+    else:
+        kn = vn = sm = None
+    stride = k_cache.stride(0) if L > 1 else num_blocks * BLOCK_TOKENS * Hkv * D
+    _check("paged_attention_decode_layers", _lib.paged_attention_decode_layers(
+        _dev(out, "out", _out_dtype(dt)), _dev(q, "q", dt), kn, vn, k_cache.data_ptr(), v_cache.data_ptr(), stride, L,
+        sm, _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream_handle(stream)))
     return out
@@ -189,7 +268,7 @@ def paged_attention_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.T
     dt, code = k_cache.dtype, _cache_dtype(k_cache)
     ef = _dev(error_flag, "error_flag", torch.int32) if error_flag is not None else None
     _check("paged_attention_prefill", _lib.paged_attention_prefill(
-        _dev(out, "out", dt), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(out, "out", _out_dtype(dt)), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev(context_lens, "context_lens", torch.int32), _dev(query_start, "query_start", torch.int32), B,
         int(max_query_len), num_blocks, Hq, Hkv, D, float(scale), code, ef, _stream_handle(stream)))
@@ -275,7 +354,7 @@ def paged_attention_decode_noalloc(out: torch.Tensor, q: torch.Tensor, k_cache: 
         raise ValueError("shape mismatch")
     dt, code = k_cache.dtype, _cache_dtype(k_cache)
     _check("paged_attention_decode_noalloc", _lib.paged_attention_decode_noalloc(
-        _dev(out, "out", dt), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        _dev(out, "out", _out_dtype(dt)), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
         _dev(block_tables, "block_tables", torch.int32), block_tables.shape[1],
         _dev(context_lens, "context_lens", torch.int32), B, num_blocks, Hq, Hkv, D, float(scale), code,
         _stream_handle(stream)))
@@ -399,6 +478,10 @@ class BlockPool:
 # ---------------------------------------------------------------------------
 def paged_attention_workspace_size(B: int, Hq: int, Hkv: int, D: int) -> int:
     return workspace_size(B, Hq, Hkv, D)
+
+
+def paged_attention_workspace_size_layers(B: int, Hq: int, Hkv: int, D: int, num_layers: int) -> int:
+    return workspace_size_layers(B, Hq, Hkv, D, num_layers)
 
 
 def paged_attention_workspace_init(workspace: torch.Tensor, stream=None) -> None:

@@ -21,7 +21,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libpagedkv.so")
 SOURCES = ["append.cu", "decode.cu", "prefill.cu", "blocks.cu", "pool.cpp"]
-HEADERS = ["pkv_device.cuh"]
+HEADERS = ["pkv_device.cuh", "tma_host.h", "nvtx_range.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -8,6 +8,7 @@
 // Hkv * D contiguous bf16. One thread moves one 16-byte chunk of one row with a
 // 128-bit load and store, so a warp covers 512 contiguous bytes.
 #include "pkv_device.cuh"
+#include "nvtx_range.h"
 #include "pagedkv.h"
 
 #include <cuda_runtime.h>
@@ -50,6 +51,7 @@ extern "C" kv_status kv_cache_append(const void *k_new, const void *v_new, void 
                                      const int64_t *slot_mapping, int T, int num_blocks, int Hkv, int D, int dtype,
                                      int32_t *error_flag, kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("kv_cache_append");
     if (T < 0 || num_blocks < 1 || Hkv < 1 || (dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_FP16) || (D != 64 && D != 128))
         return KV_ERR_ARG;
     if (T == 0)

@@ -16,6 +16,7 @@
 // One warp moves one block of one tensor with 16-byte loads and stores (16 * Hkv
 // * D * 2 bytes, a multiple of 256), many blocks in flight.
 #include "pkv_device.cuh"
+#include "nvtx_range.h"
 #include "pagedkv.h"
 
 #include <cuda_runtime.h>
@@ -110,6 +111,7 @@ extern "C" kv_status kv_cache_copy_blocks(void *const *caches, int n_caches, con
                                           const int32_t *dst_ids, int n, int num_blocks, int Hkv, int D, int dtype,
                                           int32_t *error_flag, kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("kv_cache_copy_blocks");
     return launch_move(caches, n_caches, nullptr, src_ids, dst_ids, n, num_blocks, Hkv, D, dtype, 0, error_flag,
                        stream);
 }
@@ -118,6 +120,7 @@ extern "C" kv_status kv_cache_gather_blocks(void *out, void *const *caches, int 
                                             int n, int num_blocks, int Hkv, int D, int dtype, int32_t *error_flag,
                                             kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("kv_cache_gather_blocks");
     return launch_move(caches, n_caches, out, block_ids, nullptr, n, num_blocks, Hkv, D, dtype, 1, error_flag,
                        stream);
 }
@@ -126,6 +129,7 @@ extern "C" kv_status kv_cache_scatter_blocks(void *const *caches, int n_caches, 
                                              const int32_t *block_ids, int n, int num_blocks, int Hkv, int D,
                                              int dtype, int32_t *error_flag, kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("kv_cache_scatter_blocks");
     return launch_move(caches, n_caches, const_cast<void *>(in), nullptr, block_ids, n, num_blocks, Hkv, D, dtype, 2,
                        error_flag, stream);
 }

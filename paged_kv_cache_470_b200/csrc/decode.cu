@@ -43,7 +43,17 @@
 // q, the cache and out are all bf16 or all fp16 (the element type E); the
 // cache holds 2 bytes per number either way ("Module 23: Serving", section
 // 23.1).
+//
+// Layers. One launch may cover L layers of one decode step ("Module 23:
+// Serving", section 23.1: every layer holds its own K and V for every token):
+// q, out and the new token rows are stacked [L][B][...], the caches are L
+// equally shaped pools a fixed stride apart, and the block tables and lengths
+// are shared by all layers (a sequence's position -> block map does not depend
+// on the layer). The work positions of layer l follow those of layer l - 1, so
+// the split-K tail of one layer overlaps the next layer's streaming; L = 1 is
+// the per-layer call.
 #include "pkv_device.cuh"
+#include "nvtx_range.h"
 #include "pagedkv.h"
 #include "tma_host.h"
 
@@ -97,8 +107,8 @@ struct Geo {
 };
 
 struct DecodeArgs {
-    uint16_t *out;        // [B][Hq][D] elements of type E
-    const uint16_t *q;    // [B][Hq][D]
+    uint16_t *out;        // [L][B][Hq][D] elements of type E (fp32 numbers when out_f32)
+    const uint16_t *q;    // [L][B][Hq][D]
     const int32_t *block_tables;
     const int32_t *context_lens;
     float *part_acc;     // [slots][kMaxHG][8][D]
@@ -106,6 +116,8 @@ struct DecodeArgs {
     int32_t *counters;   // [items]
     int32_t *status;
     int B, W, Hq, Hkv, group, num_blocks;
+    int L;               // layers in this launch
+    int out_f32;         // out holds fp32 numbers (a debug switch: the result before rounding)
     int hg;              // kv heads per unit (HG)
     int streams;         // consumer streams = 8 / HG
     int hchunks;         // query-head chunks per kv head = ceil(group / 8)
@@ -115,14 +127,16 @@ struct DecodeArgs {
     int min_chunk;
     int item_cost;       // work positions charged per work item on top of its units
     int drop_unit;       // test hook: CTA 0 never loads its unit with this index (-1: none)
+    int l2_policy;       // L2 priority of the K/V tile loads: 1 evict first, 2 evict normal, 3 evict last
     int fused;
     float scale_log2;    // scale * log2(e)
     // fused append (append != 0): this step's token of sequence b is k_new/v_new[b],
     // at slot slots[b], which must be position context_lens[b] - 1 of sequence b
     int append;
-    const uint4 *k_new, *v_new;   // [B][Hkv][D], as 16-byte chunks
-    uint4 *k_cache, *v_cache;     // [num_blocks][16][Hkv][D], as 16-byte chunks
-    const int64_t *slots;         // [B]
+    const uint4 *k_new, *v_new;   // [L][B][Hkv][D], as 16-byte chunks
+    uint4 *k_cache, *v_cache;     // layer 0's [num_blocks][16][Hkv][D], as 16-byte chunks
+    size_t cache_layer_chunks;    // 16-byte chunks from one layer's cache to the next
+    const int64_t *slots;         // [B], shared by the layers
 };
 
 // misc ints in shared memory
@@ -139,6 +153,8 @@ enum {
     kMiscStartU = 39,   // units before the CTA's range, and before its end
     kMiscEndU = 40,
     kMiscEndFound = 41,
+    kMiscLocLayer = 42, // layer of the CTA's first unit
+    kMiscStartFound = 43,
     kMiscScan64 = 44,   // 10 64-bit warp sums (ints 44..63)
 };
 
@@ -188,6 +204,7 @@ __device__ __forceinline__ long long seq_scan_value(const DecodeArgs &a, int n)
 }
 
 struct Cursor {
+    int layer; // layer
     int b;     // sequence
     int k;     // item within the sequence: head group * hchunks + query-head chunk
     int off;   // block offset within the sequence
@@ -202,11 +219,20 @@ __device__ __forceinline__ void cursor_next_item(const DecodeArgs &a, Cursor &c)
     c.off = 0;
     if (++c.k == a.items_per_seq) {
         c.k = 0;
-        do {
-            ++c.b;
-            c.ctx = (c.b < a.B) ? seq_ctx(a, c.b) : 0;
+        for (;;) {
+            if (++c.b == a.B) {
+                if (c.layer + 1 == a.L) {  // past the last item of the launch
+                    c.ctx = c.n = 0;
+                    break;
+                }
+                ++c.layer;  // the next layer starts again at the first sequence
+                c.b = 0;
+            }
+            c.ctx = seq_ctx(a, c.b);
             c.n = ctx_blocks(c.ctx);
-        } while (c.n == 0 && c.b < a.B);
+            if (c.n > 0)
+                break;
+        }
     }
 }
 
@@ -261,15 +287,27 @@ __device__ __forceinline__ float rescale(float x, float m) { return m == -INFINI
 
 // The new token of one kv head of an item, for the fused append: lane l < D/8
 // holds 16-byte chunk l of the K row, lane D/8 <= l < D/4 chunk l - D/8 of the
-// V row. `slot` is where it goes (-1: nothing to append, or a bad slot).
+// V row. `slot` is where it goes (-1: nothing to append, or a bad slot) and
+// `dst` the index of its first 16-byte chunk in the layer's K (or V) cache.
 struct AppendRow {
     uint4 chunk;
     long long slot;
+    size_t dst;
 };
+
+// Row (layer, sequence) of q and out: layer * B + b.
+__device__ __forceinline__ int layer_row(const DecodeArgs &a, const Cursor &cur) { return cur.layer * a.B + cur.b; }
+
+// Work item index within the launch: (layer * B + b) * items_per_seq + k.
+__device__ __forceinline__ int item_index(const DecodeArgs &a, const Cursor &cur)
+{
+    return layer_row(a, cur) * a.items_per_seq + cur.k;
+}
 
 // Where an item's outputs go.
 struct ItemOut {
-    int b, h0, gc;   // sequence, first query head of this warp's kv head, valid query heads (<= 8)
+    int lb, h0, gc;  // row (layer, sequence) of q and out, first query head of this warp's kv head,
+                     // valid query heads (<= 8)
     size_t slot;     // split-K piece slot (only for partial items)
     int hh;          // kv head within the group
 };
@@ -278,12 +316,22 @@ __device__ __forceinline__ ItemOut item_out(const DecodeArgs &a, const Cursor &c
 {
     const int hg = cur.k / a.hchunks, hc = cur.k - hg * a.hchunks;
     ItemOut o;
-    o.b = cur.b;
+    o.lb = layer_row(a, cur);
     o.hh = hh;
     o.h0 = (hg * a.hg + hh) * a.group + hc * kGroupMax;
     o.gc = min(kGroupMax, a.group - hc * kGroupMax);
-    o.slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(cur.b) * a.items_per_seq + cur.k;
+    o.slot = static_cast<size_t>(blockIdx.x) + static_cast<size_t>(item_index(a, cur));
     return o;
+}
+
+// One output number at element index i of out (element type E, or fp32 when out_f32).
+template <class E>
+__device__ __forceinline__ void put_out(const DecodeArgs &a, size_t i, float v)
+{
+    if (a.out_f32)
+        reinterpret_cast<float *>(a.out)[i] = v;
+    else
+        a.out[i] = E::from_f32(v);
 }
 
 // ---------------------------------------------------------------------------
@@ -310,7 +358,7 @@ struct Consumer<E, D, kPathMma, NH> {
     {
         const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
         const uint32_t *qrow =
-            reinterpret_cast<const uint32_t *>(a.q + (static_cast<size_t>(o.b) * a.Hq + o.h0 + r) * D);
+            reinterpret_cast<const uint32_t *>(a.q + (static_cast<size_t>(o.lb) * a.Hq + o.h0 + r) * D);
 #pragma unroll
         for (int kk = 0; kk < kMt; ++kk) {
             qn[kk][0] = (r < o.gc) ? __ldg(qrow + kk * 8 + c) : 0u;
@@ -452,18 +500,18 @@ struct Consumer<E, D, kPathMma, NH> {
         const int lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
         const int n0 = 2 * c, n1 = 2 * c + 1;
         const float i0 = 1.f / l0, i1 = 1.f / l1;
-        uint16_t *o0 = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n0) * D;
-        uint16_t *o1 = o0 + D;
+        const size_t o0 = (static_cast<size_t>(o.lb) * a.Hq + o.h0 + n0) * D;
+        const size_t o1 = o0 + D;
 #pragma unroll
         for (int mt = 0; mt < kMt; ++mt) {
             const int d = mt * 16 + r;
             if (n0 < o.gc) {
-                o0[d] = E::from_f32(acc[mt][0] * i0);
-                o0[d + 8] = E::from_f32(acc[mt][2] * i0);
+                put_out<E>(a, o0 + d, acc[mt][0] * i0);
+                put_out<E>(a, o0 + d + 8, acc[mt][2] * i0);
             }
             if (n1 < o.gc) {
-                o1[d] = E::from_f32(acc[mt][1] * i1);
-                o1[d + 8] = E::from_f32(acc[mt][3] * i1);
+                put_out<E>(a, o1 + d, acc[mt][1] * i1);
+                put_out<E>(a, o1 + d + 8, acc[mt][3] * i1);
             }
         }
     }
@@ -658,10 +706,10 @@ struct Consumer<E, D, kPathSimt, NH> {
         for (int n = 0; n < NH; ++n) {
             if (n < o.gc) {
                 const float inv = 1.f / l[n];
-                uint16_t *dst = a.out + (static_cast<size_t>(o.b) * a.Hq + o.h0 + n) * D + lane * C;
+                const size_t dst = (static_cast<size_t>(o.lb) * a.Hq + o.h0 + n) * D + lane * C;
 #pragma unroll
                 for (int e = 0; e < C; ++e)
-                    dst[e] = E::from_f32(acc[n][e] * inv);
+                    put_out<E>(a, dst + e, acc[n][e] * inv);
             }
         }
     }
@@ -696,7 +744,7 @@ struct Consumer<E, D, kPathSimt, NH> {
 // merges.
 template <class E, int D>
 __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int item, int first_cta, int last_cta,
-                                                    int b, int k, int tid, int nthreads, int own_cta = -1,
+                                                    int lb, int k, int tid, int nthreads, int own_cta = -1,
                                                     const float *own_acc = nullptr, const float *own_ml = nullptr)
 {
     constexpr int NC = D == 128 ? 4 : 2;          // float4 column groups per thread
@@ -773,13 +821,18 @@ __device__ __forceinline__ void merge_pieces_global(const DecodeArgs &a, int ite
         }
         const int h = (hg * a.hg + hh) * a.group + hc * kGroupMax + n;
         const float inv = 1.f / L;
-        uint16_t *dst = a.out + (static_cast<size_t>(b) * a.Hq + h) * D + col0;
+        const size_t dst = (static_cast<size_t>(lb) * a.Hq + h) * D + col0;
 #pragma unroll
         for (int e = 0; e < NC; ++e) {
-            uint2 packed;
-            packed.x = E::pack(O[e].x * inv, O[e].y * inv);
-            packed.y = E::pack(O[e].z * inv, O[e].w * inv);
-            *reinterpret_cast<uint2 *>(dst + e * 4) = packed;
+            if (a.out_f32) {
+                *reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + dst + e * 4) =
+                    make_float4(O[e].x * inv, O[e].y * inv, O[e].z * inv, O[e].w * inv);
+            } else {
+                uint2 packed;
+                packed.x = E::pack(O[e].x * inv, O[e].y * inv);
+                packed.y = E::pack(O[e].z * inv, O[e].w * inv);
+                *reinterpret_cast<uint2 *>(a.out + dst + e * 4) = packed;
+            }
         }
     }
 }
@@ -803,13 +856,14 @@ __device__ __forceinline__ AppendRow load_append_row(const DecodeArgs &a, const 
     const int blk = __ldg(a.block_tables + static_cast<size_t>(cur.b) * a.W + last / kBlockTokens);
     const long long expect = static_cast<long long>(blk) * kBlockTokens + last % kBlockTokens;
     if (slot != expect || blk < 0 || blk >= a.num_blocks) {
-        if (report && lane == 0)
+        if (report && lane == 0 && cur.layer == 0)  // every layer sees the same slot: report it once
             atomicOr(a.status, KV_STATUS_BAD_SLOT);
         return r;
     }
     r.slot = slot;
     constexpr int C = D / 8;  // 16-byte chunks per head row
-    const size_t row = (static_cast<size_t>(cur.b) * a.Hkv + j) * C;
+    r.dst = cur.layer * a.cache_layer_chunks + (static_cast<size_t>(slot) * a.Hkv + j) * C;
+    const size_t row = (static_cast<size_t>(layer_row(a, cur)) * a.Hkv + j) * C;
     if (lane < C)
         r.chunk = __ldg(a.k_new + row + lane);
     else if (lane < 2 * C)
@@ -833,7 +887,7 @@ __device__ __forceinline__ void apply_append_row(const DecodeArgs &a, const Appe
                      "r"(r.chunk.z), "r"(r.chunk.w)
                      : "memory");
         if (write) {
-            uint4 *dst = (is_v ? a.v_cache : a.k_cache) + (static_cast<size_t>(r.slot) * a.Hkv + j) * C + ch;
+            uint4 *dst = (is_v ? a.v_cache : a.k_cache) + r.dst + ch;
             *dst = r.chunk;
         }
         // the stage is refilled by TMA later: order these writes before that
@@ -842,18 +896,21 @@ __device__ __forceinline__ void apply_append_row(const DecodeArgs &a, const Appe
     __syncwarp();
 }
 
-// Outputs of empty sequences are zero; also flag out-of-range lengths. Run by CTA 0.
+// Outputs of empty sequences are zero (in every layer); also flag out-of-range
+// lengths. Run by CTA 0.
 template <int D>
 __device__ __forceinline__ void zero_empty_outputs(const DecodeArgs &a, int tid, int nthreads)
 {
-    for (int b = tid; b < a.B; b += nthreads) {
+    const int row16 = a.Hq * D * (a.out_f32 ? 2 : 1);  // 16-bit words per output row
+    for (int lb = tid; lb < a.L * a.B; lb += nthreads) {
+        const int b = lb % a.B;
         const int c = __ldg(a.context_lens + b);
-        if (c < 0 || c > a.W * kBlockTokens)
+        if (lb < a.B && (c < 0 || c > a.W * kBlockTokens))
             atomicOr(a.status, KV_STATUS_BAD_CONTEXT);
         if (clamp_ctx(c, a.W) == 0) {
-            uint16_t *o = a.out + static_cast<size_t>(b) * a.Hq * D;
-            for (int i = 0; i < a.Hq * D; ++i)
-                o[i] = 0;  // +0.0 in both element types
+            uint16_t *o = a.out + static_cast<size_t>(lb) * row16;
+            for (int i = 0; i < row16; ++i)
+                o[i] = 0;  // +0.0 in both element types and in fp32
         }
     }
 }
@@ -910,6 +967,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         misc[kMiscAbort] = 0;
         misc[kMiscLocB] = -1;
         misc[kMiscEndFound] = 0;
+        misc[kMiscStartFound] = 0;
         misc[kMiscZero] = 0;
     }
     if (warp == kProducerWarp && lane == 0) {
@@ -926,7 +984,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         mine += seq_scan_value(a, ctx_blocks(seq_ctx(a, b)));
     long long sum64;
     block_scan_incl64(mine, scan64, &sum64);
-    const int total = static_cast<int>(sum64 >> kNonEmptyBits);  // work positions
+    // Work positions of one layer; every layer has the same (tables and lengths are shared), and
+    // layer l's positions follow layer l - 1's.
+    const int per_layer = static_cast<int>(sum64 >> kNonEmptyBits);
+    const int nonempty = static_cast<int>(sum64 & ((1 << kNonEmptyBits) - 1));
+    const int units_layer = per_layer - w * a.items_per_seq * nonempty;
+    const int total = a.L * per_layer;  // the host checked that it fits
     int chunk = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
     if (chunk < a.min_chunk)
         chunk = a.min_chunk;
@@ -934,7 +997,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int end = min(start + chunk, total);
 
     if (start < total) {
-        // locate the CTA's first unit and count the units in [start, end)
+        // locate the CTA's first unit and count the units in [start, end): the layer of each end
+        // by division, the position within the layer by a scan over the sequences
+        const int ls = start / per_layer, ss = start - ls * per_layer;
+        const int le = (end - 1) / per_layer, se = end - 1 - le * per_layer;
         long long running = 0;
         for (int base_b = 0; base_b < a.B; base_b += kThreads) {
             const int b = base_b + tid;
@@ -945,22 +1011,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             const int lo = static_cast<int>(before >> kNonEmptyBits);
             const int hi = lo + static_cast<int>(v >> kNonEmptyBits);
             const int units_before = lo - w * a.items_per_seq * static_cast<int>(before & ((1 << kNonEmptyBits) - 1));
-            if (n > 0 && start >= lo && start < hi) {
-                const int r = start - lo, k = r / (n + w), rr = r - k * (n + w);
+            if (n > 0 && ss >= lo && ss < hi) {
+                const int r = ss - lo, k = r / (n + w), rr = r - k * (n + w);
+                misc[kMiscLocLayer] = ls;
                 misc[kMiscLocB] = b;
                 misc[kMiscLocK] = k;
                 misc[kMiscLocOff] = max(0, rr - w);
-                misc[kMiscLocPos] = lo + k * (n + w) + w;
-                misc[kMiscStartU] = units_before + k * n + max(0, rr - w);
+                misc[kMiscLocPos] = ls * per_layer + lo + k * (n + w) + w;
+                misc[kMiscStartU] = ls * units_layer + units_before + k * n + max(0, rr - w);
+                misc[kMiscStartFound] = 1;
             }
-            if (n > 0 && end - 1 >= lo && end - 1 < hi) {
-                const int r = end - 1 - lo, k = r / (n + w), rr = r - k * (n + w);
-                misc[kMiscEndU] = units_before + k * n + max(0, rr - w) + (rr >= w ? 1 : 0);
+            if (n > 0 && se >= lo && se < hi) {
+                const int r = se - lo, k = r / (n + w), rr = r - k * (n + w);
+                misc[kMiscEndU] = le * units_layer + units_before + k * n + max(0, rr - w) + (rr >= w ? 1 : 0);
                 misc[kMiscEndFound] = 1;
             }
             running += tot;
             __syncthreads();
-            if (misc[kMiscEndFound])
+            if (misc[kMiscEndFound] && misc[kMiscStartFound])
                 break;
         }
     }
@@ -975,6 +1043,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
 
     Cursor cur0;
+    cur0.layer = misc[kMiscLocLayer];
     cur0.b = misc[kMiscLocB];
     cur0.ctx = seq_ctx(a, cur0.b);
     cur0.n = ctx_blocks(cur0.ctx);
@@ -995,7 +1064,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         grid_launch_dependents();
         if (bad_first)
             atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
-        const uint64_t policy = l2_policy_evict_first();
+        const uint64_t policy = a.l2_policy == 2   ? l2_policy_evict_normal()
+                                : a.l2_policy == 3 ? l2_policy_evict_last()
+                                                   : l2_policy_evict_first();
         const int NL = a.prod_lanes;
         Cursor cur = cur0;
         int u = 0, issued = 0;
@@ -1029,11 +1100,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                             const uint32_t dst = ring + s * a.stage_bytes;
 #pragma unroll
                             for (int t = 0; t < G::kTiles; ++t)
-                                tma_load_4d(dst + t * a.tile_stride, &tmK, t * 64, 0, head0, phys, &full[s], policy);
+                                tma_load_5d(dst + t * a.tile_stride, &tmK, t * 64, 0, head0, phys, cur.layer,
+                                            &full[s], policy);
 #pragma unroll
                             for (int t = 0; t < G::kTiles; ++t)
-                                tma_load_4d(dst + (G::kTiles + t) * a.tile_stride, &tmV, t * 64, 0, head0, phys,
-                                            &full[s], policy);
+                                tma_load_5d(dst + (G::kTiles + t) * a.tile_stride, &tmV, t * 64, 0, head0, phys,
+                                            cur.layer, &full[s], policy);
                         } else {
                             *abort_flag = 1;
                             atomicOr(a.status, KV_STATUS_WAIT_TIMEOUT);
@@ -1073,7 +1145,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (!mbar_wait_bounded(qbar + q, (k / kPieceQueue) & 1, abort_flag))
                 break;
             const volatile int *desc = misc + kMiscQueue + 5 * q;
-            const int item = desc[0], first_cta = desc[1], last_cta = desc[2], b = desc[3], kk = desc[4];
+            const int item = desc[0], first_cta = desc[1], last_cta = desc[2], lb = desc[3], kk = desc[4];
             if (item < 0)
                 break;
             int last = 0;
@@ -1082,7 +1154,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             }
             last = __shfl_sync(kFull, last, 0);
             if (last) {
-                merge_pieces_global<E, D>(a, item, first_cta, last_cta, b, kk, lane, 32);
+                merge_pieces_global<E, D>(a, item, first_cta, last_cta, lb, kk, lane, 32);
                 __syncwarp();
                 if (lane == 0)
                     a.counters[item] = 0;
@@ -1116,7 +1188,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     int pushed = 0;  // split pieces handed to the helper (thread 0's count)
     while (u < count) {
         const int run = min(cur.n - cur.off, count - u);
-        const int item = cur.b * a.items_per_seq + cur.k;
+        const int item = item_index(a, cur);
         const int hg = cur.k / a.hchunks, hc = cur.k - hg * a.hchunks;
         const ItemOut o = item_out(a, cur, hh);
         const int first_cta = cur.pos / chunk;
@@ -1138,7 +1210,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 const int rem = idx - h2 * per;
                 const int n = rem / D, d = rem - n * D;
                 const int h = (hg * a.hg + h2) * a.group + hc * kGroupMax + n;
-                const float v = (n < o.gc) ? E::to_f32(a.q[(static_cast<size_t>(cur.b) * a.Hq + h) * D + d]) : 0.f;
+                const float v =
+                    (n < o.gc) ? E::to_f32(a.q[(static_cast<size_t>(o.lb) * a.Hq + h) * D + d]) : 0.f;
                 scratch[(h2 * kGroupMax + n) * G::kQStride + d + ((d >= D / 2) ? 4 : 0)] = v;
             }
             named_barrier(kBarConsumers, kConsumerThreads);
@@ -1225,7 +1298,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         if (!single && solo) {
             // every other piece is done: merge them with this one (read from shared memory)
             named_barrier(kBarConsumers, kConsumerThreads);
-            merge_pieces_global<E, D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads,
+            merge_pieces_global<E, D>(a, item, first_cta, last_cta, o.lb, cur.k, tid, kConsumerThreads,
                                       static_cast<int>(blockIdx.x), own_acc, own_ml);
             if (tid == 0)
                 a.counters[item] = 0;
@@ -1241,7 +1314,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         desc[0] = item;
                         desc[1] = first_cta;
                         desc[2] = last_cta;
-                        desc[3] = cur.b;
+                        desc[3] = o.lb;
                         desc[4] = cur.k;
                         mbar_arrive(qbar + q);
                         ++pushed;
@@ -1258,7 +1331,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                 }
                 named_barrier(kBarConsumers, kConsumerThreads);
                 if (misc[kMiscLast]) {
-                    merge_pieces_global<E, D>(a, item, first_cta, last_cta, cur.b, cur.k, tid, kConsumerThreads);
+                    merge_pieces_global<E, D>(a, item, first_cta, last_cta, o.lb, cur.k, tid, kConsumerThreads);
                     if (tid == 0)
                         a.counters[item] = 0;
                 }
@@ -1289,7 +1362,8 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int gr
     grid_dependency_wait();
     grid_launch_dependents();
     const int item = blockIdx.x;
-    const int b = item / a.items_per_seq, k = item - b * a.items_per_seq;
+    const int lb = item / a.items_per_seq, k = item - lb * a.items_per_seq;
+    const int layer = lb / a.B, b = lb - layer * a.B;
     // work positions, as the decode kernel counts them
     int pre = 0, tot = 0;
     for (int bb = threadIdx.x; bb < a.B; bb += 128) {
@@ -1313,14 +1387,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const DecodeArgs a, int gr
     const int n = ctx_blocks(seq_ctx(a, b));
     if (n == 0)
         return;
-    int chunk = (tot + grid_ctas - 1) / grid_ctas;
+    const int total = a.L * tot;  // tot: positions of one layer
+    int chunk = (total + grid_ctas - 1) / grid_ctas;
     if (chunk < a.min_chunk)
         chunk = a.min_chunk;
-    const int item_pos = pre + k * (n + a.item_cost) + a.item_cost;  // its first unit
+    const int item_pos = layer * tot + pre + k * (n + a.item_cost) + a.item_cost;  // its first unit
     const int first_cta = item_pos / chunk, last_cta = (item_pos + n - 1) / chunk;
     if (first_cta == last_cta)
         return;
-    merge_pieces_global<E, D>(a, item, first_cta, last_cta, b, k, threadIdx.x, 128);
+    merge_pieces_global<E, D>(a, item, first_cta, last_cta, lb, k, threadIdx.x, 128);
 }
 
 }  // namespace pkv
@@ -1342,6 +1417,8 @@ std::atomic<int> g_opt_item_cost{0};
 std::atomic<int> g_opt_prefill_path{0};
 std::atomic<int> g_opt_drop_load{0};
 std::atomic<int> g_opt_slow_softmax{0};
+std::atomic<int> g_opt_out_f32{0};
+std::atomic<int> g_opt_l2_policy{0};
 constexpr int kDefaultMinChunk = 4;
 
 // Work positions charged per work item (its fixed cost, in units of one work
@@ -1390,22 +1467,26 @@ struct Layout {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-bool make_layout(int B, int Hq, int Hkv, int D, int sms, Layout *L)
+// Workspace of a launch over `layers` layers of B sequences on a device with
+// `sms` SMs: the status word, one counter per work item, and per split-K piece
+// slot (m, l) and the accumulator.
+bool make_layout(int B, int Hq, int Hkv, int D, int layers, int sms, Layout *lay)
 {
-    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (D != 64 && D != 128) || sms < 1)
+    if (B < 0 || layers < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (D != 64 && D != 128) || sms < 1)
         return false;
     const int group = Hq / Hkv;
     const long long hchunks = (group + kGroupMax - 1) / kGroupMax;
-    const long long items = static_cast<long long>(B) * (Hkv / heads_per_unit(Hkv)) * hchunks;
+    const long long items =
+        static_cast<long long>(layers) * B * (Hkv / heads_per_unit(Hkv)) * hchunks;
     if (items > (1ll << 30))
         return false;
-    L->items = static_cast<int>(items);
-    L->max_grid = kCtasPerSm * sms;
-    L->slots = L->max_grid + L->items;
-    L->off_counters = kStatusBytes;
-    L->off_ml = L->off_counters + round256(static_cast<size_t>(L->items) * 4);
-    L->off_acc = L->off_ml + round256(static_cast<size_t>(L->slots) * kMaxHG * kGroupMax * 2 * 4);
-    L->bytes = L->off_acc + round256(static_cast<size_t>(L->slots) * kMaxHG * kGroupMax * D * 4);
+    lay->items = static_cast<int>(items);
+    lay->max_grid = kCtasPerSm * sms;
+    lay->slots = lay->max_grid + lay->items;
+    lay->off_counters = kStatusBytes;
+    lay->off_ml = lay->off_counters + round256(static_cast<size_t>(lay->items) * 4);
+    lay->off_acc = lay->off_ml + round256(static_cast<size_t>(lay->slots) * kMaxHG * kGroupMax * 2 * 4);
+    lay->bytes = lay->off_acc + round256(static_cast<size_t>(lay->slots) * kMaxHG * kGroupMax * D * 4);
     return true;
 }
 
@@ -1466,38 +1547,28 @@ int prepare_kernel(DecodeFn fn, int smem, int dev)
 
 bool misaligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
 
-}  // namespace
+// A checked decode launch: everything it needs, built on the host before
+// anything is enqueued. grid == 0 means there is nothing to launch (B == 0).
+struct DecodePlan {
+    DecodeFn fn = nullptr;
+    int smem = 0, grid = 0, dtype = 0, D = 0;
+    Layout lay;
+    CUtensorMap tmK, tmV;
+    DecodeArgs a;
+};
 
-extern "C" size_t paged_attention_workspace_size(int B, int Hq, int Hkv, int D)
+// Validate a decode over `layers` layers (k_new == nullptr: no append) and fill
+// *p. Enqueues nothing; KV_ERR_ARG / KV_ERR_CUDA as the entry points document.
+// cache_layer_stride is in elements (ignored when layers == 1).
+kv_status plan_decode(DecodePlan *p, void *out, const void *q, const void *k_new, const void *v_new,
+                      const void *k_cache, const void *v_cache, size_t cache_layer_stride, int layers,
+                      const int64_t *slot_mapping, const int32_t *block_tables, int max_blocks_per_seq,
+                      const int32_t *context_lens, int B, int num_blocks, int Hq, int Hkv, int D, float scale,
+                      int dtype, void *workspace, size_t workspace_bytes)
 {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess)
-        return 0;
-    Layout L;
-    if (!make_layout(B, Hq, Hkv, D, device_sm_count(dev), &L))
-        return 0;
-    return L.bytes;
-}
-
-extern "C" kv_status paged_attention_workspace_init(void *workspace, size_t workspace_bytes, kv_stream_t stream)
-{
-    if (!workspace || workspace_bytes == 0)
-        return KV_ERR_ARG;
-    return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
-               ? KV_OK
-               : KV_ERR_CUDA;
-}
-
-// Shared by paged_attention_decode (k_new == nullptr) and the fused
-// append + decode entry point.
-static kv_status decode_impl(void *out, const void *q, const void *k_new, const void *v_new, const void *k_cache,
-                             const void *v_cache, const int64_t *slot_mapping, const int32_t *block_tables,
-                             int max_blocks_per_seq, const int32_t *context_lens, int B, int num_blocks, int Hq,
-                             int Hkv, int D, float scale, int dtype, void *workspace, size_t workspace_bytes,
-                             kv_stream_t stream)
-{
-    if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_FP16) || B < 0 || max_blocks_per_seq < 1 || num_blocks < 1 || Hq < 1 || Hkv < 1 ||
-        Hq % Hkv != 0 || (D != 64 && D != 128))
+    p->grid = 0;
+    if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_FP16) || B < 0 || layers < 1 || max_blocks_per_seq < 1 ||
+        num_blocks < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || (D != 64 && D != 128))
         return KV_ERR_ARG;
     if (B == 0)
         return KV_OK;
@@ -1506,11 +1577,17 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     if (misaligned(out, 16) || misaligned(q, 16) || misaligned(k_cache, 16) || misaligned(v_cache, 16) ||
         misaligned(block_tables, 4) || misaligned(context_lens, 4) || misaligned(workspace, 256))
         return KV_ERR_ARG;
+    const size_t layer_elems = static_cast<size_t>(num_blocks) * kBlockTokens * Hkv * D;
+    if (layers == 1)
+        cache_layer_stride = layer_elems;  // the map's layer dimension has one entry
+    else if (cache_layer_stride < layer_elems || cache_layer_stride % 8 != 0 ||
+             cache_layer_stride > (static_cast<size_t>(1) << 38))
+        return KV_ERR_ARG;  // overlapping layers, a stride that is not a multiple of 16 bytes, or too large
     const int group = Hq / Hkv;
     const int hg = heads_per_unit(Hkv);
     const int hchunks = (group + kGroupMax - 1) / kGroupMax;
     const int cost = item_cost(D);
-    if (static_cast<long long>(B) * (max_blocks_per_seq + cost) * (Hkv / hg) * hchunks >= (1ll << 31) ||
+    if (static_cast<long long>(layers) * B * (max_blocks_per_seq + cost) * (Hkv / hg) * hchunks >= (1ll << 31) ||
         B >= (1 << 24))
         return KV_ERR_ARG;
 
@@ -1518,10 +1595,9 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     if (cudaGetDevice(&dev) != cudaSuccess)
         return KV_ERR_CUDA;
     const int sms = device_sm_count(dev);
-    Layout L;
-    if (!make_layout(B, Hq, Hkv, D, sms, &L))
+    if (!make_layout(B, Hq, Hkv, D, layers, sms, &p->lay))
         return KV_ERR_ARG;
-    if (workspace_bytes < L.bytes)
+    if (workspace_bytes < p->lay.bytes)
         return KV_ERR_ARG;
 
     int path = g_opt_compute.load();
@@ -1532,17 +1608,16 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
         const int gmin = group < kGroupMax ? group : kGroupMax;
         nh = gmin <= 1 ? 1 : gmin <= 2 ? 2 : gmin <= 4 ? 4 : 8;
     }
-    int smem = 0;
-    DecodeFn fn = pick_kernel(dtype, D, path, nh, &smem);
-    if (!fn)
+    p->fn = pick_kernel(dtype, D, path, nh, &p->smem);
+    if (!p->fn)
         return KV_ERR_ARG;
-    const int occ = prepare_kernel(fn, smem, dev);
+    const int occ = prepare_kernel(p->fn, p->smem, dev);
     if (occ < 1)
         return KV_ERR_CUDA;
     int grid = (occ < kCtasPerSm ? occ : kCtasPerSm) * sms;
     const int want = g_opt_grid.load();
     if (want > 0)
-        grid = want < L.max_grid ? want : L.max_grid;
+        grid = want < p->lay.max_grid ? want : p->lay.max_grid;
 
     // ring geometry: stages a multiple of the consumer streams and of the producer lanes
     const int tiles = D / 64;
@@ -1560,20 +1635,20 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     if (stages < unit_of)
         return KV_ERR_ARG;
 
-    CUtensorMap tmK, tmV;
-    if (!pkv_host::make_cache_map(&tmK, k_cache, num_blocks, Hkv, D, hg, dtype) ||
-        !pkv_host::make_cache_map(&tmV, v_cache, num_blocks, Hkv, D, hg, dtype))
+    const unsigned long long stride_bytes = static_cast<unsigned long long>(cache_layer_stride) * 2;
+    if (!pkv_host::make_layered_cache_map(&p->tmK, k_cache, num_blocks, Hkv, D, hg, dtype, layers, stride_bytes) ||
+        !pkv_host::make_layered_cache_map(&p->tmV, v_cache, num_blocks, Hkv, D, hg, dtype, layers, stride_bytes))
         return KV_ERR_CUDA;
 
     unsigned char *ws = static_cast<unsigned char *>(workspace);
-    DecodeArgs a;
+    DecodeArgs &a = p->a;
     a.out = static_cast<uint16_t *>(out);
     a.q = static_cast<const uint16_t *>(q);
     a.block_tables = block_tables;
     a.context_lens = context_lens;
-    a.part_acc = reinterpret_cast<float *>(ws + L.off_acc);
-    a.part_ml = reinterpret_cast<float *>(ws + L.off_ml);
-    a.counters = reinterpret_cast<int32_t *>(ws + L.off_counters);
+    a.part_acc = reinterpret_cast<float *>(ws + p->lay.off_acc);
+    a.part_ml = reinterpret_cast<float *>(ws + p->lay.off_ml);
+    a.counters = reinterpret_cast<int32_t *>(ws + p->lay.off_counters);
     a.status = reinterpret_cast<int32_t *>(ws);
     a.B = B;
     a.W = max_blocks_per_seq;
@@ -1581,6 +1656,8 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     a.Hkv = Hkv;
     a.group = group;
     a.num_blocks = num_blocks;
+    a.L = layers;
+    a.out_f32 = g_opt_out_f32.load();
     a.hg = hg;
     a.streams = streams;
     a.hchunks = hchunks;
@@ -1593,50 +1670,89 @@ static kv_status decode_impl(void *out, const void *q, const void *k_new, const 
     a.min_chunk = mc > 0 ? mc : kDefaultMinChunk;
     a.item_cost = cost;
     a.drop_unit = g_opt_drop_load.load() - 1;
-    const int combine_mode = g_opt_combine.load();
-    a.fused = combine_mode == 0 ? 1 : 0;
+    a.l2_policy = g_opt_l2_policy.load() == 0 ? 1 : g_opt_l2_policy.load();
+    a.fused = g_opt_combine.load() == 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.append = k_new != nullptr ? 1 : 0;
     a.k_new = static_cast<const uint4 *>(k_new);
     a.v_new = static_cast<const uint4 *>(v_new);
     a.k_cache = static_cast<uint4 *>(const_cast<void *>(k_cache));
     a.v_cache = static_cast<uint4 *>(const_cast<void *>(v_cache));
+    a.cache_layer_chunks = cache_layer_stride / 8;
     a.slots = slot_mapping;
+    p->grid = grid;
+    p->dtype = dtype;
+    p->D = D;
+    return KV_OK;
+}
 
+// Enqueue a planned decode (and the separate combine kernel when that mode is set).
+kv_status launch_decode(const DecodePlan &p, kv_stream_t stream)
+{
+    if (p.grid == 0)
+        return KV_OK;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
+    cfg.gridDim = dim3(p.grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, fn, tmK, tmV, a) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, p.fn, p.tmK, p.tmV, p.a) != cudaSuccess)
         return KV_ERR_CUDA;
 
-    if (!a.fused) {
+    if (!p.a.fused) {
         cudaLaunchConfig_t c2 = {};
-        c2.gridDim = dim3(L.items);
+        c2.gridDim = dim3(p.lay.items);
         c2.blockDim = dim3(128);
         c2.dynamicSmemBytes = 0;
         c2.stream = st;
         c2.attrs = attr;
         c2.numAttrs = 1;
         cudaError_t e;
-        if (dtype == KV_DTYPE_FP16)
-            e = (D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<ElemF16, 64>, a, grid)
-                          : cudaLaunchKernelEx(&c2, combine_kernel<ElemF16, 128>, a, grid);
+        if (p.dtype == KV_DTYPE_FP16)
+            e = (p.D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<ElemF16, 64>, p.a, p.grid)
+                            : cudaLaunchKernelEx(&c2, combine_kernel<ElemF16, 128>, p.a, p.grid);
         else
-            e = (D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<ElemBf16, 64>, a, grid)
-                          : cudaLaunchKernelEx(&c2, combine_kernel<ElemBf16, 128>, a, grid);
+            e = (p.D == 64) ? cudaLaunchKernelEx(&c2, combine_kernel<ElemBf16, 64>, p.a, p.grid)
+                            : cudaLaunchKernelEx(&c2, combine_kernel<ElemBf16, 128>, p.a, p.grid);
         if (e != cudaSuccess)
             return KV_ERR_CUDA;
     }
     return KV_OK;
+}
+
+}  // namespace
+
+extern "C" size_t paged_attention_workspace_size(int B, int Hq, int Hkv, int D)
+{
+    return paged_attention_workspace_size_layers(B, Hq, Hkv, D, 1);
+}
+
+extern "C" size_t paged_attention_workspace_size_layers(int B, int Hq, int Hkv, int D, int num_layers)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return 0;
+    Layout lay;
+    if (!make_layout(B, Hq, Hkv, D, num_layers, device_sm_count(dev), &lay))
+        return 0;
+    return lay.bytes;
+}
+
+extern "C" kv_status paged_attention_workspace_init(void *workspace, size_t workspace_bytes, kv_stream_t stream)
+{
+    pkv_host::NvtxRange nvtx_range("paged_attention_workspace_init");
+    if (!workspace || workspace_bytes == 0)
+        return KV_ERR_ARG;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? KV_OK
+               : KV_ERR_CUDA;
 }
 
 extern "C" kv_status paged_attention_decode(void *out, const void *q, const void *k_cache, const void *v_cache,
@@ -1645,8 +1761,12 @@ extern "C" kv_status paged_attention_decode(void *out, const void *q, const void
                                             int D, float scale, int dtype, void *workspace,
                                             size_t workspace_bytes, kv_stream_t stream)
 {
-    return decode_impl(out, q, nullptr, nullptr, k_cache, v_cache, nullptr, block_tables, max_blocks_per_seq,
-                       context_lens, B, num_blocks, Hq, Hkv, D, scale, dtype, workspace, workspace_bytes, stream);
+    pkv_host::NvtxRange nvtx_range("paged_attention_decode");
+    DecodePlan p;
+    const kv_status r = plan_decode(&p, out, q, nullptr, nullptr, k_cache, v_cache, 0, 1, nullptr, block_tables,
+                                    max_blocks_per_seq, context_lens, B, num_blocks, Hq, Hkv, D, scale, dtype,
+                                    workspace, workspace_bytes);
+    return r != KV_OK ? r : launch_decode(p, stream);
 }
 
 extern "C" kv_status paged_attention_decode_append(void *out, const void *q, const void *k_new, const void *v_new,
@@ -1656,11 +1776,36 @@ extern "C" kv_status paged_attention_decode_append(void *out, const void *q, con
                                                    int Hkv, int D, float scale, int dtype, void *workspace,
                                                    size_t workspace_bytes, kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("paged_attention_decode_append");
     if (!k_new || !v_new || !slot_mapping || misaligned(k_new, 16) || misaligned(v_new, 16) ||
         misaligned(slot_mapping, 8))
         return KV_ERR_ARG;
-    return decode_impl(out, q, k_new, v_new, k_cache, v_cache, slot_mapping, block_tables, max_blocks_per_seq,
-                       context_lens, B, num_blocks, Hq, Hkv, D, scale, dtype, workspace, workspace_bytes, stream);
+    DecodePlan p;
+    const kv_status r = plan_decode(&p, out, q, k_new, v_new, k_cache, v_cache, 0, 1, slot_mapping, block_tables,
+                                    max_blocks_per_seq, context_lens, B, num_blocks, Hq, Hkv, D, scale, dtype,
+                                    workspace, workspace_bytes);
+    return r != KV_OK ? r : launch_decode(p, stream);
+}
+
+extern "C" kv_status paged_attention_decode_layers(void *out, const void *q, const void *k_new, const void *v_new,
+                                                   void *k_cache, void *v_cache, size_t cache_layer_stride,
+                                                   int num_layers, const int64_t *slot_mapping,
+                                                   const int32_t *block_tables, int max_blocks_per_seq,
+                                                   const int32_t *context_lens, int B, int num_blocks, int Hq,
+                                                   int Hkv, int D, float scale, int dtype, void *workspace,
+                                                   size_t workspace_bytes, kv_stream_t stream)
+{
+    pkv_host::NvtxRange nvtx_range("paged_attention_decode_layers");
+    const bool append = k_new != nullptr;
+    if (append != (v_new != nullptr) || append != (slot_mapping != nullptr))
+        return KV_ERR_ARG;  // the new rows and their slots come together, or not at all
+    if (append && (misaligned(k_new, 16) || misaligned(v_new, 16) || misaligned(slot_mapping, 8)))
+        return KV_ERR_ARG;
+    DecodePlan p;
+    const kv_status r = plan_decode(&p, out, q, k_new, v_new, k_cache, v_cache, cache_layer_stride, num_layers,
+                                    slot_mapping, block_tables, max_blocks_per_seq, context_lens, B, num_blocks, Hq,
+                                    Hkv, D, scale, dtype, workspace, workspace_bytes);
+    return r != KV_OK ? r : launch_decode(p, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -1674,8 +1819,53 @@ extern "C" kv_status paged_attention_decode_append(void *out, const void *q, con
 // ---------------------------------------------------------------------------
 namespace {
 constexpr size_t kNoAllocScratchBytes = KV_NOALLOC_SCRATCH_BYTES;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CUcontext current_context()
+{
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    });
+    CUcontext c = nullptr;
+    if (!fn || fn(&c) != CUDA_SUCCESS)
+        return nullptr;
+    return c;
 }
+}  // namespace
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+// The array's device address on device `dev` (current). In host code the
+// array's name is a host-side stand-in, not a device address, so it is looked
+// up with cudaGetSymbolAddress: once per device, and again if the device's
+// current context changed since (a context created anew loads the module anew).
+void *noalloc_scratch(int dev)
+{
+    struct Entry {
+        CUcontext ctx;
+        void *ptr;
+    };
+    static std::mutex mu;
+    static Entry cache[kMaxDevices];
+    std::lock_guard<std::mutex> lock(mu);
+    CUcontext ctx = current_context();
+    if (ctx != nullptr && cache[dev].ctx == ctx && cache[dev].ptr != nullptr)
+        return cache[dev].ptr;
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+        return nullptr;
+    cache[dev].ctx = current_context();  // the runtime has made the device's context current by now
+    cache[dev].ptr = p;
+    return p;
+}
+}  // namespace
 
 extern "C" kv_status paged_attention_decode_noalloc(void *out, const void *q, const void *k_cache,
                                                     const void *v_cache, const int32_t *block_tables,
@@ -1683,43 +1873,31 @@ extern "C" kv_status paged_attention_decode_noalloc(void *out, const void *q, co
                                                     int num_blocks, int Hq, int Hkv, int D, float scale, int dtype,
                                                     kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("paged_attention_decode_noalloc");
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return KV_ERR_CUDA;
-    // In host code the array's name is not a device address: look the address
-    // up once per device, with that device current.
-    static std::atomic<void *> scratch[kMaxDevices];
-    static std::mutex setup_mu;
-    void *ws = scratch[dev].load();
-    if (!ws) {
-        std::lock_guard<std::mutex> lock(setup_mu);
-        ws = scratch[dev].load();
-        if (!ws) {
-            void *p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
-                return KV_ERR_CUDA;
-            scratch[dev].store(p);
-            ws = p;
-        }
-    }
-    Layout L;
-    if (!make_layout(B, Hq, Hkv, D, device_sm_count(dev), &L))
-        return KV_ERR_ARG;
-    if (L.bytes > kNoAllocScratchBytes)
-        return KV_ERR_ARG;  // more split-K scratch than the fixed array holds
-    if (B == 0)
-        return KV_OK;
+    void *ws = noalloc_scratch(dev);
+    if (!ws)
+        return KV_ERR_CUDA;
+    // every check first (a scratch larger than the array is KV_ERR_ARG): a rejected call touches nothing
+    DecodePlan p;
+    const kv_status r = plan_decode(&p, out, q, nullptr, nullptr, k_cache, v_cache, 0, 1, nullptr, block_tables,
+                                    max_blocks_per_seq, context_lens, B, num_blocks, Hq, Hkv, D, scale, dtype, ws,
+                                    kNoAllocScratchBytes);
+    if (r != KV_OK || p.grid == 0)
+        return r;
     // The array keeps the previous call's contents: the status word and the
     // per-item counters must start at zero.
-    if (cudaMemsetAsync(ws, 0, L.off_ml, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (cudaMemsetAsync(ws, 0, p.lay.off_ml, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
         return KV_ERR_CUDA;
-    return paged_attention_decode(out, q, k_cache, v_cache, block_tables, max_blocks_per_seq, context_lens, B,
-                                  num_blocks, Hq, Hkv, D, scale, dtype, ws, kNoAllocScratchBytes, stream);
+    return launch_decode(p, stream);
 }
 
 extern "C" kv_status paged_attention_read_status(const void *workspace, int32_t *status_out, int clear,
                                                  kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("paged_attention_read_status");
     if (!workspace || !status_out)
         return KV_ERR_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1785,6 +1963,16 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_slow_softmax.store(value);
         return KV_OK;
+    case KV_OPT_OUT_F32:
+        if (value < 0 || value > 1)
+            return KV_ERR_ARG;
+        g_opt_out_f32.store(value);
+        return KV_OK;
+    case KV_OPT_L2_POLICY:
+        if (value < 0 || value > 3)
+            return KV_ERR_ARG;
+        g_opt_l2_policy.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -1813,6 +2001,10 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_drop_load.load();
     case KV_OPT_TEST_SLOW_SOFTMAX:
         return g_opt_slow_softmax.load();
+    case KV_OPT_OUT_F32:
+        return g_opt_out_f32.load();
+    case KV_OPT_L2_POLICY:
+        return g_opt_l2_policy.load();
     default:
         return -1;
     }
@@ -1821,3 +2013,4 @@ extern "C" int kv_decode_get_option(int key)
 // The prefill path switch and test hook (read by prefill.cu).
 int pkv_prefill_path() { return g_opt_prefill_path.load(); }
 int pkv_prefill_slow_softmax() { return g_opt_slow_softmax.load(); }
+int pkv_out_f32() { return g_opt_out_f32.load(); }

@@ -11,6 +11,7 @@
 // are in use. Free ids sit on a stack (most recently freed first), reference
 // counts in a flat array. Every call validates its whole request before
 // changing anything, so a failed call leaves the pool as it was.
+#include "nvtx_range.h"
 #include "pagedkv.h"
 
 #include <mutex>
@@ -138,6 +139,7 @@ extern "C" int kv_pool_refcount(const void *pool, int32_t id)
 extern "C" kv_status kv_pool_append_slots(void *pool, int32_t *block_tables, int W, int32_t *context_lens, int B,
                                           int64_t *slot_mapping_out)
 {
+    pkv_host::NvtxRange nvtx_range("kv_pool_append_slots");
     if (!pool || B < 0 || W < 1 || (B > 0 && (!block_tables || !context_lens || !slot_mapping_out)))
         return KV_ERR_ARG;
     BlockPool *p = as_pool(pool);
@@ -198,6 +200,7 @@ extern "C" kv_status kv_pool_append_slots_cow(void *pool, int32_t *block_tables,
                                               int64_t *slot_mapping_out, int32_t *copy_src_out,
                                               int32_t *copy_dst_out, int *n_copies_out)
 {
+    pkv_host::NvtxRange nvtx_range("kv_pool_append_slots_cow");
     if (!pool || B < 0 || W < 1 || !n_copies_out ||
         (B > 0 && (!block_tables || !context_lens || !slot_mapping_out || !copy_src_out || !copy_dst_out)))
         return KV_ERR_ARG;

@@ -24,6 +24,7 @@
 // base 2 (one rescale of O per stage), then O[16 x D] += P V with P rounded to
 // the element type.
 #include "pkv_device.cuh"
+#include "nvtx_range.h"
 #include "pagedkv.h"
 #include "tma_host.h"
 
@@ -63,6 +64,7 @@ struct PrefillArgs {
     int B, W, Hq, Hkv, group, num_blocks, max_tiles, max_query_len;
     float scale_log2;
     int slow_softmax;  // test hook: the tcgen05 path's first softmax warp hands over its first P late
+    int out_f32;       // out holds fp32 numbers (a debug switch: the result before rounding)
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
@@ -356,8 +358,22 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
     lB += __shfl_xor_sync(kFullMask, lB, 1);
     lB += __shfl_xor_sync(kFullMask, lB, 2);
     const float iA = 1.f / lA, iB = 1.f / lB;
-    uint32_t *outA = reinterpret_cast<uint32_t *>(a.out + (static_cast<size_t>(q0 + tokA) * a.Hq + j * g + hA) * D);
-    uint32_t *outB = reinterpret_cast<uint32_t *>(a.out + (static_cast<size_t>(q0 + tokB) * a.Hq + j * g + hB) * D);
+    const size_t offA = (static_cast<size_t>(q0 + tokA) * a.Hq + j * g + hA) * D;
+    const size_t offB = (static_cast<size_t>(q0 + tokB) * a.Hq + j * g + hB) * D;
+    if (a.out_f32) {
+        float2 *outA = reinterpret_cast<float2 *>(reinterpret_cast<float *>(a.out) + offA);
+        float2 *outB = reinterpret_cast<float2 *>(reinterpret_cast<float *>(a.out) + offB);
+#pragma unroll
+        for (int dt = 0; dt < 2 * kK; ++dt) {
+            if (okA)
+                outA[dt * 4 + cq] = make_float2(o[dt][0] * iA, o[dt][1] * iA);
+            if (okB)
+                outB[dt * 4 + cq] = make_float2(o[dt][2] * iB, o[dt][3] * iB);
+        }
+        return;
+    }
+    uint32_t *outA = reinterpret_cast<uint32_t *>(a.out + offA);
+    uint32_t *outB = reinterpret_cast<uint32_t *>(a.out + offB);
 #pragma unroll
     for (int dt = 0; dt < 2 * kK; ++dt) {
         if (okA)
@@ -805,12 +821,24 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
         if (__all_sync(kFullMask, good && mbar_wait_bounded(o_done, 0, abort_flag))) {
             tcgen05_after_sync();
             const float inv = 1.f / l;
-            uint16_t *dst = a.out + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D;
+            const size_t row = (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D;
+            uint16_t *dst = a.out + row;
             uint32_t v[16];
 #pragma unroll 1
             for (int q4 = 0; q4 < D / 16; ++q4) {
                 tmem_ld16(lane_base + G::kOCol + q4 * 16, v);
                 tmem_wait_ld();
+                if (a.out_f32) {
+                    if (ok) {
+                        float4 *f = reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + row + q4 * 16);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            f[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
+                                               __uint_as_float(v[4 * i + 2]) * inv,
+                                               __uint_as_float(v[4 * i + 3]) * inv);
+                    }
+                    continue;
+                }
                 uint4 o0, o1;
                 o0.x = E::pack(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
                 o0.y = E::pack(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv);
@@ -846,6 +874,7 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
 // KV_OPT_PREFILL_PATH and KV_OPT_TEST_SLOW_SOFTMAX, kept with the other switches in decode.cu
 int pkv_prefill_path();
 int pkv_prefill_slow_softmax();
+int pkv_out_f32();
 
 namespace {
 
@@ -901,6 +930,7 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
                                              int max_query_len, int num_blocks, int Hq, int Hkv, int D, float scale,
                                              int dtype, int32_t *error_flag, kv_stream_t stream)
 {
+    pkv_host::NvtxRange nvtx_range("paged_attention_prefill");
     using namespace pkv::prefill;
     if ((dtype != KV_DTYPE_BF16 && dtype != KV_DTYPE_FP16) || B < 0 || B > 65535 || max_query_len < 0 ||
         max_blocks_per_seq < 1 || num_blocks < 1 || Hq < 1 || Hkv < 1 || Hkv > 65535 || Hq % Hkv != 0 ||
@@ -948,6 +978,7 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
     a.max_query_len = max_query_len;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.slow_softmax = pkv_prefill_slow_softmax();
+    a.out_f32 = pkv_out_f32();
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));

@@ -50,4 +50,27 @@ inline bool make_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, i
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A stack of `layers` such caches, layer l starting layer_stride_bytes * l
+// after the first, as a 5-D map (column, row, kv head, block, layer) with the
+// same box and one layer per box.
+inline bool make_layered_cache_map(CUtensorMap *tm, const void *cache, int num_blocks, int Hkv, int D, int hg,
+                                   int dtype, int layers, unsigned long long layer_stride_bytes)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || layers < 1)
+        return false;
+    const cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), 16, static_cast<cuuint64_t>(Hkv),
+                                static_cast<cuuint64_t>(num_blocks), static_cast<cuuint64_t>(layers)};
+    const cuuint64_t strides[4] = {static_cast<cuuint64_t>(Hkv) * D * 2, static_cast<cuuint64_t>(D) * 2,
+                                   static_cast<cuuint64_t>(16) * Hkv * D * 2,
+                                   static_cast<cuuint64_t>(layer_stride_bytes)};
+    const cuuint32_t box[5] = {64, 16, static_cast<cuuint32_t>(hg), 1, 1};
+    const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUtensorMapDataType dt =
+        dtype == KV_DTYPE_FP16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    return enc(tm, dt, 5, const_cast<void *>(cache), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace pkv_host

@@ -205,6 +205,22 @@ def make_layer_cache(num_blocks: int, Hkv: int, D: int, gen: torch.Generator, de
     return k, v
 
 
+def make_stacked_caches(n_layers: int, num_blocks: int, Hkv: int, D: int, gen: torch.Generator, device,
+                        dtype=torch.bfloat16, spare_blocks: int = 0):
+    """Every layer's K and V pools in two tensors [n_layers, num_blocks + spare_blocks, 16, Hkv, D], drawn in the
+    order of n_layers calls of make_layer_cache (the same values); the spare blocks, if any, hold zeros and sit
+    after each layer's pool, so layer l's [:num_blocks] views lie a larger stride apart."""
+    shape = (n_layers, num_blocks + spare_blocks, BLOCK_TOKENS, Hkv, D)
+    k = torch.zeros(shape, dtype=dtype, device=device)
+    v = torch.zeros(shape, dtype=dtype, device=device)
+    for layer in range(n_layers):
+        kl, vl = make_layer_cache(num_blocks, Hkv, D, gen, device, dtype)
+        k[layer, :num_blocks].copy_(kl)
+        v[layer, :num_blocks].copy_(vl)
+        del kl, vl
+    return k[:, :num_blocks], v[:, :num_blocks]
+
+
 def make_step_inputs(cfg: DecodeConfig, gen: torch.Generator, device, n_layers=None):
     """Per-layer q [B,Hq,D] and new-token K/V [B,Hkv,D], all of the config's element type."""
     L = cfg.n_layers if n_layers is None else n_layers

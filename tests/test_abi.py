@@ -3,6 +3,7 @@ import ctypes
 import os
 import re
 import subprocess
+import sys
 
 import pytest
 
@@ -64,7 +65,9 @@ def test_option_ranges_need_no_gpu(pkv):
     cases = {pkv.KV_OPT_PREFILL_PATH: ([0, 1, 2], [-1, 3]),
              pkv.KV_OPT_TEST_SLOW_SOFTMAX: ([0, 1], [-1, 2]),
              pkv.KV_OPT_TEST_DROP_LOAD: ([0, 5], [-1]),
-             pkv.KV_OPT_ITEM_COST: ([-1, 0, 64], [-2, 65])}
+             pkv.KV_OPT_ITEM_COST: ([-1, 0, 64], [-2, 65]),
+             pkv.KV_OPT_OUT_F32: ([0, 1], [-1, 2]),
+             pkv.KV_OPT_L2_POLICY: ([0, 1, 2, 3], [-1, 4])}
     for key, (good, bad) in cases.items():
         before = lib.kv_decode_get_option(key)
         for v in good:
@@ -137,3 +140,40 @@ def test_a_plain_c_program_uses_the_library(pkv, tmp_path):
                     "-L", libdir, "-lpagedkv", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "c client ok", (out.returncode, out.stdout, out.stderr)
+
+
+def test_importing_the_package_maps_no_library():
+    """The package's input generator can be imported by code that must not load the CUDA library (the oracle's
+    timed arm): the library is mapped by the first call that needs it."""
+    code = ("import sys; sys.path.insert(0, %r); import paged_kv_cache_470_b200 as p; "
+            "from paged_kv_cache_470_b200 import workloads; "
+            "maps = open('/proc/self/maps').read(); assert 'libpagedkv' not in maps, 'mapped at import'; "
+            "p.load(); assert 'libpagedkv' in open('/proc/self/maps').read(); print('ok')") % ROOT
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stderr
+
+
+def test_multi_layer_checks_need_no_gpu(pkv):
+    """paged_attention_decode_layers refuses bad layer arguments on the host, before any CUDA call."""
+    lib = ctypes.CDLL(pkv.LIB_PATH)
+    f = lib.paged_attention_decode_layers
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [P, P, P, P, P, P, ctypes.c_size_t, I, P, P, I, P, I, I, I, I, I, ctypes.c_float, I, P,
+                  ctypes.c_size_t, P]
+    f.restype = I
+    fake = 1 << 20   # an aligned non-null address; nothing is dereferenced before the checks fail
+    good = dict(out=fake, q=fake, kn=None, vn=None, kc=fake, vc=fake, stride=4 * 16 * 4 * 64, L=2, slots=None,
+                tables=fake, W=4, lens=fake, B=3, nb=4, Hq=8, Hkv=4, D=64, scale=0.1, dtype=0, ws=fake,
+                wsb=1 << 30)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return f(a["out"], a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["stride"], a["L"], a["slots"],
+                 a["tables"], a["W"], a["lens"], a["B"], a["nb"], a["Hq"], a["Hkv"], a["D"], a["scale"],
+                 a["dtype"], a["ws"], a["wsb"], None)
+    assert call(L=0) == pkv.KV_ERR_ARG                           # no layer
+    assert call(stride=4 * 16 * 4 * 64 - 8) == pkv.KV_ERR_ARG    # layers would overlap
+    assert call(stride=4 * 16 * 4 * 64 + 4) == pkv.KV_ERR_ARG    # not a multiple of 16 bytes
+    assert call(kn=fake) == pkv.KV_ERR_ARG                       # new K rows without V rows and slots
+    assert call(kn=fake, vn=fake, slots=fake + 4) == pkv.KV_ERR_ARG   # misaligned slots
+    assert call(B=0) == pkv.KV_OK                                # nothing to do

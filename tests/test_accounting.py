@@ -87,14 +87,18 @@ def test_profiled_traffic_needs_the_current_source_and_workload(bench, tmp_path,
     cfg = workloads.WORKLOADS[2]
     monkeypatch.setattr(bench, "PROFILE_DIR", str(tmp_path))
 
-    def write(h, cid=2, elem="bf16"):
-        (tmp_path / "p.txt").write_text(f"config_id: {cid}\nelem: {elem}\ndecode.cu sha256[:16]: {h}\n"
-                                        f"dram_bytes_per_launch: 123456\n")
+    def write(h, cid=2, elem="bf16", launch="per_layer"):
+        (tmp_path / "p.txt").write_text(f"config_id: {cid}\nelem: {elem}\nlaunch: {launch}\n"
+                                        f"decode.cu sha256[:16]: {h}\n"
+                                        f"dram_bytes_per_launch: 123456\ndram_bytes_per_layer: 1000\n")
     write(src)
-    assert bench.profiled_traffic(cfg) == 123456.0
+    assert bench.profiled_traffic(cfg, "per_layer") == 123456.0
+    assert bench.profiled_traffic(cfg, "layers") is None      # a capture of the other kind of launch
+    write(src, launch="layers")
+    assert bench.profiled_traffic(cfg, "layers") == 1000.0 * cfg.n_layers   # scaled to the workload's layers
     write("0" * 16)                                           # a capture of another kernel source
-    assert bench.profiled_traffic(cfg) is None
+    assert bench.profiled_traffic(cfg, "per_layer") is None
     write(src, cid=3)                                         # another workload
-    assert bench.profiled_traffic(cfg) is None
+    assert bench.profiled_traffic(cfg, "per_layer") is None
     write(src, elem="fp16")                                   # another element type
-    assert bench.profiled_traffic(cfg) is None
+    assert bench.profiled_traffic(cfg, "per_layer") is None

@@ -67,3 +67,22 @@ def test_reference_arm_under_torchrun_prints_one_line(tmp_path):
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["value"] > 0 and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_maps_no_product_library_and_shares_the_config():
+    """The oracle's arm loads the oracle's library only, and its `config` is the GPU line's."""
+    code = ("import sys, json, io, contextlib; sys.path.insert(0, %r); import bench\n"
+            "buf = io.StringIO()\n"
+            "with contextlib.redirect_stdout(buf):\n"
+            "    bench.main(['--impl', 'reference', '--steps', '1', '--warmup', '3', '--config', '1',"
+            " '--reference-budget', '0.5'])\n"
+            "maps = open('/proc/self/maps').read()\n"
+            "assert 'libpagedkv' not in maps, 'product library mapped'\n"
+            "line = json.loads([l for l in buf.getvalue().splitlines() if l.startswith('{')][0])\n"
+            "from paged_kv_cache_470_b200 import workloads\n"
+            "cfg = workloads.WORKLOADS[1]\n"
+            "assert line['config'] == bench.config_record(cfg, workloads.draw_layout(cfg), 1), line['config']\n"
+            "print('ok')") % ROOT
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout + r.stderr

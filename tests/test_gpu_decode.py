@@ -281,3 +281,96 @@ def test_fused_append_rejects_a_slot_that_is_not_the_last_token(pkv, oracle_mod,
     pkv.paged_attention_decode_append(out, case.q[0], case.k_new[0], case.v_new[0], case.k[0], case.v[0],
                                       slots_none, case.tables, case.lens, cfg.scale, ws)
     assert pkv.read_status(ws) == 0
+
+
+# ---------------------------------------------------------------------------
+# several layers in one launch (paged_attention_decode_layers)
+# ---------------------------------------------------------------------------
+def run_layers_and_check(pkv, oracle_mod, case, layers=None, append=True, what=""):
+    """One multi-layer launch over all of the case's layers; the listed layers against the oracle (append
+    bit-exact, attention within tolerance)."""
+    cfg, L = case.cfg, case.n_layers
+    check = list(range(L)) if layers is None else layers
+    host = {layer: case.host_inputs(layer) for layer in check}
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D, num_layers=L)
+    out = torch.full_like(case.q, float("nan"))
+    kw = dict(k_new=case.k_new, v_new=case.v_new, slot_mapping=case.slots) if append else {}
+    pkv.paged_attention_decode_layers(out, case.q, case.k_all, case.v_all, case.tables, case.lens, cfg.scale, ws,
+                                      **kw)
+    torch.cuda.synchronize()
+    assert pkv.read_status(ws) == 0
+    for layer in check:
+        q, k, v, kn, vn = host[layer]
+        if append:
+            k2, v2, ref = oracle_step(oracle_mod, case, layer, host[layer])
+            assert np.array_equal(bf16_bits_np(case.k[layer]), k2), f"{what} layer {layer}: K append not bit-exact"
+            assert np.array_equal(bf16_bits_np(case.v[layer]), v2), f"{what} layer {layer}: V append not bit-exact"
+        else:
+            assert torch.equal(case.k[layer].cpu(), k) and torch.equal(case.v[layer].cpu(), v)
+            ref = oracle_mod.paged_attention_decode(q, k, v, case.layout.block_tables.numpy(),
+                                                    case.layout.context_lens.numpy(), cfg.scale, dtype=cfg.elem)
+        compare(out[layer], ref, f"{what} layer {layer} (one launch for {L} layers)")
+    return out
+
+
+@pytest.mark.parametrize("append", [True, False])
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_layers_in_one_launch(pkv, oracle_mod, cuda_device, path, append):
+    pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
+    cfg = workloads.small_config(2, batch=9, ctx_lo=1, ctx_hi=700, W=48)
+    case = Case(cfg, cuda_device, n_layers=5)
+    run_layers_and_check(pkv, oracle_mod, case, append=append, what=f"layers/{path}")
+
+
+@pytest.mark.parametrize("cid", [2, 3])
+@pytest.mark.parametrize("grid,min_chunk,combine", [(1, 1, 0), (3, 1, 0), (7, 2, 1), (296, 1, 0), (0, 1, 1)])
+def test_layers_split_everywhere(pkv, oracle_mod, cuda_device, cid, grid, min_chunk, combine):
+    """Grids from one CTA (one piece per item, every layer in it) to twice the SMs; CTA ranges start and end in
+    different layers; the merge in the last CTA or in the combine kernel."""
+    pkv.set_option(pkv.KV_OPT_GRID, grid)
+    pkv.set_option(pkv.KV_OPT_MIN_CHUNK, min_chunk)
+    pkv.set_option(pkv.KV_OPT_COMBINE, combine)
+    cfg = workloads.small_config(cid, batch=6, ctx_lo=1, ctx_hi=900, W=64)
+    case = Case(cfg, cuda_device, n_layers=4)
+    run_layers_and_check(pkv, oracle_mod, case, what=f"layers cfg{cid} grid {grid} combine {combine}")
+
+
+def test_layers_with_a_stride_larger_than_a_pool_and_empty_sequences(pkv, oracle_mod, cuda_device):
+    cfg = workloads.small_config(3, batch=7, W=40)
+    case = Case(cfg, cuda_device, n_layers=3, lens=[0, 1, 16, 17, 0, 640, 33], spare_blocks=5)
+    assert case.k_all.stride(0) > case.k_all[0].numel()
+    run_layers_and_check(pkv, oracle_mod, case, what="layers, strided pools")
+
+
+def test_layers_one_layer_equals_the_per_layer_call(pkv, cuda_device):
+    """num_layers = 1 is the per-layer call: the same grid and split, so the same bits."""
+    cfg = workloads.small_config(2, batch=20, ctx_lo=1, ctx_hi=2000)
+    case = Case(cfg, cuda_device, n_layers=1)
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
+    a = torch.empty_like(case.q[:1])
+    pkv.paged_attention_decode_layers(a, case.q[:1], case.k_all, case.v_all, case.tables, case.lens, cfg.scale, ws)
+    b = torch.empty_like(case.q[0])
+    pkv.paged_attention_decode(b, case.q[0], case.k[0], case.v[0], case.tables, case.lens, cfg.scale, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b)
+
+
+def test_layers_workspace_too_small_is_refused(pkv, cuda_device):
+    cfg = workloads.small_config(2, batch=8, ctx_lo=1, ctx_hi=300, W=32)
+    case = Case(cfg, cuda_device, n_layers=3)
+    ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D, num_layers=2)
+    out = torch.empty_like(case.q)
+    with pytest.raises(pkv.KVError):
+        pkv.paged_attention_decode_layers(out, case.q, case.k_all, case.v_all, case.tables, case.lens, cfg.scale, ws)
+
+
+@pytest.mark.parametrize("cid", [2, 3, 4, 5])
+def test_full_size_layers_in_one_launch(pkv, oracle_mod, cuda_device, cid):
+    """The bench's multi-layer step at full size: every layer of the 0.5B and 70B-mix workloads in one launch,
+    four layers of the larger ones (memory of the oracle's host copies); first, last and one random layer
+    checked."""
+    cfg = workloads.WORKLOADS[cid]
+    L = cfg.n_layers if cid in (2, 5) else 4
+    case = Case(cfg, cuda_device, n_layers=L)
+    layers = sorted({0, L - 1, random.Random(cid).randrange(L)})
+    run_layers_and_check(pkv, oracle_mod, case, layers=layers, what=f"config {cid}")
