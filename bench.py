@@ -746,6 +746,8 @@ def run_ours(args, world, rank, local):
         pkv.set_option(pkv.KV_OPT_HEAD_GROUP, args.head_group)
     if args.item_cost:
         pkv.set_option(pkv.KV_OPT_ITEM_COST, args.item_cost)
+    if args.producer_lanes:
+        pkv.set_option(pkv.KV_OPT_PRODUCER_LANES, args.producer_lanes)
     if args.l2_policy:
         pkv.set_option(pkv.KV_OPT_L2_POLICY, {"first": 1, "normal": 2, "last": 3}[args.l2_policy])
     if args.profile_step:
@@ -871,6 +873,8 @@ def main(argv=None):
     ap.add_argument("--head-group", type=int, default=0, help="kv heads per work unit (0: auto)")
     ap.add_argument("--item-cost", type=int, default=0,
                     help="work positions charged per work item when dividing work between CTAs (0 auto, -1 none)")
+    ap.add_argument("--producer-lanes", type=int, default=0, choices=[0, 1, 2, 4, 8],
+                    help="lanes of the decode producer warp that issue tile loads (0: the library's choice)")
     ap.add_argument("--l2-policy", choices=["first", "normal", "last"], default=None,
                     help="L2 priority of the decode kernels' K/V tile loads (default: the library's)")
     ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16", help="element type of q, K, V and out")

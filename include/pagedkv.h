@@ -312,8 +312,12 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *   KV_OPT_GRID:      0 auto (CTAs resident on all SMs), n > 0 launch n CTAs
  *                     (n is capped by what the workspace was sized for)
  *   KV_OPT_MIN_CHUNK: 0 auto, n > 0 minimum work positions per CTA
- *   KV_OPT_PRODUCER_LANES: 0 auto, 1/2/4/8 lanes of the producer warp that
- *                     issue tile loads
+ *   KV_OPT_PRODUCER_LANES: 0 auto (2, or 4 with one kv head per unit),
+ *                     1/2/4/8 lanes of the producer warp that issue tile
+ *                     loads. The ring's stage count is rounded down to a
+ *                     multiple of the lanes; a value that leaves fewer stages
+ *                     than lanes (8 with D = 128) makes the decode calls
+ *                     return KV_ERR_ARG.
  *   KV_OPT_HEAD_GROUP: 0 auto (4 if it divides Hkv, else 2 or 1), or 1/2/4 kv
  *                     heads per work unit when it divides Hkv. It changes
  *                     paged_attention_workspace_size: set it before sizing.
@@ -344,8 +348,10 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     result before any rounding to the element type. The
  *                     other arguments keep their element type.
  *   KV_OPT_L2_POLICY: L2 priority of the decode kernels' K/V tile loads: 0
- *                     auto (evict first), 1 evict first, 2 evict normal,
- *                     3 evict last.
+ *                     auto (evict first for one layer; evict normal for a
+ *                     multi-layer launch, where blocks that several sequences
+ *                     share are re-read far apart), 1 evict first, 2 evict
+ *                     normal, 3 evict last.
  * Kernels are launched with programmatic dependent launch. q, k_new, v_new,
  * the caches, the workspace and out are touched only after the previous kernel
  * in the stream has completed; block_tables and context_lens are read before

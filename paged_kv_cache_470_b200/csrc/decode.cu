@@ -1624,7 +1624,7 @@ kv_status plan_decode(DecodePlan *p, void *out, const void *q, const void *k_new
     const int streams = kConsumerWarps / hg;
     int lanes = g_opt_prod_lanes.load();
     if (lanes <= 0)
-        lanes = hg >= 4 ? 1 : (hg == 2 ? 2 : 4);
+        lanes = hg >= 2 ? 2 : 4;  // one lane cannot issue a D = 64 unit's two boxes as fast as 148 SMs drain them
     const int stage_bytes = 2 * tiles * hg * kHeadTileBytes;
     const int unit_of = streams > lanes ? streams : lanes;
     const int ring = D == 64 ? Geo<64>::kRingBytes : Geo<128>::kRingBytes;
@@ -1670,7 +1670,10 @@ kv_status plan_decode(DecodePlan *p, void *out, const void *q, const void *k_new
     a.min_chunk = mc > 0 ? mc : kDefaultMinChunk;
     a.item_cost = cost;
     a.drop_unit = g_opt_drop_load.load() - 1;
-    a.l2_policy = g_opt_l2_policy.load() == 0 ? 1 : g_opt_l2_policy.load();
+    // Auto: a single layer streams its K/V once, so evict-first keeps the rest of L2 for other data; a
+    // multi-layer launch has every layer in flight at once, and blocks shared by several sequences (a common
+    // prefix) are re-read far enough apart that evict-first loses them: evict-normal keeps them.
+    a.l2_policy = g_opt_l2_policy.load() != 0 ? g_opt_l2_policy.load() : (layers > 1 ? 2 : 1);
     a.fused = g_opt_combine.load() == 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.append = k_new != nullptr ? 1 : 0;
