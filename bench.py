@@ -665,10 +665,17 @@ def measure_config(args, cfg, device, world, rank, headline):
     step_bytes0 = cfg_rec["algorithmic_bytes_per_step"]
     combine = pkv.get_option(pkv.KV_OPT_COMBINE) == 1
     res = {}
+    early_default = pkv.get_option(pkv.KV_OPT_EARLY_LOADS)
     for name, fn, launches in (("layers", wl.step, 1 + combine),
                                ("per_layer", wl.step_per_layer,
                                 cfg.n_layers * ((1 if wl.fused else 2) + combine))):
+        # Per layer, the launch before layer l's is layer l-1's (its own cache) or, for layer 0, the previous
+        # step's last layer: none writes the caches that the launch reads, so the per-layer step may start its
+        # first tile loads early. The multi-layer launch follows the previous step's launch over the same caches
+        # (it appended rows to them), so it may not.
+        pkv.set_option(pkv.KV_OPT_EARLY_LOADS, 1 if (name == "per_layer" and wl.fused) else early_default)
         graph = capture(fn)
+        pkv.set_option(pkv.KV_OPT_EARLY_LOADS, early_default)
         for _ in range(args.warmup):
             graph.replay()
         torch.cuda.synchronize()
@@ -699,8 +706,9 @@ def measure_config(args, cfg, device, world, rank, headline):
         "clocks": ml["clocks"],
         "device_status": ml["status"],
         "per_layer": {
-            "api": ("paged_attention_decode_append" if wl.fused else "kv_cache_append + paged_attention_decode")
-                   + " per layer, in a CUDA graph with programmatic dependent launch",
+            "api": ("paged_attention_decode_append per layer with KV_OPT_EARLY_LOADS (the launch before each "
+                    "reads no cache it writes)" if wl.fused else "kv_cache_append + paged_attention_decode per layer")
+                   + ", in a CUDA graph with programmatic dependent launch",
             "ms_per_step": round(pl["ms"], 5),
             "value": round(pl["step_bytes"] * world / (pl["ms"] * 1e-3) / 1e9, 2),
             "pct_of_nominal_8TBs": round(100 * pl["step_bytes"] / (pl["ms"] * 1e-3) / 1e9 / NOMINAL_HBM_GBS, 2),
@@ -748,6 +756,8 @@ def run_ours(args, world, rank, local):
         pkv.set_option(pkv.KV_OPT_ITEM_COST, args.item_cost)
     if args.producer_lanes:
         pkv.set_option(pkv.KV_OPT_PRODUCER_LANES, args.producer_lanes)
+    if args.early_loads:
+        pkv.set_option(pkv.KV_OPT_EARLY_LOADS, 1)
     if args.l2_policy:
         pkv.set_option(pkv.KV_OPT_L2_POLICY, {"first": 1, "normal": 2, "last": 3}[args.l2_policy])
     if args.profile_step:
@@ -875,6 +885,8 @@ def main(argv=None):
                     help="work positions charged per work item when dividing work between CTAs (0 auto, -1 none)")
     ap.add_argument("--producer-lanes", type=int, default=0, choices=[0, 1, 2, 4, 8],
                     help="lanes of the decode producer warp that issue tile loads (0: the library's choice)")
+    ap.add_argument("--early-loads", action="store_true",
+                    help="KV_OPT_EARLY_LOADS for every call (valid for the per-layer step only)")
     ap.add_argument("--l2-policy", choices=["first", "normal", "last"], default=None,
                     help="L2 priority of the decode kernels' K/V tile loads (default: the library's)")
     ap.add_argument("--dtype", choices=["bf16", "fp16"], default="bf16", help="element type of q, K, V and out")

@@ -352,10 +352,22 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     multi-layer launch, where blocks that several sequences
  *                     share are re-read far apart), 1 evict first, 2 evict
  *                     normal, 3 evict last.
+ *   KV_OPT_EARLY_LOADS: 0 (default) off; 1: the caller promises that, for
+ *                     every decode call in a stream, the kernel launched just
+ *                     before it in that stream does not write the caches the
+ *                     call reads (true for one launch per layer after a
+ *                     projection kernel; false right after kv_cache_append
+ *                     into the same cache, or after a previous step's launch
+ *                     over the same caches). The decode kernels then issue
+ *                     their first ring of K/V tile loads before that kernel
+ *                     has finished (programmatic dependent launch); q, the
+ *                     new rows, out and the workspace still wait for it. With
+ *                     the promise broken, results are unspecified.
  * Kernels are launched with programmatic dependent launch. q, k_new, v_new,
- * the caches, the workspace and out are touched only after the previous kernel
- * in the stream has completed; block_tables and context_lens are read before
- * that, so the kernel launched just before a decode call must not write them.
+ * the caches (unless KV_OPT_EARLY_LOADS is set), the workspace and out are
+ * touched only after the previous kernel in the stream has completed;
+ * block_tables and context_lens are read before that, so the kernel launched
+ * just before a decode call must not write them.
  * Returns KV_ERR_ARG for an unknown key or value.
  */
 #define KV_OPT_COMPUTE 1
@@ -370,6 +382,7 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
 #define KV_OPT_TEST_SLOW_SOFTMAX 10
 #define KV_OPT_OUT_F32 11
 #define KV_OPT_L2_POLICY 12
+#define KV_OPT_EARLY_LOADS 13
 KV_API kv_status kv_decode_set_option(int key, int value);
 KV_API int kv_decode_get_option(int key);
 

@@ -30,6 +30,7 @@ KV_OPT_ITEM_COST, KV_OPT_PREFILL_PATH, KV_OPT_TEST_DROP_LOAD = 7, 8, 9
 KV_OPT_TEST_SLOW_SOFTMAX = 10
 KV_OPT_OUT_F32 = 11
 KV_OPT_L2_POLICY = 12
+KV_OPT_EARLY_LOADS = 13
 COMPUTE_AUTO, COMPUTE_TENSOR_CORES, COMPUTE_CUDA_CORES = 0, 1, 2
 
 _P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t

@@ -128,6 +128,7 @@ struct DecodeArgs {
     int item_cost;       // work positions charged per work item on top of its units
     int drop_unit;       // test hook: CTA 0 never loads its unit with this index (-1: none)
     int l2_policy;       // L2 priority of the K/V tile loads: 1 evict first, 2 evict normal, 3 evict last
+    int early_loads;     // issue the first ring of tile loads before the grid dependency wait (caller's promise)
     int fused;
     float scale_log2;    // scale * log2(e)
     // fused append (append != 0): this step's token of sequence b is k_new/v_new[b],
@@ -1059,14 +1060,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // grid (the tables must not come from the kernel launched just before);
         // the cache is only touched after the wait.
         int bad_first = 0;
-        int blk_first = load_block_ids(a, cur0, min(32, min(cur0.n - cur0.off, count)), lane, &bad_first);
+        const int m_first = min(32, min(cur0.n - cur0.off, count));
+        int blk_first = load_block_ids(a, cur0, m_first, lane, &bad_first);
+        const uint64_t policy = a.l2_policy == 2   ? l2_policy_evict_normal()
+                                : a.l2_policy == 3 ? l2_policy_evict_last()
+                                                   : l2_policy_evict_first();
+        // With the caller's promise that the kernel before this one does not write the caches, the first
+        // ring of tile loads goes out before the wait (lane i: unit i into stage i, their first use), so the
+        // CTA's first data arrives while the previous kernel finishes. q and the new rows still wait.
+        const int pre = a.early_loads ? min(S, m_first) : 0;
+        if (lane < pre && !(lane == a.drop_unit && blockIdx.x == 0)) {
+            const int head0 = (cur0.k / a.hchunks) * a.hg;
+            mbar_arrive_expect_tx(&full[lane], a.stage_bytes);
+            const uint32_t dst = ring + lane * a.stage_bytes;
+#pragma unroll
+            for (int t = 0; t < G::kTiles; ++t)
+                tma_load_5d(dst + t * a.tile_stride, &tmK, t * 64, 0, head0, blk_first, cur0.layer, &full[lane],
+                            policy);
+#pragma unroll
+            for (int t = 0; t < G::kTiles; ++t)
+                tma_load_5d(dst + (G::kTiles + t) * a.tile_stride, &tmV, t * 64, 0, head0, blk_first, cur0.layer,
+                            &full[lane], policy);
+        }
         grid_dependency_wait();
         grid_launch_dependents();
         if (bad_first)
             atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
-        const uint64_t policy = a.l2_policy == 2   ? l2_policy_evict_normal()
-                                : a.l2_policy == 3 ? l2_policy_evict_last()
-                                                   : l2_policy_evict_first();
         const int NL = a.prod_lanes;
         Cursor cur = cur0;
         int u = 0, issued = 0;
@@ -1089,7 +1108,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                     const int i = i0 + lane;
                     const int phys = __shfl_sync(kFull, blk, i & 31);
                     int ok = 1;
-                    if (lane < NL && i < m) {
+                    if (lane < NL && i < m && u + bi + i >= pre) {  // units below `pre` went out before the wait
                         const int uu = u + bi + i;
                         const int s = uu % S;
                         ok = mbar_wait_bounded(&empty[s], ((uu / S) & 1) ^ 1, abort_flag);
@@ -1419,6 +1438,7 @@ std::atomic<int> g_opt_drop_load{0};
 std::atomic<int> g_opt_slow_softmax{0};
 std::atomic<int> g_opt_out_f32{0};
 std::atomic<int> g_opt_l2_policy{0};
+std::atomic<int> g_opt_early_loads{0};
 constexpr int kDefaultMinChunk = 4;
 
 // Work positions charged per work item (its fixed cost, in units of one work
@@ -1674,6 +1694,7 @@ kv_status plan_decode(DecodePlan *p, void *out, const void *q, const void *k_new
     // multi-layer launch has every layer in flight at once, and blocks shared by several sequences (a common
     // prefix) are re-read far enough apart that evict-first loses them: evict-normal keeps them.
     a.l2_policy = g_opt_l2_policy.load() != 0 ? g_opt_l2_policy.load() : (layers > 1 ? 2 : 1);
+    a.early_loads = g_opt_early_loads.load();
     a.fused = g_opt_combine.load() == 0 ? 1 : 0;
     a.scale_log2 = scale * 1.4426950408889634f;
     a.append = k_new != nullptr ? 1 : 0;
@@ -1976,6 +1997,11 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
             return KV_ERR_ARG;
         g_opt_l2_policy.store(value);
         return KV_OK;
+    case KV_OPT_EARLY_LOADS:
+        if (value < 0 || value > 1)
+            return KV_ERR_ARG;
+        g_opt_early_loads.store(value);
+        return KV_OK;
     default:
         return KV_ERR_ARG;
     }
@@ -2008,6 +2034,8 @@ extern "C" int kv_decode_get_option(int key)
         return g_opt_out_f32.load();
     case KV_OPT_L2_POLICY:
         return g_opt_l2_policy.load();
+    case KV_OPT_EARLY_LOADS:
+        return g_opt_early_loads.load();
     default:
         return -1;
     }

@@ -67,7 +67,8 @@ def test_option_ranges_need_no_gpu(pkv):
              pkv.KV_OPT_TEST_DROP_LOAD: ([0, 5], [-1]),
              pkv.KV_OPT_ITEM_COST: ([-1, 0, 64], [-2, 65]),
              pkv.KV_OPT_OUT_F32: ([0, 1], [-1, 2]),
-             pkv.KV_OPT_L2_POLICY: ([0, 1, 2, 3], [-1, 4])}
+             pkv.KV_OPT_L2_POLICY: ([0, 1, 2, 3], [-1, 4]),
+             pkv.KV_OPT_EARLY_LOADS: ([0, 1], [-1, 2])}
     for key, (good, bad) in cases.items():
         before = lib.kv_decode_get_option(key)
         for v in good:

@@ -20,7 +20,7 @@ PATHS = {"tensor_cores": 1, "cuda_cores": 2}
 def _default_options(pkv):
     yield
     for key in (pkv.KV_OPT_COMPUTE, pkv.KV_OPT_COMBINE, pkv.KV_OPT_GRID, pkv.KV_OPT_MIN_CHUNK,
-                pkv.KV_OPT_PRODUCER_LANES, pkv.KV_OPT_HEAD_GROUP, pkv.KV_OPT_ITEM_COST):
+                pkv.KV_OPT_PRODUCER_LANES, pkv.KV_OPT_HEAD_GROUP, pkv.KV_OPT_ITEM_COST, pkv.KV_OPT_EARLY_LOADS):
         pkv.set_option(key, 0)
 
 
@@ -88,12 +88,16 @@ def test_item_cost_changes_only_the_split(pkv, oracle_mod, cuda_device, cid, cos
     run_and_check(pkv, oracle_mod, case, what=f"config {cid} shape, item cost {cost}")
 
 
+@pytest.mark.parametrize("early", [0, 1])
 @pytest.mark.parametrize("grid", [0, 5])
 @pytest.mark.parametrize("cid", [2, 3])
-def test_back_to_back_layers(pkv, oracle_mod, cuda_device, cid, grid):
+def test_back_to_back_layers(pkv, oracle_mod, cuda_device, cid, grid, early):
     """Fused launches of several layers back to back on one stream and one workspace, no
-    synchronisation between them: each launch's prologue overlaps the previous launch."""
+    synchronisation between them: each launch's prologue overlaps the previous launch. With early loads,
+    each launch's first tiles are read while the previous layer's launch still runs (it writes only its own
+    layer's cache, so the promise holds)."""
     pkv.set_option(pkv.KV_OPT_GRID, grid)
+    pkv.set_option(pkv.KV_OPT_EARLY_LOADS, early)
     cfg = workloads.small_config(cid, batch=7, ctx_lo=1, ctx_hi=1300, W=96, n_layers=4)
     case = Case(cfg, cuda_device, n_layers=4)
     hosts = [case.host_inputs(layer) for layer in range(4)]
