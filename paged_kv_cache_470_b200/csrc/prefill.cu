@@ -387,8 +387,9 @@ __global__ void __launch_bounds__(kThreads, 2) prefill_kernel(const __grid_const
 // tcgen05 path. The same computation on the 5th-generation tensor cores: a CTA
 // takes 128 query rows; S = Q K^T (M=128, N=64 tokens) and O += P V
 // (M=128, N=D) are each a few tcgen05.mma issued by one thread, accumulating in
-// tensor memory. S is double-buffered (columns 0-63 and 64-127): the MMAs of
-// the next tile's S run while warps 0-3 turn this tile's S into P. Those warps
+// tensor memory. S is double-buffered (columns 0-63 and 64-127; at D = 64 a
+// third buffer sits after O): the MMAs of the next tile's S run while warps
+// 0-3 turn this tile's S into P. Those warps
 // own one row per thread: they read the row of S from tensor memory, run the
 // online softmax (all in the thread: no shuffles) and write the row of P, as
 // 16-bit pairs, over the first half of the same S buffer, where the P V MMA
@@ -420,16 +421,54 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// Two fp32 lanes in one 64-bit register, for the paired arithmetic of sm_100 (fma / add .f32x2:
+// one instruction for two elements), and a three-input maximum: the softmax warps are bound by
+// their own instruction stream, so fewer instructions per score is what shortens a tile.
+__device__ __forceinline__ unsigned long long f2pack(float lo, float hi)
+{
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2unpack(unsigned long long v, float &lo, float &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ unsigned long long fma_f2(unsigned long long a, unsigned long long b, unsigned long long c)
+{
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long add_f2(unsigned long long a, unsigned long long b)
+{
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 template <int D>
 struct TGeo {
     static constexpr int kTiles = D / 64;
     static constexpr int kQBytes = kTiles * kRows * 128;
     static constexpr int kKVTileBytes = kTok * 128;              // one 64-column tile of 64 tokens
     static constexpr int kStageBytes = kTiles * kKVTileBytes;     // K (or V) of one tile
-    // tiles of K and of V in flight (two each measured faster than three or four of K, and than
-    // four of each at D = 64)
-    static constexpr int kStagesK = 2;
-    static constexpr int kStagesV = 2;
+    // S buffers in tensor memory: two at D = 128 (with O they fill the CTA's 256 columns), three at
+    // D = 64, where O leaves 64 columns free. S of tile j + kSBufs - 1 needs the P V of tile j - 1
+    // (its buffer holds that tile's P), so a third buffer takes that P V off the path from one
+    // tile's softmax to the next but one's.
+    static constexpr int kSBufs = D == 64 ? 3 : 2;
+    // tiles of K and of V in flight: two each at D = 128 (measured faster than three or four of K);
+    // as many as S buffers at D = 64, so that the softmax of a tile (which follows S of that tile,
+    // hence the P V kSBufs tiles back) never waits on a V stage two loads behind
+    static constexpr int kStagesK = D == 64 ? 3 : 2;
+    static constexpr int kStagesV = D == 64 ? 3 : 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStagesK * kStageBytes;
@@ -441,10 +480,13 @@ struct TGeo {
     // mbarriers (full and empty per K and V stage, two S buffers, two P, P V, all MMAs, Q), the TMEM
     // address and two flags
     static constexpr int kBarBytes = 256;
-    static_assert((2 * kStagesK + 2 * kStagesV + 7) * 8 + 12 <= kBarBytes, "barrier area");
+    static_assert((2 * kStagesK + 2 * kStagesV + 3 * kSBufs + 2) * 8 + 12 <= kBarBytes, "barrier area");
     static constexpr int kSmemBytes = kOffBar + kBarBytes < 80 * 1024 ? 80 * 1024 : kOffBar + kBarBytes;
     static constexpr int kTmemCols = 256;                       // S/P buffers at 0 and 64, O at kOCol
     static constexpr int kOCol = 128;
+    // tensor-memory column of S buffer b: 0 and 64, and the third (D = 64) after O
+    static __device__ __forceinline__ uint32_t scol(int b) { return b < 2 ? b * kTok : kOCol + D; }
+    static_assert(kSBufs < 3 || kOCol + D + kTok <= kTmemCols, "third S buffer");
 };
 
 template <class E, int D>
@@ -453,7 +495,7 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                                                               const PrefillArgs a)
 {
     using G = TGeo<D>;
-    constexpr int kStagesK = G::kStagesK, kStagesV = G::kStagesV;
+    constexpr int kStagesK = G::kStagesK, kStagesV = G::kStagesV, kSB = G::kSBufs;
     extern __shared__ __align__(1024) unsigned char smem_tc[];
     const uint32_t base_s = smem_addr(smem_tc);
     unsigned char *base = smem_tc;
@@ -469,17 +511,19 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
     uint64_t *emptyK = fullK + kStagesK;
     uint64_t *fullV = emptyK + kStagesK;
     uint64_t *emptyV = fullV + kStagesV;
-    uint64_t *s_full = emptyV + kStagesV;  // [2]: one per S buffer
-    // P of tile j is ready: one barrier per tile parity. With one, a warp that finished tile j + 1
-    // could arrive again before a slower warp had arrived for tile j, completing that phase early;
-    // with two, arriving twice on one would take a warp two tiles ahead, and S of tile j + 2 waits
-    // for the P V of tile j
-    uint64_t *p_full = s_full + 2;
-    uint64_t *pv_done = p_full + 2;
+    uint64_t *s_full = emptyV + kStagesV;  // [kSB]: one per S buffer
+    // P of tile j is ready: one barrier per S buffer (tile j uses buffer j % kSB). With fewer, a warp
+    // that finished a later tile could arrive again before a slower warp had arrived for tile j,
+    // completing that phase early; with one per buffer, a warp's next arrival on it is for tile
+    // j + kSB, which needs S of that tile, which waits for the P V of tile j
+    uint64_t *p_full = s_full + kSB;
+    // the P V of tile j is done: one barrier per S buffer, so that each wait (the MMA thread's before
+    // it refills a buffer, a softmax warp's before it rescales O) is at most one phase behind
+    uint64_t *pv_done = p_full + kSB;
     // every MMA of the CTA is done: one phase, committed once after the last P V. The epilogue cannot
     // use pv_done: while another warp is a tile behind, pv_done can be two phases short of the last,
     // and a parity wait cannot tell two phases apart
-    uint64_t *o_done = pv_done + 1;
+    uint64_t *o_done = pv_done + kSB;
     uint64_t *q_ready = o_done + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_ready + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
@@ -521,11 +565,11 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             mbar_init(&fullV[s], 1);
             mbar_init(&emptyV[s], 1);
         }
-        mbar_init(&s_full[0], 1);
-        mbar_init(&s_full[1], 1);
-        mbar_init(&p_full[0], kRows);
-        mbar_init(&p_full[1], kRows);
-        mbar_init(pv_done, 1);
+        for (int b2 = 0; b2 < kSB; ++b2) {
+            mbar_init(&s_full[b2], 1);
+            mbar_init(&p_full[b2], kRows);
+            mbar_init(&pv_done[b2], 1);
+        }
         mbar_init(o_done, 1);
         mbar_init(q_ready, kRows);
         mbar_fence_init();
@@ -617,7 +661,7 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
             const uint32_t idesc_o = umma_idesc_f16(kRows, D, fmt, 0, 1);
             bool ok = mbar_wait_bounded(q_ready, 0, abort_flag);
             tcgen05_after_sync();
-            // S = Q K^T for tile jt into S buffer jt & 1
+            // S = Q K^T for tile jt into S buffer jt % kSB
             auto issue_s = [&](int jt) -> bool {
                 const int s = jt % kStagesK;
                 if (!mbar_wait_bounded(&fullK[s], (jt / kStagesK) & 1, abort_flag))
@@ -629,45 +673,47 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                     const uint32_t koff = (kk & 3) * 32;  // 16 elements along the 128-byte row
                     const uint64_t ad = umma_desc_sw128(sQ + (kk >> 2) * (kRows * 128) + koff, 16, 1024);
                     const uint64_t bd = umma_desc_sw128(kst + (kk >> 2) * G::kKVTileBytes + koff, 16, 1024);
-                    umma_f16(tmem + (jt & 1) * kTok, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                    umma_f16(tmem + G::scol(jt % kSB), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[jt & 1]);
+                umma_commit(&s_full[jt % kSB]);
                 // S read this K stage: it may be refilled (only a refill waits for this arrival, and
                 // no arrival may still be on its way when the CTA exits)
                 if (jt + kStagesK < ntiles)
                     umma_commit(&emptyK[s]);
                 return true;
             };
-            if (ok && ntiles > 0)
-                ok = issue_s(0);
+            // S of the first kSB - 1 tiles
+            for (int t = 0; t < kSB - 1 && t < ntiles && ok; ++t)
+                ok = issue_s(t);
             for (int jt = 0; jt < ntiles && ok; ++jt) {
                 const int s = jt % kStagesV;
                 const uint32_t vst = sV + s * G::kStageBytes;
-                if (jt + 1 < ntiles) {
-                    // the next S goes into the buffer that P of tile jt-1 used: wait for that PV
-                    if (jt >= 1 && !mbar_wait_bounded(pv_done, (jt - 1) & 1, abort_flag)) {
+                const int t = jt + kSB - 1;
+                if (t < ntiles) {
+                    // S of tile t goes into the buffer that P of tile t - kSB used: wait for that PV
+                    if (t >= kSB && !mbar_wait_bounded(&pv_done[t % kSB], ((t - kSB) / kSB) & 1, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    if (!issue_s(jt + 1)) {
+                    if (!issue_s(t)) {
                         ok = false;
                         break;
                     }
                 }
-                if (!mbar_wait_bounded(&p_full[jt & 1], (jt >> 1) & 1, abort_flag) ||
+                if (!mbar_wait_bounded(&p_full[jt % kSB], (jt / kSB) & 1, abort_flag) ||
                     !mbar_wait_bounded(&fullV[s], (jt / kStagesV) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tcgen05_after_sync();
-                // O += P V, P (16-bit pairs) in the first 32 columns of S buffer jt & 1
+                // O += P V, P (16-bit pairs) in the first 32 columns of S buffer jt % kSB
 #pragma unroll
                 for (int kk = 0; kk < kTok / 16; ++kk) {
                     const uint64_t bd = umma_desc_sw128(vst + kk * 2048, G::kKVTileBytes, 1024);
-                    umma_f16_tmem_a(tmem + G::kOCol, tmem + (jt & 1) * kTok + kk * 8, bd, idesc_o,
+                    umma_f16_tmem_a(tmem + G::kOCol, tmem + G::scol(jt % kSB) + kk * 8, bd, idesc_o,
                                     (jt > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(pv_done);
+                umma_commit(&pv_done[jt % kSB]);
                 if (jt + kStagesV < ntiles)
                     umma_commit(&emptyV[s]);
             }
@@ -710,23 +756,25 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
         bool good = true;
         for (int jt = 0; jt < ntiles; ++jt) {
             // tcgen05.ld/st are warp-wide: a warp takes every branch below as one
-            if (!__all_sync(kFullMask, mbar_wait_bounded(&s_full[jt & 1], (jt >> 1) & 1, abort_flag))) {
+            if (!__all_sync(kFullMask, mbar_wait_bounded(&s_full[jt % kSB], (jt / kSB) & 1, abort_flag))) {
                 good = false;
                 break;
             }
             tcgen05_after_sync();
-            const uint32_t sbuf = lane_base + (jt & 1) * kTok;
+            const uint32_t sbuf = lane_base + G::scol(jt % kSB);
             float x[kTok];
             {
-                uint32_t v[16];
+                // the row's four loads in flight together, one wait
+                uint32_t v[kTok / 16][16];
 #pragma unroll
-                for (int q4 = 0; q4 < kTok / 16; ++q4) {
-                    tmem_ld16(sbuf + q4 * 16, v);
-                    tmem_wait_ld();
+                for (int q4 = 0; q4 < kTok / 16; ++q4)
+                    tmem_ld16(sbuf + q4 * 16, v[q4]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q4 = 0; q4 < kTok / 16; ++q4)
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
-                        x[q4 * 16 + i] = __uint_as_float(v[i]);
-                }
+                        x[q4 * 16 + i] = __uint_as_float(v[q4][i]);
             }
             const int tok0 = jt * kTok;
             // raw scores: tokens after this row's position are -inf (scale > 0, so the maximum of
@@ -736,10 +784,12 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 for (int i = 0; i < kTok; ++i)
                     x[i] = (tok0 + i <= pos) ? x[i] : -INFINITY;
             }
-            float rmax = -INFINITY;
+            // the maximum in four independent chains of three-input maxima
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int i = 0; i < kTok; ++i)
-                rmax = fmaxf(rmax, x[i]);
+            for (int i = 0; i < kTok; i += 2)
+                mx[(i >> 1) & 3] = max3(mx[(i >> 1) & 3], x[i], x[i + 1]);
+            const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
             const float xmax = rmax * sl2;
             bool rescale = false;
             float alpha = 1.f;
@@ -753,7 +803,8 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 alpha = 1.f;  // lanes that keep their scale rewrite their row unchanged
             if (__any_sync(kFullMask, rescale)) {
                 // O is rescaled once the previous tile's PV has finished with it
-                if (!__all_sync(kFullMask, mbar_wait_bounded(pv_done, (jt - 1) & 1, abort_flag))) {
+                if (!__all_sync(kFullMask,
+                                mbar_wait_bounded(&pv_done[(jt - 1) % kSB], ((jt - 1) / kSB) & 1, abort_flag))) {
                     good = false;
                     break;
                 }
@@ -770,21 +821,29 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 }
                 tmem_wait_st();
             }
-            float psum = 0.f;
+            // scores two at a time: y = x * scale log2(e) - m (one paired FMA), P = 2^y, the row sum in
+            // two paired chains
+            const unsigned long long sc2 = f2pack(sl2, sl2), mm2 = f2pack(-m_used, -m_used);
+            unsigned long long ps2[2] = {f2pack(0.f, 0.f), f2pack(0.f, 0.f)};
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float pa = ex2_approx(fmaf(x[half * 32 + 2 * e], sl2, -m_used));
-                    const float pb = ex2_approx(fmaf(x[half * 32 + 2 * e + 1], sl2, -m_used));
-                    psum += pa + pb;
+                    const int i0 = half * 32 + 2 * e;
+                    float ya, yb;
+                    f2unpack(fma_f2(f2pack(x[i0], x[i0 + 1]), sc2, mm2), ya, yb);
+                    const float pa = ex2_approx(ya), pb = ex2_approx(yb);
+                    ps2[e & 1] = add_f2(ps2[e & 1], f2pack(pa, pb));
                     w[e] = E::pack(pa, pb);
                 }
                 tmem_st16(sbuf + half * 16, w);
             }
             tmem_wait_st();
-            l += psum;
+            float s0, s1, s2, s3;
+            f2unpack(ps2[0], s0, s1);
+            f2unpack(ps2[1], s2, s3);
+            l += (s0 + s1) + (s2 + s3);
             // rows of the CTA's last tile from its last visible token on hold whatever the pool holds
             // (past the context) or whatever the stage held before (blocks not loaded): zero those V
             // rows, whose P is 0, so that 0 * V stays 0 -- once V's loads have landed (S only says
@@ -815,7 +874,7 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
                 while (global_timer_ns() - t0 < 30000u)
                     __nanosleep(1000);
             }
-            mbar_arrive(&p_full[jt & 1]);
+            mbar_arrive(&p_full[jt % kSB]);
         }
         // epilogue: O / l
         if (__all_sync(kFullMask, good && mbar_wait_bounded(o_done, 0, abort_flag))) {

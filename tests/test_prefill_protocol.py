@@ -2,24 +2,27 @@
 paged_kv_cache_470_b200/csrc/prefill.cu), on the CPU.
 
 The model follows the kernel's actors and barriers: the producer warp (TMA loads of K and V into
-two-stage rings, K two tiles ahead), the MMA thread (S = Q K^T into one of two S buffers, P V into
+their own rings, K issued ahead of V), the MMA thread (S = Q K^T into one of SB S buffers, P V into
 O, tcgen05.commit arrivals), four softmax warps (32 rows each: read S, maybe rescale O, write P
-over S, zero the V rows of the last tile, hand P over) and the epilogue. Barriers behave like
-mbarriers: an arrival count per phase, and a wait by parity that succeeds while the current phase
-differs in parity from the one asked for (so it cannot tell phases two apart). Loads land and MMAs
-complete late, MMAs and their commits in issue order. A random scheduler runs many interleavings
-and checks that every read sees the data of its own tile (K, V, S, every warp's P, O after all
-P V) and that no run deadlocks. The two hand-off mistakes the kernel once had (one P-ready barrier
-for both tile parities; the epilogue waiting for the last P V by the parity of the P-V barrier)
-are planted in the model and must be caught, as must a producer that refills a stage without
-waiting for it to come free (which shows that the stage checks have teeth).
+over S, zero the V rows of the last tile, hand P over) and the epilogue. The kernel has SB = 2 S
+buffers at D = 128 and SB = 3 (with three K and three V stages) at D = 64, where tensor memory has room: S of
+tile j + SB - 1 is issued once the P V of tile j - 1 is done, and the S-full, P-ready and P-V-done
+barriers are one per S buffer. Barriers behave like mbarriers: an arrival count per phase, and a wait
+by parity that succeeds while the current phase differs in parity from the one asked for (so it
+cannot tell phases two apart). Loads land and MMAs complete late, MMAs and their commits in issue
+order. A random scheduler runs many interleavings and checks that every read sees the data of its
+own tile (K, V, S, every warp's P, O after all P V) and that no run deadlocks. Mistakes are planted
+in the model and must be caught: the two the kernel once had (one P-ready barrier for both tile
+parities; the epilogue waiting for the last P V by the parity of one P-V barrier), the two a third
+buffer invites (P-ready barriers by tile parity; one P-V barrier waited by parity), and a producer
+that refills a stage without waiting for it to come free (which shows that the stage checks have
+teeth).
 """
 import random
 
 import pytest
 
 WARPS = 4
-STAGES = 2
 
 
 class Violation(AssertionError):
@@ -43,36 +46,55 @@ class MBar:
 
 
 class Model:
-    def __init__(self, ntiles, one_p_barrier=False, epilogue_by_pv_parity=False, loads_ignore_empty=False,
-                 seed=0):
+    def __init__(self, ntiles, sbufs=2, kstages=2, vstages=2, one_p_barrier=False, epilogue_by_pv_parity=False,
+                 loads_ignore_empty=False, p_by_parity=False, one_pv_barrier=False, seed=0):
         self.n = ntiles
+        self.sb, self.ks, self.vs = sbufs, kstages, vstages
         self.rng = random.Random(seed)
         self.one_p = one_p_barrier
+        self.p_parity = p_by_parity
+        self.one_pv = one_pv_barrier
         self.epi_parity = epilogue_by_pv_parity
         self.no_empty = loads_ignore_empty
-        self.fullK = [MBar(1) for _ in range(STAGES)]
-        self.emptyK = [MBar(1) for _ in range(STAGES)]
-        self.fullV = [MBar(1) for _ in range(STAGES)]
-        self.emptyV = [MBar(1) for _ in range(STAGES)]
-        self.s_full = [MBar(1), MBar(1)]
-        self.p_full = [MBar(WARPS * 32), MBar(WARPS * 32)]
-        self.pv_done = MBar(1)
+        self.fullK = [MBar(1) for _ in range(kstages)]
+        self.emptyK = [MBar(1) for _ in range(kstages)]
+        self.fullV = [MBar(1) for _ in range(vstages)]
+        self.emptyV = [MBar(1) for _ in range(vstages)]
+        self.s_full = [MBar(1) for _ in range(sbufs)]
+        self.p_full = [MBar(WARPS * 32) for _ in range(sbufs)]
+        self.pv_done = [MBar(1) for _ in range(sbufs)]
+        self.pv_all = MBar(1)        # one barrier committed after every P V: only the planted mistakes use it
         self.o_done = MBar(1)
         # contents: which tile each stage / buffer holds (None: nothing yet)
-        self.k_stage = [None] * STAGES
-        self.v_stage = [None] * STAGES
-        self.s_buf = [None, None]                       # the tile whose S each buffer holds
-        self.p_rows = [[None] * WARPS for _ in range(2)]  # tile whose P each warp wrote in a buffer
-        self.o_tiles = 0                                # P V done
+        self.k_stage = [None] * kstages
+        self.v_stage = [None] * vstages
+        self.s_buf = [None] * sbufs                            # the tile whose S each buffer holds
+        self.p_rows = [[None] * WARPS for _ in range(sbufs)]   # tile whose P each warp wrote in a buffer
+        self.o_tiles = 0                                       # P V done
         self.v_zeroed = set()
-        self.inflight = []                              # (landing step, action)
-        self.tc_queue = []                              # tensor-core ops in issue order
-        self.reads = {}                                 # stage readers still in flight
+        self.inflight = []                                     # (landing step, action)
+        self.tc_queue = []                                     # tensor-core ops in issue order
+        self.reads = {}                                        # stage readers still in flight
         self.step = 0
+
+    # barrier and parity of P-ready (and of the P-V-done wait) for tile j, as the kernel (or a mistake) picks
+    def p_bar(self, j):
+        if self.one_p:
+            return self.p_full[0], j & 1
+        if self.p_parity:
+            return self.p_full[j & 1], (j >> 1) & 1
+        return self.p_full[j % self.sb], (j // self.sb) & 1
+
+    def pv_wait(self, j):
+        """(barrier, parity) of a wait for P V(j) to be done."""
+        if self.one_pv:
+            return self.pv_all, j & 1
+        return self.pv_done[j % self.sb], (j // self.sb) & 1
 
     # ---- asynchronous units ----
     def land(self, kind, t):
-        s = t % STAGES
+        ns = self.ks if kind == "K" else self.vs
+        s = t % ns
         stage = self.k_stage if kind == "K" else self.v_stage
         # the load overwrites the stage: its previous tile's MMA must be done
         if self.reads.get((kind, s)):
@@ -84,91 +106,100 @@ class Model:
         kind = op[0]
         if kind == "S":
             t = op[1]
-            if self.k_stage[t % STAGES] != t:
-                raise Violation(f"S({t}) reads K stage holding tile {self.k_stage[t % STAGES]}")
-            self.s_buf[t & 1] = t
-            self.p_rows[t & 1] = [None] * WARPS
-            self.reads[("K", t % STAGES)] = False
+            if self.k_stage[t % self.ks] != t:
+                raise Violation(f"S({t}) reads K stage holding tile {self.k_stage[t % self.ks]}")
+            b = t % self.sb
+            if self.s_buf[b] is not None and self.o_tiles <= self.s_buf[b]:
+                raise Violation(f"S({t}) overwrites the P of tile {self.s_buf[b]} before its P V")
+            self.s_buf[b] = t
+            self.p_rows[b] = [None] * WARPS
+            self.reads[("K", t % self.ks)] = False
         elif kind == "PV":
             t = op[1]
-            if self.v_stage[t % STAGES] != t:
-                raise Violation(f"PV({t}) reads V stage holding tile {self.v_stage[t % STAGES]}")
-            if any(w != t for w in self.p_rows[t & 1]):
-                raise Violation(f"PV({t}) reads P rows {self.p_rows[t & 1]} (not all of tile {t})")
+            b = t % self.sb
+            if self.v_stage[t % self.vs] != t:
+                raise Violation(f"PV({t}) reads V stage holding tile {self.v_stage[t % self.vs]}")
+            if self.s_buf[b] != t or any(w != t for w in self.p_rows[b]):
+                raise Violation(f"PV({t}) reads P rows {self.p_rows[b]} (not all of tile {t})")
             if t == self.n - 1 and t not in self.v_zeroed:
                 raise Violation(f"PV({t}) reads the last tile's V before its tail rows are zeroed")
             if self.o_tiles != t:
                 raise Violation("P V out of order")
             self.o_tiles = t + 1
-            self.reads[("V", t % STAGES)] = False
+            self.reads[("V", t % self.vs)] = False
         elif kind == "commit":
-            op[1].arrive()
+            for bar in op[1:]:
+                bar.arrive()
 
     # ---- actors (generators yielding wait conditions) ----
     def producer(self):
-        order = [("K", t) for t in range(min(STAGES, self.n))]
+        order = [("K", t) for t in range(min(self.ks, self.n))]
         for t in range(self.n):
             order.append(("V", t))
-            if t + STAGES < self.n:
-                order.append(("K", t + STAGES))
+            if t + self.ks < self.n:
+                order.append(("K", t + self.ks))
         for kind, t in order:
-            s = t % STAGES
+            ns = self.ks if kind == "K" else self.vs
+            s = t % ns
             empty = (self.emptyK if kind == "K" else self.emptyV)[s]
             if self.no_empty:
                 yield lambda: True
             else:
-                yield lambda e=empty, p=((t // STAGES) & 1) ^ 1: e.done(p)
+                yield lambda e=empty, p=((t // ns) & 1) ^ 1: e.done(p)
             self.inflight.append((self.step + self.rng.randint(1, 40), ("land", kind, t)))
 
     def mma(self):
         def issue_s(j):
-            self.reads[("K", j % STAGES)] = True
+            self.reads[("K", j % self.ks)] = True
             self.tc_queue.append(("S", j))
-            self.tc_queue.append(("commit", self.s_full[j & 1]))
-            if j + STAGES < self.n:
-                self.tc_queue.append(("commit", self.emptyK[j % STAGES]))
-        yield lambda: self.fullK[0].done(0)
-        issue_s(0)
+            self.tc_queue.append(("commit", self.s_full[j % self.sb]))
+            if j + self.ks < self.n:
+                self.tc_queue.append(("commit", self.emptyK[j % self.ks]))
+        for j in range(min(self.sb - 1, self.n)):                 # S of the first SB - 1 tiles
+            yield lambda s=j % self.ks, p=(j // self.ks) & 1: self.fullK[s].done(p)
+            issue_s(j)
         for j in range(self.n):
-            if j + 1 < self.n:
-                if j >= 1:
-                    yield lambda p=(j - 1) & 1: self.pv_done.done(p)
-                yield lambda s=(j + 1) % STAGES, p=((j + 1) // STAGES) & 1: self.fullK[s].done(p)
-                issue_s(j + 1)
-            pf = self.p_full[0] if self.one_p else self.p_full[j & 1]
-            pp = (j & 1) if self.one_p else ((j >> 1) & 1)
-            yield lambda b=pf, p=pp: b.done(p)
-            yield lambda s=j % STAGES, p=(j // STAGES) & 1: self.fullV[s].done(p)
-            self.reads[("V", j % STAGES)] = True
+            t = j + self.sb - 1
+            if t < self.n:
+                if t >= self.sb:                                  # its S buffer's previous P V
+                    yield lambda bp=self.pv_wait(t - self.sb): bp[0].done(bp[1])
+                yield lambda s=t % self.ks, p=(t // self.ks) & 1: self.fullK[s].done(p)
+                issue_s(t)
+            yield lambda bp=self.p_bar(j): bp[0].done(bp[1])
+            yield lambda s=j % self.vs, p=(j // self.vs) & 1: self.fullV[s].done(p)
+            self.reads[("V", j % self.vs)] = True
             self.tc_queue.append(("PV", j))
-            self.tc_queue.append(("commit", self.pv_done))
-            if j + STAGES < self.n:
-                self.tc_queue.append(("commit", self.emptyV[j % STAGES]))
+            self.tc_queue.append(("commit", self.pv_done[j % self.sb], self.pv_all))
+            if j + self.vs < self.n:
+                self.tc_queue.append(("commit", self.emptyV[j % self.vs]))
         self.tc_queue.append(("commit", self.o_done))
         yield lambda: self.o_done.done(0)
 
     def softmax(self, w):
         for j in range(self.n):
-            yield lambda b=self.s_full[j & 1], p=(j >> 1) & 1: b.done(p)
-            if self.s_buf[j & 1] != j:
-                raise Violation(f"warp {w} reads S buffer holding {self.s_buf[j & 1]} at tile {j}")
+            b = j % self.sb
+            yield lambda bar=self.s_full[b], p=(j // self.sb) & 1: bar.done(p)
+            if self.s_buf[b] != j:
+                raise Violation(f"warp {w} reads S buffer holding {self.s_buf[b]} at tile {j}")
             if j > 0 and self.rng.random() < 0.3:          # the row maximum grew: rescale O
-                yield lambda p=(j - 1) & 1: self.pv_done.done(p)
+                yield lambda bp=self.pv_wait(j - 1): bp[0].done(bp[1])
                 if self.o_tiles != j:
                     raise Violation(f"warp {w} rescales O with {self.o_tiles} of {j} P V done")
             for _ in range(self.rng.randint(0, 3)):        # the softmax takes a while
                 yield lambda: True
-            self.p_rows[j & 1][w] = j
+            if self.s_buf[b] != j:
+                raise Violation(f"warp {w} writes P over S buffer holding {self.s_buf[b]} at tile {j}")
+            self.p_rows[b][w] = j
             if j == self.n - 1:                            # zero the last tile's tail V rows
-                yield lambda s=j % STAGES, p=(j // STAGES) & 1: self.fullV[s].done(p)
-                if self.v_stage[j % STAGES] != j:
-                    raise Violation(f"warp {w} zeroes rows of V stage holding {self.v_stage[j % STAGES]}")
+                yield lambda s=j % self.vs, p=(j // self.vs) & 1: self.fullV[s].done(p)
+                if self.v_stage[j % self.vs] != j:
+                    raise Violation(f"warp {w} zeroes rows of V stage holding {self.v_stage[j % self.vs]}")
                 self.v_zeroed.add(j)
-            bar = self.p_full[0] if self.one_p else self.p_full[j & 1]
+            bar = self.p_bar(j)[0]
             for _ in range(32):
                 bar.arrive()
         if self.epi_parity:
-            yield lambda p=(self.n - 1) & 1: self.pv_done.done(p)
+            yield lambda p=(self.n - 1) & 1: self.pv_all.done(p)
         else:
             yield lambda: self.o_done.done(0)
         if self.o_tiles != self.n:
@@ -209,18 +240,31 @@ class Model:
         return True
 
 
+GEOMETRIES = {"D128": dict(sbufs=2, kstages=2, vstages=2), "D64": dict(sbufs=3, kstages=3, vstages=3)}
+
+
+@pytest.mark.parametrize("geo", sorted(GEOMETRIES))
 @pytest.mark.parametrize("ntiles", [1, 2, 3, 4, 7])
-def test_kernel_hand_offs_hold_under_random_schedules(ntiles):
+def test_kernel_hand_offs_hold_under_random_schedules(ntiles, geo):
     for seed in range(150):
-        Model(ntiles, seed=seed).run()
+        Model(ntiles, seed=seed, **GEOMETRIES[geo]).run()
 
 
-@pytest.mark.parametrize("bug", ["one_p_barrier", "epilogue_by_pv_parity", "loads_ignore_empty"])
-def test_the_model_catches_the_hand_off_mistakes(bug):
+@pytest.mark.parametrize("geo,bug", [("D128", "one_p_barrier"), ("D128", "epilogue_by_pv_parity"),
+                                     ("D128", "loads_ignore_empty"), ("D64", "p_by_parity"),
+                                     ("D64", "one_pv_barrier"), ("D64", "loads_ignore_empty"),
+                                     ("D64", "epilogue_by_pv_parity"), ("D64", "two_v_stages")])
+def test_the_model_catches_the_hand_off_mistakes(geo, bug):
     caught = 0
+    geometry = dict(GEOMETRIES[geo])
+    if bug == "two_v_stages":       # three S buffers run far enough ahead to wrap a two-stage V ring
+        geometry["vstages"] = 2
+        planted = {}
+    else:
+        planted = {bug: True}
     for seed in range(300):
         try:
-            Model(5, seed=seed, **{bug: True}).run()
+            Model(7, seed=seed, **geometry, **planted).run()
         except Violation:
             caught += 1
     assert caught > 0, f"{bug} never showed up in 300 schedules"
