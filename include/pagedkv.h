@@ -330,8 +330,9 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *   KV_OPT_PREFILL_PATH: paged_attention_prefill on 0 auto (tcgen05), 1
  *                     tcgen05.mma with tensor-memory accumulators, 2 mma.sync.
  *   KV_OPT_TEST_DROP_LOAD: test hook for the timeout path, 0 (default) off;
- *                     n > 0: in the decode kernels' CTA 0 the tile load of
- *                     work unit n - 1 is never issued, so the wait for it runs
+ *                     n > 0: in the decode kernels' CTA that holds the
+ *                     launch's first work unit, the tile load of its work
+ *                     unit n - 1 is never issued, so the wait for it runs
  *                     out (after about a second): the call completes with
  *                     KV_STATUS_WAIT_TIMEOUT in the status word and its output
  *                     is not valid; the context stays usable (re-initialise

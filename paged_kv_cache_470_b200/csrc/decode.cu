@@ -126,7 +126,8 @@ struct DecodeArgs {
     int prod_lanes;      // producer lanes issuing TMA
     int min_chunk;
     int item_cost;       // work positions charged per work item on top of its units
-    int drop_unit;       // test hook: CTA 0 never loads its unit with this index (-1: none)
+    int drop_unit;       // test hook: the CTA holding the launch's first unit never loads its unit with
+                         // this index (-1: none)
     int l2_policy;       // L2 priority of the K/V tile loads: 1 evict first, 2 evict normal, 3 evict last
     int early_loads;     // issue the first ring of tile loads before the grid dependency wait (caller's promise)
     int fused;
@@ -1069,7 +1070,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         // ring of tile loads goes out before the wait (lane i: unit i into stage i, their first use), so the
         // CTA's first data arrives while the previous kernel finishes. q and the new rows still wait.
         const int pre = a.early_loads ? min(S, m_first) : 0;
-        if (lane < pre && !(lane == a.drop_unit && blockIdx.x == 0)) {
+        const bool drop_here = misc[kMiscStartU] == 0;  // the test hook's CTA: it holds the launch's first unit
+        if (lane < pre && !(lane == a.drop_unit && drop_here)) {
             const int head0 = (cur0.k / a.hchunks) * a.hg;
             mbar_arrive_expect_tx(&full[lane], a.stage_bytes);
             const uint32_t dst = ring + lane * a.stage_bytes;
@@ -1112,7 +1114,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         const int uu = u + bi + i;
                         const int s = uu % S;
                         ok = mbar_wait_bounded(&empty[s], ((uu / S) & 1) ^ 1, abort_flag);
-                        if (ok && uu == a.drop_unit && blockIdx.x == 0) {
+                        if (ok && uu == a.drop_unit && drop_here) {
                             // test hook: this stage is never filled, so its consumers' wait runs out
                         } else if (ok) {
                             mbar_arrive_expect_tx(&full[s], a.stage_bytes);

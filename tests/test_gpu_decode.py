@@ -378,3 +378,23 @@ def test_full_size_layers_in_one_launch(pkv, oracle_mod, cuda_device, cid):
     case = Case(cfg, cuda_device, n_layers=L)
     layers = sorted({0, L - 1, random.Random(cid).randrange(L)})
     run_layers_and_check(pkv, oracle_mod, case, layers=layers, what=f"config {cid}")
+
+
+@pytest.mark.parametrize("layers", [1, 3])
+@pytest.mark.parametrize("policy", [1, 2, 3])
+def test_l2_priorities_and_early_loads_keep_the_result(pkv, oracle_mod, cuda_device, policy, layers):
+    """Every L2 priority of the tile loads, with and without early loads (whose promise holds here: the
+    launch before each is the previous one over other layers' caches, or none), gives the oracle's result."""
+    pkv.set_option(pkv.KV_OPT_L2_POLICY, policy)
+    try:
+        for early in (0, 1):
+            pkv.set_option(pkv.KV_OPT_EARLY_LOADS, early)
+            cfg = workloads.small_config(2, batch=10, ctx_lo=1, ctx_hi=900, W=64)
+            case = Case(cfg, cuda_device, n_layers=layers, seed=policy * 10 + early)
+            if layers == 1:
+                run_and_check(pkv, oracle_mod, case, what=f"L2 policy {policy}, early {early}", fused=True)
+            else:
+                run_layers_and_check(pkv, oracle_mod, case, what=f"L2 policy {policy}, early {early}")
+    finally:
+        pkv.set_option(pkv.KV_OPT_L2_POLICY, 0)
+        pkv.set_option(pkv.KV_OPT_EARLY_LOADS, 0)

@@ -103,3 +103,14 @@ def test_dtype_mismatch_is_refused(pkv, cuda_device):
     with pytest.raises(ValueError):
         pkv.paged_attention_decode(torch.empty_like(case.q[0]), case.q[0].float(), case.k[0].float(),
                                    case.v[0].float(), case.tables, case.lens, cfg.scale, ws)
+
+
+@pytest.mark.parametrize("path", sorted(PATHS))
+def test_layers_in_one_launch_fp16(pkv, oracle_mod, cuda_device, path):
+    """The multi-layer launch on the fp16 LLaMA-2-7B shape (32 kv heads, D = 128): three full-size layers."""
+    from test_gpu_decode import run_layers_and_check
+    pkv.set_option(pkv.KV_OPT_COMPUTE, PATHS[path])
+    cfg = workloads.small_config(4, elem="fp16", batch=8, pool_blocks=2048)
+    case = Case(cfg, cuda_device, n_layers=3)
+    assert case.k_all.dtype == torch.float16
+    run_layers_and_check(pkv, oracle_mod, case, what=f"fp16 layers/{path}")

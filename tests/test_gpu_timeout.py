@@ -22,7 +22,7 @@ def test_wait_runs_out_and_the_context_survives(pkv, oracle_mod, cuda_device, fu
     ws = pkv.make_workspace(cfg.batch, cfg.Hq, cfg.Hkv, cfg.D)
     host = case.host_inputs(0)
     try:
-        pkv.set_option(pkv.KV_OPT_TEST_DROP_LOAD, 1)     # CTA 0 never loads its first unit
+        pkv.set_option(pkv.KV_OPT_TEST_DROP_LOAD, 1)     # the CTA with the first unit never loads it
         t0 = time.perf_counter()
         gpu_step(pkv, case, 0, ws, fused=fused)
         status = pkv.read_status(ws)                    # synchronises
