@@ -474,74 +474,23 @@ class BlockPool:
 
 
 # ---------------------------------------------------------------------------
-# the C ABI's names: each call of include/pagedkv.h under its own name (the same marshalling as above;
-# a pool is a BlockPool, whose handle the kv_pool_* calls take)
+# the C ABI's names: each call of include/pagedkv.h under its own name, bound to the marshalling above
+# (a pool is a BlockPool, whose handle the kv_pool_* calls take)
 # ---------------------------------------------------------------------------
-def paged_attention_workspace_size(B: int, Hq: int, Hkv: int, D: int) -> int:
-    return workspace_size(B, Hq, Hkv, D)
-
-
-def paged_attention_workspace_size_layers(B: int, Hq: int, Hkv: int, D: int, num_layers: int) -> int:
-    return workspace_size_layers(B, Hq, Hkv, D, num_layers)
-
-
-def paged_attention_workspace_init(workspace: torch.Tensor, stream=None) -> None:
-    workspace_init(workspace, stream)
-
-
-def paged_attention_read_status(workspace: torch.Tensor, clear: bool = True, stream=None) -> int:
-    return read_status(workspace, clear, stream)
-
-
-def kv_decode_set_option(key: int, value: int) -> None:
-    set_option(key, value)
-
-
-def kv_decode_get_option(key: int) -> int:
-    return get_option(key)
-
-
-def kv_pool_create(num_blocks: int) -> BlockPool:
-    return BlockPool(num_blocks)
-
-
-def kv_pool_destroy(pool: BlockPool) -> None:
-    pool.close()
-
-
-def kv_pool_alloc(pool: BlockPool, n: int) -> list[int]:
-    return pool.alloc(n)
-
-
-def kv_pool_incref(pool: BlockPool, ids) -> None:
-    pool.incref(ids)
-
-
-def kv_pool_free(pool: BlockPool, ids) -> None:
-    pool.free(ids)
-
-
-def kv_pool_num_free(pool: BlockPool) -> int:
-    return pool.num_free()
-
-
-def kv_pool_num_blocks(pool: BlockPool) -> int:
-    return pool.num_blocks()
-
-
-def kv_pool_refcount(pool: BlockPool, block_id: int) -> int:
-    return pool.refcount(block_id)
-
-
-def kv_pool_append_slots(pool: BlockPool, block_tables: torch.Tensor, context_lens: torch.Tensor,
-                         slot_mapping: torch.Tensor) -> None:
-    pool.append_slots(block_tables, context_lens, slot_mapping)
-
-
-def kv_pool_fork(pool: BlockPool, parent_ids) -> list[int]:
-    return pool.fork(parent_ids)
-
-
-def kv_pool_append_slots_cow(pool: BlockPool, block_tables: torch.Tensor, context_lens: torch.Tensor,
-                             slot_mapping: torch.Tensor) -> tuple[list[int], list[int]]:
-    return pool.append_slots_cow(block_tables, context_lens, slot_mapping)
+paged_attention_workspace_size = workspace_size
+paged_attention_workspace_size_layers = workspace_size_layers
+paged_attention_workspace_init = workspace_init
+paged_attention_read_status = read_status
+kv_decode_set_option = set_option
+kv_decode_get_option = get_option
+kv_pool_create = BlockPool
+kv_pool_destroy = BlockPool.close
+kv_pool_alloc = BlockPool.alloc
+kv_pool_incref = BlockPool.incref
+kv_pool_free = BlockPool.free
+kv_pool_num_free = BlockPool.num_free
+kv_pool_num_blocks = BlockPool.num_blocks
+kv_pool_refcount = BlockPool.refcount
+kv_pool_append_slots = BlockPool.append_slots
+kv_pool_fork = BlockPool.fork
+kv_pool_append_slots_cow = BlockPool.append_slots_cow
