@@ -349,10 +349,9 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     result before any rounding to the element type. The
  *                     other arguments keep their element type.
  *   KV_OPT_L2_POLICY: L2 priority of the decode kernels' K/V tile loads: 0
- *                     auto (evict first for one layer; evict normal for a
- *                     multi-layer launch, where blocks that several sequences
- *                     share are re-read far apart), 1 evict first, 2 evict
- *                     normal, 3 evict last.
+ *                     auto (evict normal for a multi-layer launch at D = 128,
+ *                     evict first otherwise: the faster on every workload
+ *                     measured), 1 evict first, 2 evict normal, 3 evict last.
  *   KV_OPT_EARLY_LOADS: 0 (default) off; 1: the caller promises that, for
  *                     every decode call in a stream, the kernel launched just
  *                     before it in that stream does not write the caches the
