@@ -411,6 +411,16 @@ def block_moves_measure(wl, peak, reps=10):
     return res
 
 
+def prefill_arithmetic(path: int, elem: str) -> str:
+    """What the chunked-prefill kernel of KV_OPT_PREFILL_PATH computes with (0 is the default kernel)."""
+    if path == 2:
+        return f"mma.sync m16n8k16 {elem} in, fp32 accumulate"
+    if path == 1:
+        return f"tcgen05.mma kind::f16 M=128 N=64 {elem} in, fp32 accumulate in tensor memory; one query tile per CTA"
+    return (f"tcgen05.mma kind::f16 M=128 N=128 {elem} in, fp32 accumulate in tensor memory; two query tiles per "
+            f"CTA sharing each 128-token K/V tile")
+
+
 def prefill_measure(pkv, device, elem, reps=20, keys=("llama3_8b", "0p5b")):
     """The chunked-prefill workloads: one layer's paged_attention_prefill each, timed with CUDA events.
     Algorithmic flops = 4 * Hq * D per (query, visible token) pair (Q K^T and P V, a multiply-add = 2)."""
@@ -447,9 +457,7 @@ def prefill_measure(pkv, device, elem, reps=20, keys=("llama3_8b", "0p5b")):
         res[key] = {"workload": cfg.name, "bound": "tensor", "achieved": round(tf, 1), "unit": "TFLOP/s",
                     "peak": peak, "peak_kind": kind, "frac": round(tf / peak, 4), "ms": round(ms, 4),
                     "flops_per_launch": flops, "status": int(flag.item()),
-                    "arithmetic": (f"mma.sync m16n8k16 {elem} in, fp32 accumulate"
-                                   if pkv.get_option(pkv.KV_OPT_PREFILL_PATH) == 2 else
-                                   f"tcgen05.mma kind::f16 M=128 {elem} in, fp32 accumulate in tensor memory"),
+                    "arithmetic": prefill_arithmetic(pkv.get_option(pkv.KV_OPT_PREFILL_PATH), elem),
                     "timing": f"CUDA events, mean of {reps} back-to-back launches after 3 warm-up launches; "
                               f"KV {2 * k.numel() * k.element_size() / 1e6:.0f} MB + q "
                               f"{q.numel() * q.element_size() / 1e6:.0f} MB per launch (L2 126 MB)"}
@@ -748,6 +756,8 @@ def run_ours(args, world, rank, local):
         pkv.set_option(pkv.KV_OPT_COMPUTE, {"tensor": 1, "cuda": 2}[args.compute])
     if args.grid:
         pkv.set_option(pkv.KV_OPT_GRID, args.grid)
+    if args.prefill_path:
+        pkv.set_option(pkv.KV_OPT_PREFILL_PATH, args.prefill_path)
     if args.combine_kernel:
         pkv.set_option(pkv.KV_OPT_COMBINE, 1)
     if args.head_group:
@@ -879,6 +889,9 @@ def main(argv=None):
     ap.add_argument("--profile-prefill", choices=sorted(workloads.PREFILL_CONFIGS), default=None,
                     help="only run the chunked-prefill workload: 3 warm-up and --steps timed launches (for ncu)")
     ap.add_argument("--grid", type=int, default=0, help="decode CTAs per launch (0: one per SM)")
+    ap.add_argument("--prefill-path", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="chunked prefill kernel: 0 auto, 1 tcgen05 one query tile per CTA, 2 mma.sync, "
+                         "3 tcgen05 two query tiles per CTA")
     ap.add_argument("--combine-kernel", action="store_true", help="split-K merge in a separate kernel")
     ap.add_argument("--head-group", type=int, default=0, help="kv heads per work unit (0: auto)")
     ap.add_argument("--item-cost", type=int, default=0,

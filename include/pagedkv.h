@@ -287,7 +287,9 @@ KV_API kv_status paged_attention_decode_noalloc(void *out, const void *q,
  * int32, non-decreasing from 0; max_query_len >= every n_b (it sizes the
  * grid). Tensor cores (tcgen05.mma with tensor-memory accumulators; mma.sync
  * with KV_OPT_PREFILL_PATH = 2), fp32 accumulation, the probabilities rounded
- * to the element type before they multiply V. No workspace. Data errors are
+ * to the element type before they multiply V. No workspace. The default
+ * kernel takes 256 query rows of one (sequence, kv head) per CTA, so
+ * ceil(max_query_len * Hq / Hkv / 256) must be <= 65535. Data errors are
  * OR-ed into *error_flag (device int32, may be NULL): KV_STATUS_BAD_CONTEXT
  * when n_b > c_b, c_b > 16 * max_blocks_per_seq or n_b > max_query_len (that
  * sequence's rows are not written), KV_STATUS_BAD_BLOCK_ID for ids outside the
@@ -327,8 +329,11 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     group and query-head chunk) adds this many more for its
  *                     fixed cost; CTAs take equal ranges of positions.
  *                     0 auto, -1 none, 1..64 that many.
- *   KV_OPT_PREFILL_PATH: paged_attention_prefill on 0 auto (tcgen05), 1
- *                     tcgen05.mma with tensor-memory accumulators, 2 mma.sync.
+ *   KV_OPT_PREFILL_PATH: paged_attention_prefill on 0 auto (3), 1
+ *                     tcgen05.mma with tensor-memory accumulators, one tile of
+ *                     128 query rows per CTA (two CTAs per SM), 2 mma.sync,
+ *                     3 tcgen05.mma, two tiles of 128 query rows per CTA
+ *                     sharing each 128-token K/V tile (one CTA per SM).
  *   KV_OPT_TEST_DROP_LOAD: test hook for the timeout path, 0 (default) off;
  *                     n > 0: in the decode kernels' CTA that holds the
  *                     launch's first work unit, the tile load of its work
@@ -338,7 +343,7 @@ KV_API kv_status paged_attention_prefill(void *out, const void *q, const void *k
  *                     is not valid; the context stays usable (re-initialise
  *                     the workspace, as after any timed-out call).
  *   KV_OPT_TEST_SLOW_SOFTMAX: test hook for the hand-offs of the tcgen05
- *                     prefill, 0 (default) off; 1: in every CTA the first
+ *                     prefill kernels, 0 (default) off; 1: in every CTA the first
  *                     softmax warp waits about 30 microseconds before it hands
  *                     over P of the first tile, so the other warps run a tile
  *                     ahead of it. The output must not change.

@@ -1978,7 +1978,7 @@ extern "C" kv_status kv_decode_set_option(int key, int value)
         g_opt_item_cost.store(value);
         return KV_OK;
     case KV_OPT_PREFILL_PATH:
-        if (value < 0 || value > 2)
+        if (value < 0 || value > 3)
             return KV_ERR_ARG;
         g_opt_prefill_path.store(value);
         return KV_OK;

@@ -927,6 +927,563 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
 }
 
 }  // namespace tc
+
+// ===========================================================================
+// tcgen05 path, two query tiles per CTA. One CTA per SM takes 256 query rows
+// (two tiles of 128) and streams each 128-token K/V tile once for both. A
+// tcgen05.mma of M = 128 with N = 128 runs at the tensor pipe's full rate,
+// where N = 64 (the one-tile kernel's S) does not; a tile of 128 tokens also
+// halves the hand-offs per flop. Tensor memory (all 512 columns of the SM):
+// S of tile t at 128 t, O of tile t at 256 + D t; P of tile t is written over
+// the first half of its S at D = 128 and has columns of its own at D = 64
+// (384 + 64 t), where O leaves room. Warps 0-3 run the softmax of tile 0 and
+// warps 4-7 that of tile 1 (one row per thread, as in the one-tile kernel),
+// warp 8 issues the TMA loads, warp 9 the MMAs. The MMA thread alternates the
+// tiles: while one tile's softmax runs, the tensor pipe does the other tile's
+// P V and next S. At D = 128 the S of the next tile goes where P of this one
+// is, so it waits for that P V; at D = 64 it only waits until the softmax
+// has read S, and runs while the softmax computes. Every hand-off is an
+// mbarrier with a bounded wait, as in the one-tile kernel.
+// ===========================================================================
+namespace pair {
+
+constexpr int kRows = 128;     // query rows per tile; a CTA takes two
+constexpr int kTok = 128;      // KV tokens per tile (8 blocks)
+constexpr int kThreads = 320;  // 8 softmax warps, the producer warp, the MMA warp
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kRankMax = 256;  // batches up to this size are launched longest sequence first
+
+
+template <int D>
+struct Geo {
+    static constexpr int kChunks = D / 64;                 // 128-byte chunks of a row of D elements
+    static constexpr int kQBytes = kChunks * kRows * 128;  // one query tile
+    static constexpr int kChunkBytes = kTok * 128;         // one chunk of a K or V tile
+    static constexpr int kStageBytes = kChunks * kChunkBytes;
+    static constexpr int kStagesK = D == 64 ? 3 : 2;
+    static constexpr int kStagesV = D == 64 ? 3 : 2;
+    // P in columns of its own (D = 64) or over S (D = 128, where the two O take 256 columns)
+    static constexpr bool kSepP = D == 64;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = 2 * kQBytes;
+    static constexpr int kOffV = kOffK + kStagesK * kStageBytes;
+    static constexpr int kOffBar = kOffV + kStagesV * kStageBytes;
+    // full and empty per K and V stage; per query tile S full, S read, P full, P V done and Q
+    // ready; all MMAs done; the tensor-memory address and two flags
+    static constexpr int kBarBytes = 256;
+    static_assert((2 * kStagesK + 2 * kStagesV + 5 * 2 + 1) * 8 + 12 <= kBarBytes, "barrier area");
+    static constexpr int kSmemBytes = kOffBar + kBarBytes;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+    static constexpr int kTmemCols = 512;
+    static __device__ __forceinline__ uint32_t scol(int t) { return t * kTok; }
+    static __device__ __forceinline__ uint32_t ocol(int t) { return 2 * kTok + t * D; }
+    static __device__ __forceinline__ uint32_t pcol(int t)
+    {
+        return kSepP ? 2 * kTok + 2 * D + t * (kTok / 2) : t * kTok;
+    }
+    static_assert(!kSepP || 2 * kTok + 2 * D + kTok <= kTmemCols, "P columns");
+    static_assert(2 * kTok + 2 * D <= kTmemCols, "O columns");
+};
+
+template <class E, int D>
+__global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                   const __grid_constant__ CUtensorMap tmV,
+                                                                   const PrefillArgs a)
+{
+    using G = Geo<D>;
+    constexpr int SK = G::kStagesK, SV = G::kStagesV;
+    extern __shared__ __align__(1024) unsigned char smem_pair[];
+    const uint32_t base_s = smem_addr(smem_pair);
+    unsigned char *base = smem_pair;
+    if (base_s & 1023u) {  // the swizzle atoms need 1024-byte alignment
+        if (threadIdx.x == 0) {
+            grid_dependency_wait();
+            flag(a, KV_STATUS_BAD_CONTEXT);
+        }
+        return;
+    }
+    const uint32_t sQ = base_s + G::kOffQ, sK = base_s + G::kOffK, sV = base_s + G::kOffV;
+    uint64_t *fullK = reinterpret_cast<uint64_t *>(base + G::kOffBar);
+    uint64_t *emptyK = fullK + SK;
+    uint64_t *fullV = emptyK + SK;
+    uint64_t *emptyV = fullV + SV;
+    uint64_t *s_full = emptyV + SV;  // [2]: S of the tile's current KV tile is in tensor memory
+    uint64_t *s_read = s_full + 2;   // [2]: the softmax has read it (used with P apart from S)
+    uint64_t *p_full = s_read + 2;   // [2]: P is in tensor memory (and the last V rows zeroed)
+    uint64_t *pv_done = p_full + 2;  // [2]: O += P V is done
+    uint64_t *o_done = pv_done + 2;  // every MMA of the CTA is done (one phase)
+    uint64_t *q_ready = o_done + 1;  // [2]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(q_ready + 2);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    volatile int *zero_flag = abort_flag + 1;
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // grid: x the kv head, y the pair of query tiles (later rows, which see more KV, first), z the
+    // sequence's rank by context length (longest first, ties by index). CTAs start in that order, so
+    // with one CTA per SM the long ones do not wait for the short ones' SMs at the end of the launch
+    int b = blockIdx.z;
+    if (a.B <= kRankMax) {
+        __shared__ int s_lens[kRankMax];
+        __shared__ int s_seq;
+        for (int i = tid; i < a.B; i += kThreads)
+            s_lens[i] = __ldg(a.context_lens + i);
+        __syncthreads();
+        for (int i = tid; i < a.B; i += kThreads) {
+            const int ci = s_lens[i];
+            int rank = 0;
+            for (int k = 0; k < a.B; ++k)
+                rank += (s_lens[k] > ci || (s_lens[k] == ci && k < i)) ? 1 : 0;
+            if (rank == static_cast<int>(blockIdx.z))  // the ranks are a permutation: one writer
+                s_seq = i;
+        }
+        __syncthreads();
+        b = s_seq;
+    }
+    const int j = blockIdx.x;
+    const int tile = a.max_tiles - 1 - static_cast<int>(blockIdx.y);  // pair of query tiles
+    const int g = a.group;
+    const int q0 = __ldg(a.query_start + b);
+    const int n = __ldg(a.query_start + b + 1) - q0;
+    const int c = __ldg(a.context_lens + b);
+    if (n <= 0)
+        return;
+    if (n > c || c > a.W * kBlockTokens || n > a.max_query_len) {
+        if (tid == 0 && j == 0 && tile == a.max_tiles - 1) {
+            grid_dependency_wait();
+            flag(a, KV_STATUS_BAD_CONTEXT);
+        }
+        return;
+    }
+    const int rows_total = n * g;
+    const int row0 = tile * 2 * kRows;
+    if (row0 >= rows_total)
+        return;
+    const int p0 = c - n;
+    const int last_row = min(row0 + 2 * kRows, rows_total) - 1;
+    const int kv_len = p0 + last_row / g + 1;
+    const int nblk = (kv_len + kBlockTokens - 1) / kBlockTokens;
+    const int ntiles = (kv_len + kTok - 1) / kTok;
+    constexpr int fmt = E::kDtype == KV_DTYPE_BF16 ? 1 : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < SK; ++s) {
+            mbar_init(&fullK[s], 1);
+            mbar_init(&emptyK[s], 1);
+        }
+        for (int s = 0; s < SV; ++s) {
+            mbar_init(&fullV[s], 1);
+            mbar_init(&emptyV[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&s_read[t], kRows);
+            mbar_init(&p_full[t], kRows);
+            mbar_init(&pv_done[t], 1);
+            mbar_init(&q_ready[t], kRows);
+        }
+        mbar_init(o_done, 1);
+        mbar_fence_init();
+        *abort_flag = 0;
+        *zero_flag = 0;
+    }
+    if (warp == kMmaWarp)
+        tmem_alloc(tmem_slot, G::kTmemCols);
+    tcgen05_before_sync();
+    __syncthreads();
+    tcgen05_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kProducerWarp) {
+        // ---------------- producer: block ids -> TMA loads ----------------
+        if (lane == 0) {
+            tma_prefetch_descriptor(&tmK);
+            tma_prefetch_descriptor(&tmV);
+        }
+        grid_dependency_wait();
+        grid_launch_dependents();
+        const int32_t *trow = a.block_tables + static_cast<size_t>(b) * a.W;
+        constexpr int kBlk = kTok / kBlockTokens;
+        // K (which = 0) or V (which = 1) of KV tile t: wait for its stage, then one lane per block
+        auto issue = [&](int t, int which) -> bool {
+            const int ns = which == 0 ? SK : SV;
+            const int s = t % ns;
+            const int nb = min(kBlk, nblk - t * kBlk);
+            int blk = 0;
+            if (lane < nb) {
+                blk = __ldg(trow + t * kBlk + lane);
+                if (blk < 0 || blk >= a.num_blocks) {
+                    if (which == 0)
+                        flag(a, KV_STATUS_BAD_BLOCK_ID);
+                    blk = 0;
+                }
+            }
+            uint64_t *fb = which == 0 ? &fullK[s] : &fullV[s];
+            uint64_t *eb = which == 0 ? &emptyK[s] : &emptyV[s];
+            int ok = 1;
+            if (lane == 0) {
+                ok = mbar_wait_bounded(eb, ((t / ns) & 1) ^ 1, abort_flag);
+                if (ok)
+                    mbar_arrive_expect_tx(fb, nb * G::kChunks * 2048);
+                else {
+                    *abort_flag = 1;
+                    flag(a, KV_STATUS_WAIT_TIMEOUT);
+                }
+            }
+            ok = __shfl_sync(kFullMask, ok, 0);
+            if (!ok)
+                return false;
+            __syncwarp();
+            if (lane < nb) {
+                const uint32_t dst = (which == 0 ? sK : sV) + s * G::kStageBytes + lane * 2048;
+                const CUtensorMap *tm = which == 0 ? &tmK : &tmV;
+#pragma unroll
+                for (int ch = 0; ch < G::kChunks; ++ch)
+                    tma_load_4d_nohint(dst + ch * G::kChunkBytes, tm, ch * 64, 0, j, blk, fb);
+            }
+            return true;
+        };
+        // K(t), V(t) for each t: the order in which the MMAs need them and free their stages
+        int issuedK = 0, issuedV = 0;
+        bool go = true;
+        for (int t = 0; t < ntiles && go; ++t) {
+            if ((go = issue(t, 0)))
+                issuedK = t + 1;
+            if (go && (go = issue(t, 1)))
+                issuedV = t + 1;
+        }
+        // no load may land after this CTA exits: wait (bounded) for the last ones
+        if (lane == 0) {
+            for (int t = max(0, issuedK - SK); t < issuedK; ++t)
+                mbar_wait_bounded(&fullK[t % SK], (t / SK) & 1, zero_flag);
+            for (int t = max(0, issuedV - SV); t < issuedV; ++t)
+                mbar_wait_bounded(&fullV[t % SV], (t / SV) & 1, zero_flag);
+        }
+    } else if (warp == kMmaWarp) {
+        // ---------------- MMA issuer (one thread) ----------------
+        grid_dependency_wait();
+        grid_launch_dependents();
+        if (lane == 0) {
+            const uint32_t idesc_s = umma_idesc_f16(kRows, kTok, fmt, 0, 0);
+            const uint32_t idesc_o = umma_idesc_f16(kRows, D, fmt, 0, 1);
+            // S of query tile t for KV tile jt: Q_t K^T into its S columns
+            auto issue_s = [&](int jt, int t) {
+                const uint32_t kst = sK + (jt % SK) * G::kStageBytes;
+                const uint32_t qt = sQ + t * G::kQBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32;  // 16 elements along the 128-byte row
+                    const uint64_t ad = umma_desc_sw128(qt + (kk >> 2) * (kRows * 128) + koff, 16, 1024);
+                    const uint64_t bd = umma_desc_sw128(kst + (kk >> 2) * G::kChunkBytes + koff, 16, 1024);
+                    umma_f16(tmem + G::scol(t), ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[t]);
+            };
+            // O_t += P_t V for KV tile jt, P (16-bit pairs) read from tensor memory
+            auto issue_pv = [&](int jt, int t) {
+                const uint32_t vst = sV + (jt % SV) * G::kStageBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTok / 16; ++kk) {
+                    const uint64_t bd = umma_desc_sw128(vst + kk * 2048, G::kChunkBytes, 1024);
+                    umma_f16_tmem_a(tmem + G::ocol(t), tmem + G::pcol(t) + kk * 8, bd, idesc_o,
+                                    (jt > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&pv_done[t]);
+            };
+            // Issue order: per KV tile, tile 0's P V and next S, then tile 1's. This keeps the two softmaxes
+            // about half a cycle apart, so they take turns on the special-function units; issuing whatever is
+            // ready first (watching both tiles' barriers) let them drift into step and ran 20 % slower at D = 128
+            bool ok = mbar_wait_bounded(&q_ready[0], 0, abort_flag) && mbar_wait_bounded(&fullK[0], 0, abort_flag);
+            if (ok) {
+                tcgen05_after_sync();
+                issue_s(0, 0);
+                ok = mbar_wait_bounded(&q_ready[1], 0, abort_flag);
+            }
+            if (ok) {
+                tcgen05_after_sync();
+                issue_s(0, 1);
+                if (SK < ntiles)  // only a refill waits for this arrival
+                    umma_commit(&emptyK[0]);
+            }
+            for (int jt = 0; jt < ntiles && ok; ++jt) {
+                const bool more = jt + 1 < ntiles;
+                const int kn = (jt + 1) % SK;
+                for (int t = 0; t < 2 && ok; ++t) {
+                    if (G::kSepP && more) {
+                        // the next S goes into columns the softmax has read: it runs during this softmax
+                        if (!mbar_wait_bounded(&s_read[t], jt & 1, abort_flag) ||
+                            (t == 0 && !mbar_wait_bounded(&fullK[kn], ((jt + 1) / SK) & 1, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        tcgen05_after_sync();
+                        issue_s(jt + 1, t);
+                        if (t == 1 && jt + 1 + SK < ntiles)
+                            umma_commit(&emptyK[kn]);
+                    }
+                    if (!mbar_wait_bounded(&p_full[t], jt & 1, abort_flag) ||
+                        (t == 0 && !mbar_wait_bounded(&fullV[jt % SV], (jt / SV) & 1, abort_flag))) {
+                        ok = false;
+                        break;
+                    }
+                    tcgen05_after_sync();
+                    issue_pv(jt, t);
+                    if (t == 1 && jt + SV < ntiles)
+                        umma_commit(&emptyV[jt % SV]);
+                    if (!G::kSepP && more) {
+                        // the next S overwrites this P: after its P V
+                        if ((t == 0 && !mbar_wait_bounded(&fullK[kn], ((jt + 1) / SK) & 1, abort_flag)) ||
+                            !mbar_wait_bounded(&pv_done[t], jt & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tcgen05_after_sync();
+                        issue_s(jt + 1, t);
+                        if (t == 1 && jt + 1 + SK < ntiles)
+                            umma_commit(&emptyK[kn]);
+                    }
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                flag(a, KV_STATUS_WAIT_TIMEOUT);
+            }
+            umma_commit(o_done);
+            mbar_wait_bounded(o_done, 0, zero_flag);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- softmax: warps 4t..4t+3 own query tile t, one row per thread ----------------
+        grid_dependency_wait();  // q may come from the kernel before
+        grid_launch_dependents();
+        const int t = warp >> 2;
+        const int r = tid & (kRows - 1);  // TMEM lane and row of the tile
+        const int row = row0 + t * kRows + r;
+        const bool ok = row < rows_total;
+        const int rowc = min(row, rows_total - 1);
+        const int tok = rowc / g, h = rowc - tok * g;
+        const int pos = p0 + tok;
+        {
+            const uint32_t qt = sQ + t * G::kQBytes;
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D);
+#pragma unroll
+            for (int ch = 0; ch < D / 8; ++ch) {
+                const uint4 v = ok ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t dst = qt + (ch >> 3) * (kRows * 128) + r * 128 + (((ch & 7) ^ (r & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(dst), "r"(v.x), "r"(v.y), "r"(v.z),
+                             "r"(v.w)
+                             : "memory");
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(&q_ready[t]);
+        }
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+        const float sl2 = a.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
+        bool good = true;
+        for (int jt = 0; jt < ntiles; ++jt) {
+            // tcgen05.ld/st are warp-wide: a warp takes every branch below as one
+            if (!__all_sync(kFullMask, mbar_wait_bounded(&s_full[t], jt & 1, abort_flag))) {
+                good = false;
+                break;
+            }
+            tcgen05_after_sync();
+            float x[kTok];
+            {
+                // the row's eight loads in flight together, one wait (reading the row in two halves, each
+                // twice, held fewer registers but ran 7 % slower)
+                uint32_t v[kTok / 16][16];
+#pragma unroll
+                for (int q8 = 0; q8 < kTok / 16; ++q8)
+                    tmem_ld16(lane_base + G::scol(t) + q8 * 16, v[q8]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int q8 = 0; q8 < kTok / 16; ++q8)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        x[q8 * 16 + i] = __uint_as_float(v[q8][i]);
+            }
+            if (G::kSepP) {
+                tcgen05_before_sync();
+                mbar_arrive(&s_read[t]);  // the next S may be written over these columns
+            }
+            const int tok0 = jt * kTok;
+            if (tok0 + kTok - 1 > pos) {  // tokens after this row's position are -inf
+#pragma unroll
+                for (int i = 0; i < kTok; ++i)
+                    x[i] = (tok0 + i <= pos) ? x[i] : -INFINITY;
+            }
+            // the maximum of the raw scores in four chains of three-input maxima (scale > 0, so it scales to
+            // the maximum of the scaled ones)
+            float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int i = 0; i < kTok; i += 2)
+                mx[(i >> 1) & 3] = tc::max3(mx[(i >> 1) & 3], x[i], x[i + 1]);
+            const float rmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+            const float xmax = rmax * sl2;
+            bool rescale = false;
+            float alpha = 1.f;
+            if (xmax > m_used + tc::kRescaleLog2) {  // always true on the first tile (m_used = -inf)
+                alpha = tc::ex2_approx(m_used - xmax);
+                rescale = jt > 0;
+                m_used = xmax;
+                l *= alpha;
+            }
+            if (!rescale)
+                alpha = 1.f;
+            const bool any_rescale = __any_sync(kFullMask, rescale);
+            // O is rescaled, and (P apart from S) P rewritten, once the previous P V is done with them;
+            // with P over S that is already so: S of this tile was issued after it
+            if (jt > 0 && (any_rescale || G::kSepP)) {
+                if (!__all_sync(kFullMask, mbar_wait_bounded(&pv_done[t], (jt - 1) & 1, abort_flag))) {
+                    good = false;
+                    break;
+                }
+                tcgen05_after_sync();
+            }
+            if (any_rescale) {
+                uint32_t v[16];
+#pragma unroll 1
+                for (int q4 = 0; q4 < D / 16; ++q4) {
+                    tmem_ld16(lane_base + G::ocol(t) + q4 * 16, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        v[i] = __float_as_uint(__uint_as_float(v[i]) * alpha);
+                    tmem_st16(lane_base + G::ocol(t) + q4 * 16, v);
+                }
+                tmem_wait_st();
+            }
+            // P = 2^(x scale log2(e) - m_used), two scores at a time (one paired FMA), on the special-
+            // function unit (computing part of them with a polynomial on the FMA pipe instead, and computing
+            // P against the running maximum before the tile's own maximum was known, both measured slower);
+            // the row sum in four paired chains
+            const unsigned long long sc2 = tc::f2pack(sl2, sl2), mm2 = tc::f2pack(-m_used, -m_used);
+            unsigned long long ps2[4] = {tc::f2pack(0.f, 0.f), tc::f2pack(0.f, 0.f), tc::f2pack(0.f, 0.f),
+                                         tc::f2pack(0.f, 0.f)};
+#pragma unroll
+            for (int qq = 0; qq < kTok / 32; ++qq) {
+                uint32_t w[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int i0 = qq * 32 + 2 * e;
+                    float ya, yb;
+                    tc::f2unpack(tc::fma_f2(tc::f2pack(x[i0], x[i0 + 1]), sc2, mm2), ya, yb);
+                    const float pa = tc::ex2_approx(ya), pb = tc::ex2_approx(yb);
+                    ps2[e & 3] = tc::add_f2(ps2[e & 3], tc::f2pack(pa, pb));
+                    w[e] = E::pack(pa, pb);
+                }
+                tmem_st16(lane_base + G::pcol(t) + qq * 16, w);
+            }
+            tmem_wait_st();
+            {
+                float s0, s1, s2, s3, s4, s5, s6, s7;
+                tc::f2unpack(ps2[0], s0, s1);
+                tc::f2unpack(ps2[1], s2, s3);
+                tc::f2unpack(ps2[2], s4, s5);
+                tc::f2unpack(ps2[3], s6, s7);
+                l += ((s0 + s1) + (s2 + s3)) + ((s4 + s5) + (s6 + s7));
+            }
+            // rows of the last KV tile from the CTA's last visible token on hold whatever the pool
+            // holds past the context, or what the stage held before: tile 0's warps zero those V rows
+            // (P is 0 there, and 0 * V must stay 0) once V's loads have landed; tile 1's P V is issued
+            // after tile 0's P is full, so after the zeroing
+            const int vrow0 = kv_len - tok0;
+            if (t == 0 && vrow0 < kTok) {
+                if (!__all_sync(kFullMask, mbar_wait_bounded(&fullV[jt % SV], (jt / SV) & 1, abort_flag))) {
+                    good = false;
+                    break;
+                }
+                const uint32_t vst = sV + (jt % SV) * G::kStageBytes;
+                const int cnt = (kTok - vrow0) * G::kChunks * 8;
+                for (int idx = r; idx < cnt; idx += kRows) {
+                    const int rr = vrow0 + idx / (G::kChunks * 8);
+                    const int rem = idx % (G::kChunks * 8);
+                    asm volatile("st.shared.v4.b32 [%0], {%1,%1,%1,%1};" ::"r"(vst + (rem >> 3) * G::kChunkBytes +
+                                                                               rr * 128 + ((rem & 7) << 4)),
+                                 "r"(0)
+                                 : "memory");
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the P V reads these zeros
+            }
+            tcgen05_before_sync();
+            if (a.slow_softmax && warp == 0 && jt == 0) {
+                // test hook: let the other warps run ahead of this one (a bounded wait)
+                const uint64_t t0 = global_timer_ns();
+                while (global_timer_ns() - t0 < 30000u)
+                    __nanosleep(1000);
+            }
+            mbar_arrive(&p_full[t]);
+        }
+        // epilogue: O / l. The tile's four warps decide together (a warp that gave up must not leave the
+        // others at a barrier)
+        const bool done = mbar_wait_bounded(o_done, 0, abort_flag);
+        if (named_barrier_and(1 + t, kRows, good && done)) {
+            tcgen05_after_sync();
+            const float inv = 1.f / l;
+            if (a.out_f32) {
+                const size_t orow = (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D;
+                uint32_t v[16];
+#pragma unroll 1
+                for (int q4 = 0; q4 < D / 16; ++q4) {
+                    tmem_ld16(lane_base + G::ocol(t) + q4 * 16, v);
+                    tmem_wait_ld();
+                    if (ok) {
+                        float4 *f = reinterpret_cast<float4 *>(reinterpret_cast<float *>(a.out) + orow + q4 * 16);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            f[i] = make_float4(__uint_as_float(v[4 * i]) * inv, __uint_as_float(v[4 * i + 1]) * inv,
+                                               __uint_as_float(v[4 * i + 2]) * inv,
+                                               __uint_as_float(v[4 * i + 3]) * inv);
+                    }
+                }
+            } else {
+                // Each thread's row goes to shared memory (the K/V stages: every MMA is done with them) and out
+                // with one bulk copy, issued by the thread itself: a row of O per thread stored directly would
+                // make every warp store touch 32 rows. Rows are padded to 2D + 16 bytes, so that the 32 rows a
+                // warp writes at once fall on different banks.
+                constexpr int kPitch = 2 * D + 16;
+                static_assert(2 * kRows * kPitch <= (G::kStagesK + G::kStagesV) * G::kStageBytes, "staging");
+                const uint32_t srow = sK + (t * kRows + r) * kPitch;
+                const size_t orow = (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D;
+                uint32_t v[16];
+#pragma unroll 1
+                for (int q4 = 0; q4 < D / 16; ++q4) {
+                    tmem_ld16(lane_base + G::ocol(t) + q4 * 16, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int hlf = 0; hlf < 2; ++hlf)
+                        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(srow + q4 * 32 + hlf * 16),
+                                     "r"(E::pack(__uint_as_float(v[8 * hlf]) * inv, __uint_as_float(v[8 * hlf + 1]) * inv)),
+                                     "r"(E::pack(__uint_as_float(v[8 * hlf + 2]) * inv, __uint_as_float(v[8 * hlf + 3]) * inv)),
+                                     "r"(E::pack(__uint_as_float(v[8 * hlf + 4]) * inv, __uint_as_float(v[8 * hlf + 5]) * inv)),
+                                     "r"(E::pack(__uint_as_float(v[8 * hlf + 6]) * inv, __uint_as_float(v[8 * hlf + 7]) * inv))
+                                     : "memory");
+                }
+                if (ok) {
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the copy reads these writes
+                    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(a.out + orow),
+                                 "r"(srow), "n"(2 * D)
+                                 : "memory");
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                    // the copy has read the row before the CTA (and its shared memory) is gone
+                    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                }
+            }
+        } else if (lane == 0) {
+            *abort_flag = 1;
+            flag(a, KV_STATUS_WAIT_TIMEOUT);
+        }
+    }
+    // every thread is past its last tensor-memory access; release it
+    tcgen05_before_sync();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tcgen05_after_sync();
+        tmem_dealloc(tmem, G::kTmemCols);
+    }
+}
+
+}  // namespace pair
 }  // namespace prefill
 }  // namespace pkv
 
@@ -947,6 +1504,16 @@ PrefillFn pick_prefill_tc(int dtype, int D, int *smem)
     if (dtype == KV_DTYPE_FP16)
         return D == 64 ? prefill_tc_kernel<ElemF16, 64> : prefill_tc_kernel<ElemF16, 128>;
     return D == 64 ? prefill_tc_kernel<ElemBf16, 64> : prefill_tc_kernel<ElemBf16, 128>;
+}
+
+PrefillFn pick_prefill_pair(int dtype, int D, int *smem)
+{
+    using namespace pkv;
+    using namespace pkv::prefill::pair;
+    *smem = D == 64 ? Geo<64>::kSmemBytes : Geo<128>::kSmemBytes;
+    if (dtype == KV_DTYPE_FP16)
+        return D == 64 ? prefill_pair_kernel<ElemF16, 64> : prefill_pair_kernel<ElemF16, 128>;
+    return D == 64 ? prefill_pair_kernel<ElemBf16, 64> : prefill_pair_kernel<ElemBf16, 128>;
 }
 
 PrefillFn pick_prefill(int dtype, int D, int *smem)
@@ -1004,16 +1571,19 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
     const int group = Hq / Hkv;
     if (!(scale > 0.f))
         return KV_ERR_ARG;
-    const bool use_tc = pkv_prefill_path() != 2;  // tcgen05 unless the mma.sync path is asked for
-    const int rows_per_cta = use_tc ? tc::kRows : kRows;
+    // 1: tcgen05, one query tile per CTA; 2: mma.sync; 3 (and auto): tcgen05, two query tiles per CTA
+    const int path = pkv_prefill_path() == 0 ? 3 : pkv_prefill_path();
+    const int rows_per_cta = path == 3 ? 2 * pair::kRows : path == 1 ? tc::kRows : kRows;
     const long long tiles = (static_cast<long long>(max_query_len) * group + rows_per_cta - 1) / rows_per_cta;
-    if (tiles > (1ll << 31) - 1)
+    if (tiles > (path == 3 ? 65535ll : (1ll << 31) - 1))
         return KV_ERR_ARG;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
         return KV_ERR_CUDA;
     int smem = 0;
-    PrefillFn fn = use_tc ? pick_prefill_tc(dtype, D, &smem) : pick_prefill(dtype, D, &smem);
+    PrefillFn fn = path == 3 ? pick_prefill_pair(dtype, D, &smem)
+                   : path == 1 ? pick_prefill_tc(dtype, D, &smem)
+                               : pick_prefill(dtype, D, &smem);
     if (!prepare_prefill(fn, smem, dev))
         return KV_ERR_CUDA;
     CUtensorMap tmK, tmV;
@@ -1040,8 +1610,9 @@ extern "C" kv_status paged_attention_prefill(void *out, const void *q, const voi
     a.out_f32 = pkv_out_f32();
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
-    cfg.blockDim = dim3(use_tc ? tc::kThreads : kThreads);
+    cfg.gridDim = path == 3 ? dim3(static_cast<unsigned>(Hkv), static_cast<unsigned>(tiles), static_cast<unsigned>(B))
+                            : dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(Hkv), static_cast<unsigned>(B));
+    cfg.blockDim = dim3(path == 3 ? pair::kThreads : path == 1 ? tc::kThreads : kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = reinterpret_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];

@@ -62,7 +62,7 @@ def test_option_ranges_need_no_gpu(pkv):
     lib = ctypes.CDLL(pkv.LIB_PATH)
     lib.kv_decode_set_option.restype = ctypes.c_int
     lib.kv_decode_get_option.restype = ctypes.c_int
-    cases = {pkv.KV_OPT_PREFILL_PATH: ([0, 1, 2], [-1, 3]),
+    cases = {pkv.KV_OPT_PREFILL_PATH: ([0, 1, 2, 3], [-1, 4]),
              pkv.KV_OPT_TEST_SLOW_SOFTMAX: ([0, 1], [-1, 2]),
              pkv.KV_OPT_TEST_DROP_LOAD: ([0, 5], [-1]),
              pkv.KV_OPT_ITEM_COST: ([-1, 0, 64], [-2, 65]),

@@ -12,7 +12,7 @@ from gpu_cases import compare
 
 pytestmark = pytest.mark.gpu
 
-PREFILL_PATHS = {"tcgen05": 1, "mma_sync": 2}
+PREFILL_PATHS = {"tcgen05": 1, "mma_sync": 2, "tcgen05_pair": 3}
 
 
 @pytest.fixture(autouse=True)
@@ -150,11 +150,12 @@ def test_stale_shared_memory_stays_out(pkv, oracle_mod, cuda_device, D, path):
     run_case(pkv, oracle_mod, case, f"after a NaN launch, D{D} {path}")
 
 
+@pytest.mark.parametrize("path", ["tcgen05", "tcgen05_pair"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_slow_softmax_warp_keeps_the_result(pkv, oracle_mod, cuda_device, D):
+def test_slow_softmax_warp_keeps_the_result(pkv, oracle_mod, cuda_device, D, path):
     """The first softmax warp of every CTA hands over its first P ~30 us late, so the other warps run a
     tile ahead of it: the P V of a tile must still wait for all of that tile's P."""
-    pkv.set_option(pkv.KV_OPT_PREFILL_PATH, PREFILL_PATHS["tcgen05"])
+    pkv.set_option(pkv.KV_OPT_PREFILL_PATH, PREFILL_PATHS[path])
     pkv.set_option(pkv.KV_OPT_TEST_SLOW_SOFTMAX, 1)
     try:
         Hq, Hkv = (32, 8) if D == 128 else (20, 4)
@@ -162,6 +163,6 @@ def test_slow_softmax_warp_keeps_the_result(pkv, oracle_mod, cuda_device, D):
         prior = [0, 33, 200, 111, 40, 700]
         cfg = workloads.PrefillConfig("test", Hq, Hkv, D, len(chunk), 0, 0, 0, 48, seed=21 + D)
         case = PrefillCase(cfg, cuda_device, chunk_lens=chunk, prior_lens=prior)
-        run_case(pkv, oracle_mod, case, f"slow first softmax warp, D{D}")
+        run_case(pkv, oracle_mod, case, f"slow first softmax warp, D{D} {path}")
     finally:
         pkv.set_option(pkv.KV_OPT_TEST_SLOW_SOFTMAX, 0)

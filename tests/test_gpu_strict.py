@@ -82,7 +82,7 @@ def test_multi_layer_launch_meets_the_stated_bounds(pkv, oracle_mod, cuda_device
         compare_strict(out[layer], ref, f"config {cid} layer {layer} of a {L}-layer launch")
 
 
-@pytest.mark.parametrize("prefill_path", [1, 2])
+@pytest.mark.parametrize("prefill_path", [1, 2, 3])
 @pytest.mark.parametrize("key", sorted(workloads.PREFILL_CONFIGS))
 def test_prefill_fp32_output(pkv, oracle_mod, cuda_device, key, prefill_path):
     """The chunked prefill's fp32 result: max abs <= 5e-3 outright. Its probabilities are rounded to the element
