@@ -11,15 +11,18 @@
 //     out[i][h] = sum_{t <= p} softmax_t(scale * <q[i][h], K_t>) V_t.
 //
 // Work decomposition. The query rows of one (sequence, kv head) are the chunk's
-// tokens times the group's query heads, token-major; a CTA takes 64 of them
-// (4 warps x 16 rows: the group's heads share every K/V tile) and reads the
-// sequence's KV blocks up to the last position among its rows. CTAs with
-// later rows (more KV) are launched first.
+// tokens times the group's query heads, token-major (the group's heads share
+// every K/V tile); a CTA takes a run of them and reads the sequence's KV blocks
+// up to the last position among its rows. Three kernels compute it, chosen by
+// KV_OPT_PREFILL_PATH: two tiles of 128 rows per CTA on tcgen05 (the default,
+// last in this file), one tile of 128 rows per CTA on tcgen05 (path 1), and
+// the mma.sync kernel below (path 2), kept as the comparison.
 //
-// Pipeline. Warp 4 is the producer: it reads block ids and issues TMA loads of
-// 4 KV blocks (64 tokens) per stage into a ring of 3 stages, guarded by
-// mbarriers with bounded waits. Warps 0-3 compute with tensor cores
-// (mma.sync.m16n8k16, 16-bit inputs, fp32 accumulate): per stage
+// mma.sync kernel. 64 rows per CTA (4 warps x 16 rows); CTAs with later rows
+// (more KV) are launched first. Warp 4 is the producer: it reads block ids and
+// issues TMA loads of 4 KV blocks (64 tokens) per stage into a ring of 3
+// stages, guarded by mbarriers with bounded waits. Warps 0-3 compute with
+// mma.sync.m16n8k16 (16-bit inputs, fp32 accumulate): per stage
 // S[16 rows x 64 tokens] = Q K^T, the causal mask, an fp32 online softmax in
 // base 2 (one rescale of O per stage), then O[16 x D] += P V with P rounded to
 // the element type.
@@ -942,7 +945,9 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
 // tiles: while one tile's softmax runs, the tensor pipe does the other tile's
 // P V and next S. At D = 128 the S of the next tile goes where P of this one
 // is, so it waits for that P V; at D = 64 it only waits until the softmax
-// has read S, and runs while the softmax computes. Every hand-off is an
+// has read S, and runs while the softmax computes. CTAs start longest sequence
+// first (each ranks the batch's context lengths), and the epilogue writes each
+// row of O with one bulk copy from shared memory. Every hand-off is an
 // mbarrier with a bounded wait, as in the one-tile kernel.
 // ===========================================================================
 namespace pair {
