@@ -178,3 +178,32 @@ def test_multi_layer_checks_need_no_gpu(pkv):
     assert call(kn=fake) == pkv.KV_ERR_ARG                       # new K rows without V rows and slots
     assert call(kn=fake, vn=fake, slots=fake + 4) == pkv.KV_ERR_ARG   # misaligned slots
     assert call(B=0) == pkv.KV_OK                                # nothing to do
+
+
+def test_prefill_checks_need_no_gpu(pkv):
+    """paged_attention_prefill refuses bad arguments on the host, before any CUDA call, including a batch whose
+    rows would need more than 65,535 CTAs along the default kernel's second grid dimension (256 rows each)."""
+    lib = ctypes.CDLL(pkv.LIB_PATH)
+    f = lib.paged_attention_prefill
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f.argtypes = [P, P, P, P, P, I, P, P, I, I, I, I, I, I, ctypes.c_float, I, P, P]
+    f.restype = I
+    fake = 1 << 20   # an aligned non-null address; nothing is dereferenced before the checks fail
+    good = dict(out=fake, q=fake, kc=fake, vc=fake, tables=fake, W=4, lens=fake, qs=fake, B=3, maxq=32, nb=4,
+                Hq=64, Hkv=8, D=128, scale=0.1, dtype=0)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return f(a["out"], a["q"], a["kc"], a["vc"], a["tables"], a["W"], a["lens"], a["qs"], a["B"], a["maxq"],
+                 a["nb"], a["Hq"], a["Hkv"], a["D"], a["scale"], a["dtype"], None, None)
+    assert pkv.get_option(pkv.KV_OPT_PREFILL_PATH) == 0
+    assert call(D=96) == pkv.KV_ERR_ARG                  # head dimension
+    assert call(Hkv=6) == pkv.KV_ERR_ARG                 # Hq not a multiple of Hkv
+    assert call(scale=0.0) == pkv.KV_ERR_ARG             # scale must be positive
+    assert call(dtype=2) == pkv.KV_ERR_ARG               # element type
+    assert call(q=fake + 8) == pkv.KV_ERR_ARG            # misaligned rows
+    assert call(qs=None) == pkv.KV_ERR_ARG               # no query offsets
+    # 8 query heads per kv head: ceil(maxq * 8 / 256) tile groups must stay <= 65535
+    assert call(maxq=65535 * 32 + 1) == pkv.KV_ERR_ARG
+    assert call(B=0) == pkv.KV_OK                        # nothing to do
+    assert call(maxq=0) == pkv.KV_OK

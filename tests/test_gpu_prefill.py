@@ -166,3 +166,19 @@ def test_slow_softmax_warp_keeps_the_result(pkv, oracle_mod, cuda_device, D, pat
         run_case(pkv, oracle_mod, case, f"slow first softmax warp, D{D} {path}")
     finally:
         pkv.set_option(pkv.KV_OPT_TEST_SLOW_SOFTMAX, 0)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("B,equal", [(40, True), (300, False)])
+def test_launch_order_covers_every_sequence_once(pkv, oracle_mod, cuda_device, D, B, equal):
+    """The default kernel launches its CTAs longest sequence first: each CTA ranks the batch's context lengths
+    (ties by index) for batches of up to 256 sequences and takes them in order beyond. With every length equal
+    (all ties) and with more sequences than are ranked, every sequence's rows are written, and right."""
+    chunk = [3 + (i % 5) for i in range(B)]
+    prior = [40 - chunk[i] + 3 for i in range(B)] if equal else [(i * 37) % 97 for i in range(B)]
+    if equal:
+        assert len({c + p for c, p in zip(chunk, prior)}) == 1
+    cfg = workloads.PrefillConfig("test", 16, 4, D, B, 0, 0, 0, 8, seed=31 + D + B)
+    case = PrefillCase(cfg, cuda_device, chunk_lens=chunk, prior_lens=prior)
+    out = run_case(pkv, oracle_mod, case, f"launch order, B={B}, D{D}")
+    assert torch.isfinite(out.float()).all(), "rows left unwritten"
