@@ -492,12 +492,33 @@ def pinned_near(tensors, device_index: int):
             os.sched_setaffinity(0, old)
 
 
-def e2e_measure(wl, steps, warmup, world, chunks=4):
+def e2e_groups(L: int, cap: int = 8) -> list[tuple[int, int]]:
+    """Layer groups for the end-to-end step: sizes 1, 2, 4, ... (below `cap`) at the start and the same
+    back down at the end, the layers between in even groups of at most `cap`. Only the first group's inputs
+    and the last group's outputs cross to or from the host with no launch to overlap, so those groups are
+    one layer each; every group is one launch, so the middle ones are large."""
+    cap = max(1, min(cap, L // 2))
+    up, nxt = [], 1
+    while nxt < cap and 2 * (sum(up) + nxt) <= L - cap:
+        up.append(nxt)
+        nxt *= 2
+    rest = L - 2 * sum(up)
+    n_mid = -(-rest // cap)
+    sizes = up + [rest // n_mid + (1 if i < rest % n_mid else 0) for i in range(n_mid)] + up[::-1]
+    bounds, lo = [], 0
+    for sz in sizes:
+        bounds.append((lo, lo + sz))
+        lo += sz
+    assert lo == L and all(hi > lo_ for lo_, hi in bounds)
+    return bounds
+
+
+def e2e_measure(wl, steps, warmup, world):
     """The same step through the C ABI with host buffers: every step copies its inputs from pinned host
-    memory and its outputs back. The layers go in `chunks` groups, each one multi-layer launch: the copies
-    run on two side streams, pipelined with the groups (the tables, lengths and slots, then q, k_new and v_new
-    of each group ahead of its launch; each group's output copied back while later groups run). One CUDA
-    graph. The host buffers are pinned pages on the GPU's NUMA node."""
+    memory and its outputs back. The layers go in groups (e2e_groups: small first and last), each one
+    multi-layer launch: the copies run on two side streams, pipelined with the groups (the tables, lengths
+    and slots, then q, k_new and v_new of each group ahead of its launch; each group's output copied back
+    while later groups run). One CUDA graph. The host buffers are pinned pages on the GPU's NUMA node."""
     cfg = wl.cfg
     L = cfg.n_layers
     dev_index = wl.q.device.index or 0
@@ -510,9 +531,7 @@ def e2e_measure(wl, steps, warmup, world, chunks=4):
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = host_out.numel() * host_out.element_size()
     h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
-    chunks = max(1, min(chunks, L))
-    per = -(-L // chunks)
-    groups = [(lo, min(L, lo + per)) for lo in range(0, L, per)]
+    groups = e2e_groups(L)
     ev_in = [torch.cuda.Event() for _ in groups]
     ev_done = [torch.cuda.Event() for _ in groups]
 

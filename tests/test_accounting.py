@@ -1,7 +1,8 @@
 """CPU checks of the bench's accounting, each against a brute-force count over a drawn layout: the
 algorithmic bytes of one decode layer (logical, and with a shared prefix's blocks counted once) and
-the (query, visible token) pairs of a chunked prefill; and the guard that takes a kernel's DRAM
-traffic only from a profile summary of the current kernel source and workload."""
+the (query, visible token) pairs of a chunked prefill; the guard that takes a kernel's DRAM traffic
+only from a profile summary of the current kernel source and workload; and the end-to-end step's
+groups of layers."""
 import hashlib
 import importlib.util
 import os
@@ -102,3 +103,16 @@ def test_profiled_traffic_needs_the_current_source_and_workload(bench, tmp_path,
     assert bench.profiled_traffic(cfg, "per_layer") is None
     write(src, elem="fp16")                                   # another element type
     assert bench.profiled_traffic(cfg, "per_layer") is None
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 4, 5, 7, 8, 24, 32, 80])
+def test_e2e_layer_groups_cover_every_layer_once(bench, L):
+    """The end-to-end step's groups of layers: contiguous, covering every layer once, none empty, at most 8
+    layers, and one layer at each end (its copies cannot overlap a launch) once there are two or more."""
+    groups = bench.e2e_groups(L)
+    assert groups[0][0] == 0 and groups[-1][1] == L
+    assert all(a[1] == b[0] for a, b in zip(groups, groups[1:]))
+    sizes = [hi - lo for lo, hi in groups]
+    assert all(1 <= sz <= 8 for sz in sizes)
+    if L >= 2:
+        assert sizes[0] == 1 and sizes[-1] == 1
