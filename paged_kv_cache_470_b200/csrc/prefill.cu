@@ -741,7 +741,8 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
         const int tok = rowc / g, h = rowc - tok * g;
         const int pos = p0 + tok;
         {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D);
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(a.q + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D);
 #pragma unroll
             for (int ch = 0; ch < D / 8; ++ch) {
                 const uint4 v = ok ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
@@ -1269,7 +1270,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_
         const int pos = p0 + tok;
         {
             const uint32_t qt = sQ + t * G::kQBytes;
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D);
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(a.q + (static_cast<size_t>(q0 + tok) * a.Hq + j * g + h) * D);
 #pragma unroll
             for (int ch = 0; ch < D / 8; ++ch) {
                 const uint4 v = ok ? __ldg(src + ch) : make_uint4(0u, 0u, 0u, 0u);
@@ -1455,13 +1457,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_
                 for (int q4 = 0; q4 < D / 16; ++q4) {
                     tmem_ld16(lane_base + G::ocol(t) + q4 * 16, v);
                     tmem_wait_ld();
+                    // columns i, i + 1 of the row, scaled, as one word of two 16-bit elements
+                    auto word = [&](int i) {
+                        return E::pack(__uint_as_float(v[i]) * inv, __uint_as_float(v[i + 1]) * inv);
+                    };
 #pragma unroll
                     for (int hlf = 0; hlf < 2; ++hlf)
                         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(srow + q4 * 32 + hlf * 16),
-                                     "r"(E::pack(__uint_as_float(v[8 * hlf]) * inv, __uint_as_float(v[8 * hlf + 1]) * inv)),
-                                     "r"(E::pack(__uint_as_float(v[8 * hlf + 2]) * inv, __uint_as_float(v[8 * hlf + 3]) * inv)),
-                                     "r"(E::pack(__uint_as_float(v[8 * hlf + 4]) * inv, __uint_as_float(v[8 * hlf + 5]) * inv)),
-                                     "r"(E::pack(__uint_as_float(v[8 * hlf + 6]) * inv, __uint_as_float(v[8 * hlf + 7]) * inv))
+                                     "r"(word(8 * hlf)), "r"(word(8 * hlf + 2)), "r"(word(8 * hlf + 4)),
+                                     "r"(word(8 * hlf + 6))
                                      : "memory");
                 }
                 if (ok) {

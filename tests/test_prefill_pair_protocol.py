@@ -12,8 +12,9 @@ waits for the last P V before it writes P again. Barriers behave like mbarriers 
 phase; a wait by parity cannot tell phases two apart); loads land and MMAs complete late, MMAs and their
 commits in issue order; an MMA may run before an earlier one into another accumulator (tcgen05.mma
 orders only MMAs with the same accumulator and shape), and a commit arrives once every MMA before it is
-done, which is why an S written where a P V still reads must wait for that P V's commit. A random scheduler runs many interleavings and checks that every read sees
-the data of its own tile and that no run deadlocks. Mistakes are planted and must be caught.
+done, which is why an S written where a P V still reads must wait for that P V's commit. A random
+scheduler runs many interleavings and checks that every read sees the data of its own tile and that no
+run deadlocks. Mistakes are planted and must be caught.
 """
 import random
 
