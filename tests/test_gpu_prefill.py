@@ -99,12 +99,14 @@ def test_single_token_chunk_matches_the_decode(pkv, cuda_device):
 
 
 @pytest.mark.parametrize("path", sorted(PREFILL_PATHS))
-def test_full_size_prefill_workload(pkv, oracle_mod, cuda_device, path):
-    """The bench's prefill workload (LLaMA-3-8B shape), three of its sequences against the oracle."""
+@pytest.mark.parametrize("key,elem", [("llama3_8b", "bf16"), ("llama3_8b", "fp16"), ("0p5b", "bf16")])
+def test_full_size_prefill_workload(pkv, oracle_mod, cuda_device, path, key, elem):
+    """The bench's prefill workloads (LLaMA-3-8B and 0.5B shapes), three sequences of each against the oracle."""
+    from dataclasses import replace
     pkv.set_option(pkv.KV_OPT_PREFILL_PATH, PREFILL_PATHS[path])
-    cfg = workloads.PREFILL_CONFIGS["llama3_8b"]
+    cfg = replace(workloads.PREFILL_CONFIGS[key], elem=elem)
     case = PrefillCase(cfg, cuda_device)
-    run_case(pkv, oracle_mod, case, f"full-size prefill {path}", rows=[0, 7, 15])
+    run_case(pkv, oracle_mod, case, f"full-size prefill {key} {elem} {path}", rows=[0, 7, 15])
 
 
 @pytest.mark.parametrize("path", sorted(PREFILL_PATHS))
