@@ -1090,7 +1090,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             atomicOr(a.status, KV_STATUS_BAD_BLOCK_ID);
         const int NL = a.prod_lanes;
         Cursor cur = cur0;
-        int u = 0, issued = 0;
+        int u = 0, issued = 0;  // units [0, issued) issued in order (every lane of their round got through)
+        unsigned went = 0;      // if a round stopped midway: unit issued + l was issued (bit l, l < NL)
         bool stop = false, first_batch = true;
         while (u < count && !stop) {
             const int run = min(cur.n - cur.off, count - u);
@@ -1133,6 +1134,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                         }
                     }
                     if (!__all_sync(kFull, ok)) {
+                        went = __ballot_sync(kFull, ok && lane < NL && i < m);  // (units below `pre`: early)
                         stop = true;
                         break;
                     }
@@ -1143,11 +1145,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if (u < count)
                 cursor_next_item(a, cur);
         }
-        // No load may land after this CTA exits: wait (bounded) for the last ones.
+        // No load may land after this CTA exits: wait (bounded) for the last S units issued in order, and for
+        // those issued in a round that stopped midway. A unit whose stage such a unit refilled had landed.
         if (lane < NL) {
-            for (int v = max(0, issued - S); v < issued; ++v)
-                if (v % NL == lane)
+            for (int v = max(0, issued - S); v < issued; ++v) {
+                const int l = v + S - issued;  // the lane whose unit of the stopped round refilled v's stage
+                if (v % NL == lane && !(l < NL && ((went >> l) & 1u)))
                     mbar_wait_bounded(&full[v % S], (v / S) & 1, misc + kMiscZero);
+            }
+            if ((went >> lane) & 1u)
+                mbar_wait_bounded(&full[(issued + lane) % S], ((issued + lane) / S) & 1, misc + kMiscZero);
         }
         return;
     }
