@@ -795,6 +795,10 @@ def run_ours(args, world, rank, local):
         r = prefill_measure(pkv, device, cfg.elem, reps=args.steps, keys=(args.profile_prefill,))
         print(json.dumps(r), flush=True)
         return
+    if args.profile_blocks:
+        r = block_moves_measure(Workload(cfg, device), measured_peak()[0], reps=args.steps)
+        print(json.dumps(r), flush=True)
+        return
     torch.cuda.nvtx.range_push(f"workload {cfg.cid}")
     head = measure_config(args, cfg, device, world, rank, headline=True)
     torch.cuda.nvtx.range_pop()
@@ -907,6 +911,9 @@ def main(argv=None):
     ap.add_argument("--per-layer", action="store_true", help="with --profile-step: the per-layer step")
     ap.add_argument("--profile-prefill", choices=sorted(workloads.PREFILL_CONFIGS), default=None,
                     help="only run the chunked-prefill workload: 3 warm-up and --steps timed launches (for ncu)")
+    ap.add_argument("--profile-blocks", action="store_true",
+                    help="only run the block moves of --config (swap-out gather, swap-in scatter, copies): 2 warm-up "
+                         "and --steps timed launches of each (for ncu)")
     ap.add_argument("--grid", type=int, default=0, help="decode CTAs per launch (0: one per SM)")
     ap.add_argument("--prefill-path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="chunked prefill kernel: 0 auto, 1 tcgen05 one query tile per CTA, 2 mma.sync, "

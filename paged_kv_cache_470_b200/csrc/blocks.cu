@@ -14,12 +14,15 @@
 //                           swapped out and back)
 //
 // One warp moves one block of one tensor with 16-byte loads and stores (16 * Hkv
-// * D * 2 bytes, a multiple of 256), many blocks in flight.
+// * D * 2 bytes, a multiple of 256): each lane issues four loads before their four
+// stores, and a grid of resident CTAs strides over the (tensor, block) items.
 #include "pkv_device.cuh"
 #include "nvtx_range.h"
 #include "pagedkv.h"
 
 #include <cuda_runtime.h>
+
+#include <atomic>
 
 namespace pkv {
 
@@ -58,7 +61,15 @@ __global__ void __launch_bounds__(256) block_move_kernel(const __grid_constant__
         uint4 *packed = buf + (static_cast<long long>(c) * n + i) * chunks_per_block;
         const uint4 *src = (mode == 2) ? packed : cache + s * chunks_per_block;
         uint4 *dst = (mode == 1) ? packed : cache + d * chunks_per_block;
-        for (int k = lane; k < chunks_per_block; k += 32)
+        int k = lane;
+        for (; k + 96 < chunks_per_block; k += 128) {
+            const uint4 a0 = src[k], a1 = src[k + 32], a2 = src[k + 64], a3 = src[k + 96];
+            dst[k] = a0;
+            dst[k + 32] = a1;
+            dst[k + 64] = a2;
+            dst[k + 96] = a3;
+        }
+        for (; k < chunks_per_block; k += 32)
             dst[k] = src[k];
     }
 }
@@ -66,6 +77,27 @@ __global__ void __launch_bounds__(256) block_move_kernel(const __grid_constant__
 }  // namespace pkv
 
 namespace {
+
+// CTAs of block_move_kernel (256 threads) resident on the current device at once, per device.
+long long resident_move_ctas()
+{
+    constexpr int kMaxDevices = 64;
+    static std::atomic<long long> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 0;
+    long long v = cache[dev].load();
+    if (v == 0) {
+        int sms = 0, per_sm = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pkv::block_move_kernel, 256, 0) != cudaSuccess ||
+            sms < 1 || per_sm < 1)
+            return 0;
+        v = static_cast<long long>(sms) * per_sm;
+        cache[dev].store(v);
+    }
+    return v;
+}
 
 kv_status launch_move(void *const *caches, int n_caches, void *buf, const int32_t *src_ids, const int32_t *dst_ids,
                       int n, int num_blocks, int Hkv, int D, int dtype, int mode, int32_t *error_flag,
@@ -89,8 +121,11 @@ kv_status launch_move(void *const *caches, int n_caches, void *buf, const int32_
     const int chunks = 16 * Hkv * D * 2 / 16;
     const int threads = 256;
     long long blocks = (static_cast<long long>(n) * n_caches * 32 + threads - 1) / threads;
-    if (blocks > 4096)
-        blocks = 4096;
+    const long long resident = resident_move_ctas();  // one wave: the rest is strided over
+    if (resident <= 0)
+        return KV_ERR_CUDA;
+    if (blocks > resident)
+        blocks = resident;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(blocks));
     cfg.blockDim = dim3(threads);

@@ -32,6 +32,7 @@ def ids_on(device, ids):
     (8, 128, torch.float16, 3, 300),
     (2, 64, torch.bfloat16, 64, 700),     # one launch over 64 tensors; grid-stride loop taken
     (1, 8, torch.float16, 2, 5),
+    (3, 24, torch.bfloat16, 2, 9),        # 144 chunks per block: four-chunk rounds, then a tail of 16
 ])
 def test_block_moves_bit_exact(pkv, oracle_mod, cuda_device, Hkv, D, dtype, n_caches, n):
     rng = np.random.default_rng(n)
