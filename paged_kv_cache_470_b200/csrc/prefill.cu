@@ -953,6 +953,21 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
 // ===========================================================================
 namespace pair {
 
+// Non-blocking test of an mbarrier phase (test_wait never suspends the thread, so one thread can watch
+// several barriers in turn).
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 constexpr int kRows = 128;     // query rows per tile; a CTA takes two
 constexpr int kTok = 128;      // KV tokens per tile (8 blocks)
 constexpr int kThreads = 320;  // 8 softmax warps, the producer warp, the MMA warp
@@ -1195,9 +1210,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_
                 }
                 umma_commit(&pv_done[t]);
             };
-            // Issue order: per KV tile, tile 0's P V and next S, then tile 1's. This keeps the two softmaxes
-            // about half a cycle apart, so they take turns on the special-function units; issuing whatever is
-            // ready first (watching both tiles' barriers) let them drift into step and ran 20 % slower at D = 128
+            // Issue order at D = 128 (P over S): per KV tile, tile 0's P V and next S, then tile 1's. This keeps
+            // the two softmaxes about half a cycle apart, so they take turns on the special-function units;
+            // issuing whatever is ready first (watching both tiles' barriers) let them drift into step and ran
+            // 20 % slower there. At D = 64 the next S does not wait for a P V, and ready-first is the order.
             bool ok = mbar_wait_bounded(&q_ready[0], 0, abort_flag) && mbar_wait_bounded(&fullK[0], 0, abort_flag);
             if (ok) {
                 tcgen05_after_sync();
@@ -1210,22 +1226,56 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_
                 if (SK < ntiles)  // only a refill waits for this arrival
                     umma_commit(&emptyK[0]);
             }
-            for (int jt = 0; jt < ntiles && ok; ++jt) {
+            if (G::kSepP) {
+                // P apart from S (D = 64): whichever tile's next MMA is ready goes first. S(j + 1) of a tile
+                // needs only that its softmax has read S(j) and that K(j + 1) has landed, P V(j) that P(j)
+                // is full and V(j) has landed; in the fixed order below, a tile's next S waited behind the
+                // other tile's P (a timestamp trace: ~1,160 cycles of each ~3,280-cycle query-tile cycle
+                // spent waiting for S). A K or V stage is released by a commit after the second of the
+                // two tiles' MMAs that read it; tile 1's P V of the last KV tile follows tile 0's, whose
+                // P-full arrival comes after the zeroing of that tile's V rows past the context.
+                int ns[2] = {1, 1};  // next S per tile (S of KV tile 0 went out above)
+                int np[2] = {0, 0};  // next P V per tile
+                uint64_t since = global_timer_ns();
+                uint32_t idle = 0;
+                while (ok && (np[0] < ntiles || np[1] < ntiles)) {
+                    bool moved = false;
+#pragma unroll
+                    for (int t = 0; t < 2; ++t) {
+                        const int js = ns[t];
+                        if (js < ntiles && mbar_test(&s_read[t], (js - 1) & 1) &&
+                            mbar_test(&fullK[js % SK], (js / SK) & 1)) {
+                            tcgen05_after_sync();
+                            issue_s(js, t);
+                            if (ns[t ^ 1] > js && js + SK < ntiles)
+                                umma_commit(&emptyK[js % SK]);
+                            ns[t] = js + 1;
+                            moved = true;
+                        }
+                        const int jp = np[t];
+                        if (jp < ntiles && !(t == 1 && jp == ntiles - 1 && np[0] < ntiles) &&
+                            mbar_test(&p_full[t], jp & 1) && mbar_test(&fullV[jp % SV], (jp / SV) & 1)) {
+                            tcgen05_after_sync();
+                            issue_pv(jp, t);
+                            if (np[t ^ 1] > jp && jp + SV < ntiles)
+                                umma_commit(&emptyV[jp % SV]);
+                            np[t] = jp + 1;
+                            moved = true;
+                        }
+                    }
+                    if (moved) {
+                        idle = 0;
+                        since = global_timer_ns();
+                    } else if ((++idle & 63u) == 0u && (*abort_flag || global_timer_ns() - since > kWaitLimitNs)) {
+                        ok = false;  // nothing became ready for a whole wait limit (or another warp gave up)
+                    }
+                }
+            }
+            // P over S (D = 128), a fixed order: per KV tile, tile 0's P V and next S, then tile 1's
+            for (int jt = 0; jt < ntiles && ok && !G::kSepP; ++jt) {
                 const bool more = jt + 1 < ntiles;
                 const int kn = (jt + 1) % SK;
                 for (int t = 0; t < 2 && ok; ++t) {
-                    if (G::kSepP && more) {
-                        // the next S goes into columns the softmax has read: it runs during this softmax
-                        if (!mbar_wait_bounded(&s_read[t], jt & 1, abort_flag) ||
-                            (t == 0 && !mbar_wait_bounded(&fullK[kn], ((jt + 1) / SK) & 1, abort_flag))) {
-                            ok = false;
-                            break;
-                        }
-                        tcgen05_after_sync();
-                        issue_s(jt + 1, t);
-                        if (t == 1 && jt + 1 + SK < ntiles)
-                            umma_commit(&emptyK[kn]);
-                    }
                     if (!mbar_wait_bounded(&p_full[t], jt & 1, abort_flag) ||
                         (t == 0 && !mbar_wait_bounded(&fullV[jt % SV], (jt / SV) & 1, abort_flag))) {
                         ok = false;
@@ -1235,7 +1285,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_
                     issue_pv(jt, t);
                     if (t == 1 && jt + SV < ntiles)
                         umma_commit(&emptyV[jt % SV]);
-                    if (!G::kSepP && more) {
+                    if (more) {
                         // the next S overwrites this P: after its P V
                         if ((t == 0 && !mbar_wait_bounded(&fullK[kn], ((jt + 1) / SK) & 1, abort_flag)) ||
                             !mbar_wait_bounded(&pv_done[t], jt & 1, abort_flag)) {

@@ -3,12 +3,14 @@ paged_kv_cache_470_b200/csrc/prefill.cu), on the CPU.
 
 The kernel's CTA takes two query tiles that share every K/V tile. The model follows its actors and
 barriers: the producer warp (K and V of each KV tile into their own rings), the MMA thread (S_t = Q_t K^T
-and O_t += P_t V for tiles t = 0, 1 in a fixed order: per KV tile, tile 0's then tile 1's; a K or V stage
-is released by a commit after both tiles' MMAs have read it), four softmax warps per tile (read S, maybe
-rescale O, write P, hand P over; tile 0's warps also zero the last KV tile's V rows past the context) and
-the epilogue. Two layouts: P written over S (D = 128), where the next S waits for the P V, and P in
-columns of its own (D = 64), where the next S only waits until the softmax has read S and the softmax
-waits for the last P V before it writes P again. Barriers behave like mbarriers (an arrival count per
+and O_t += P_t V for tiles t = 0, 1; a K or V stage is released by a commit after both tiles' MMAs have
+read it), four softmax warps per tile (read S, maybe rescale O, write P, hand P over; tile 0's warps also
+zero the last KV tile's V rows past the context) and the epilogue. Two layouts: P written over S
+(D = 128), where the next S waits for the P V and the MMAs go in a fixed order (per KV tile, tile 0's then
+tile 1's), and P in columns of its own (D = 64), where the next S only waits until the softmax has read S,
+the softmax waits for the last P V before it writes P again, and the MMA thread issues whichever tile's
+next S or P V is ready (the model picks among the ready ones at random; the commit that releases a stage
+follows the second of the two MMAs that read it, and tile 1's P V of the last KV tile waits for tile 0's). Barriers behave like mbarriers (an arrival count per
 phase; a wait by parity cannot tell phases two apart); loads land and MMAs complete late, MMAs and their
 commits in issue order; an MMA may run before an earlier one into another accumulator (tcgen05.mma
 orders only MMAs with the same accumulator and shape), and a commit arrives once every MMA before it is
@@ -148,6 +150,9 @@ class PairModel:
         yield lambda: self.fullK[0].done(0)
         issue_s(0, 0)
         issue_s(0, 1)
+        if self.sep_p:
+            yield from self.mma_ready_first()
+            return
         for j in range(self.n):
             more = j + 1 < self.n
             kn, kp = (j + 1) % self.ks, ((j + 1) // self.ks) & 1
@@ -169,6 +174,48 @@ class PairModel:
                     if self.bug != "s_without_pv_wait":
                         yield lambda t=t, p=j & 1: self.pv_done[t].done(p)
                     issue_s(j + 1, t)
+        self.tc_queue.append(("commit", self.o_done))
+        yield lambda: self.o_done.done(0)
+
+    def mma_ready_first(self):
+        n, ks, vs = self.n, self.ks, self.vs
+        ns, np_ = [1, 1], [0, 0]
+
+        def ready():
+            ops = []
+            for t in (0, 1):
+                j = ns[t]
+                if (j < n and (self.bug == "s_without_read_wait" or self.s_read[t].done((j - 1) & 1))
+                        and self.fullK[j % ks].done((j // ks) & 1)):
+                    ops.append(("S", t))
+                j = np_[t]
+                last_waits = t == 1 and j == n - 1 and np_[0] < n and self.bug != "last_pv_before_zeroing"
+                if (j < n and not last_waits and self.p_full[t].done(j & 1)
+                        and self.fullV[j % vs].done((j // vs) & 1)):
+                    ops.append(("PV", t))
+            return ops
+
+        while np_[0] < n or np_[1] < n:
+            yield lambda: bool(ready())
+            kind, t = self.rng.choice(ready())
+            if kind == "S":
+                j = ns[t]
+                self.readers[("K", j % ks)] = self.readers.get(("K", j % ks), 0) + 1
+                self.tc_queue.append(("S", j, t))
+                self.tc_queue.append(("commit", self.s_full[t]))
+                second = ns[1 - t] > j
+                if (second != (self.bug == "release_k_after_one")) and j + ks < n:
+                    self.tc_queue.append(("commit", self.emptyK[j % ks]))
+                ns[t] = j + 1
+            else:
+                j = np_[t]
+                self.readers[("V", j % vs)] = self.readers.get(("V", j % vs), 0) + 1
+                self.tc_queue.append(("PV", j, t))
+                self.tc_queue.append(("commit", self.pv_done[t]))
+                second = np_[1 - t] > j
+                if (second != (self.bug == "release_v_after_one")) and j + vs < n:
+                    self.tc_queue.append(("commit", self.emptyV[j % vs]))
+                np_[t] = j + 1
         self.tc_queue.append(("commit", self.o_done))
         yield lambda: self.o_done.done(0)
 
@@ -271,7 +318,7 @@ def test_pair_kernel_hand_offs_hold_under_random_schedules(ntiles, layout):
     ("P_over_S", "loads_ignore_empty"),
     ("P_apart", "release_k_after_one"), ("P_apart", "release_v_after_one"),
     ("P_apart", "s_without_read_wait"), ("P_apart", "p_without_pv_wait"),
-    ("P_apart", "tile1_first"), ("P_apart", "loads_ignore_empty")])
+    ("P_apart", "last_pv_before_zeroing"), ("P_apart", "loads_ignore_empty")])
 def test_the_pair_model_catches_the_hand_off_mistakes(layout, bug):
     caught = 0
     for seed in range(300):
