@@ -942,11 +942,12 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(const __grid_const
 // the first half of its S at D = 128 and has columns of its own at D = 64
 // (384 + 64 t), where O leaves room. Warps 0-3 run the softmax of tile 0 and
 // warps 4-7 that of tile 1 (one row per thread, as in the one-tile kernel),
-// warp 8 issues the TMA loads, warp 9 the MMAs. The MMA thread alternates the
-// tiles: while one tile's softmax runs, the tensor pipe does the other tile's
-// P V and next S. At D = 128 the S of the next tile goes where P of this one
-// is, so it waits for that P V; at D = 64 it only waits until the softmax
-// has read S, and runs while the softmax computes. CTAs start longest sequence
+// warp 8 issues the TMA loads, warp 9 the MMAs. At D = 128 the MMA thread
+// alternates the tiles in a fixed order: while one tile's softmax runs, the
+// tensor pipe does the other tile's P V and next S, which goes where P of that
+// tile is and so waits for its P V. At D = 64 the next S only waits until the
+// softmax has read S and runs while the softmax computes; there the MMA
+// thread issues whichever tile's next S or P V is ready. CTAs start longest sequence
 // first (each ranks the batch's context lengths), and the epilogue writes each
 // row of O with one bulk copy from shared memory. Every hand-off is an
 // mbarrier with a bounded wait, as in the one-tile kernel.
@@ -1229,9 +1230,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_pair_kernel(const __grid_
             if (G::kSepP) {
                 // P apart from S (D = 64): whichever tile's next MMA is ready goes first. S(j + 1) of a tile
                 // needs only that its softmax has read S(j) and that K(j + 1) has landed, P V(j) that P(j)
-                // is full and V(j) has landed; in the fixed order below, a tile's next S waited behind the
-                // other tile's P (a timestamp trace: ~1,160 cycles of each ~3,280-cycle query-tile cycle
-                // spent waiting for S). A K or V stage is released by a commit after the second of the
+                // is full and V(j) has landed; in a fixed order (per KV tile, tile 0's MMAs, then tile 1's) a
+                // tile's next S waited behind the other tile's P (a timestamp trace: ~1,160 cycles of each
+                // ~3,280-cycle query-tile cycle spent waiting for S). A K or V stage is released by a commit after the second of the
                 // two tiles' MMAs that read it; tile 1's P V of the last KV tile follows tile 0's, whose
                 // P-full arrival comes after the zeroing of that tile's V rows past the context.
                 int ns[2] = {1, 1};  // next S per tile (S of KV tile 0 went out above)
