@@ -142,3 +142,67 @@ def test_planted_exit_rules_are_caught(rule):
         assert not good
         caught += bool(problems)
     assert caught > 0, rule
+
+
+# ---------------------------------------------------------------------------------------------------------
+# Why the ring's stage count is a multiple of the consumer streams. Consumer stream j takes units j, j + NS,
+# ...; with S a multiple of NS, every stage then has a single consuming stream. A stage's full mbarrier is
+# waited on by parity, which cannot tell phases two apart: were S not a multiple of NS, two streams would
+# share a stage, and one that reached the stage's next phase while the other still held the current one
+# would pass its wait on stale data. The model runs a producer, loads landing late and the streams under
+# random schedules, and catches exactly that when S is odd.
+# ---------------------------------------------------------------------------------------------------------
+class StageBar:
+    def __init__(self):
+        self.phase = 0
+
+    def arrive(self):  # one arrival completes a phase (the model counts whole releases and landings)
+        self.phase += 1
+
+    def done(self, parity):
+        return (self.phase & 1) != parity
+
+
+def run_streams(rng, S, NS, count):
+    """Returns the first read of a stage that holds another unit's data, or None."""
+    full, empty = [StageBar() for _ in range(S)], [StageBar() for _ in range(S)]
+    stage = [None] * S
+    nxt = list(range(NS))                  # each stream's next unit
+    issued, inflight = 0, []
+    for _ in range(50 * count + 100):
+        acts = []
+        if issued < count and empty[issued % S].done(((issued // S) & 1) ^ 1):
+            acts.append("issue")
+        if inflight:
+            acts.append("land")
+        acts += [j for j in range(NS) if nxt[j] < count and full[nxt[j] % S].done((nxt[j] // S) & 1)]
+        if not acts:
+            break
+        a = rng.choice(acts)
+        if a == "issue":
+            inflight.append(issued)
+            issued += 1
+        elif a == "land":
+            uu = inflight.pop(rng.randrange(len(inflight)))
+            stage[uu % S] = uu
+            full[uu % S].arrive()
+        else:
+            uu = nxt[a]
+            if stage[uu % S] != uu:
+                return f"stream {a} passed its wait for unit {uu} with stage {uu % S} holding {stage[uu % S]}"
+            nxt[a] += NS
+            empty[uu % S].arrive()
+    assert all(n >= count for n in nxt), "the schedule stopped before every unit was read"
+    return None
+
+
+@pytest.mark.parametrize("S,NS", [(6, 2), (12, 4), (24, 8), (12, 2), (48, 8)])
+def test_a_stage_count_the_streams_divide_keeps_every_read_fresh(S, NS):
+    rng = random.Random(S * 100 + NS)
+    for _ in range(60):
+        assert run_streams(rng, S, NS, rng.randrange(1, 4 * S + 7)) is None
+
+
+def test_an_odd_stage_count_is_caught():
+    rng = random.Random(5)
+    assert sum(run_streams(rng, 13, 2, 80) is not None for _ in range(200)) > 0
