@@ -206,3 +206,22 @@ def test_a_stage_count_the_streams_divide_keeps_every_read_fresh(S, NS):
 def test_an_odd_stage_count_is_caught():
     rng = random.Random(5)
     assert sum(run_streams(rng, 13, 2, 80) is not None for _ in range(200)) > 0
+
+
+@pytest.mark.parametrize("S,NS", [(12, 2), (6, 2), (12, 4), (24, 8), (48, 8), (2, 2)])
+def test_stepped_stage_and_phase_match_the_unit_index(S, NS):
+    """Each consumer stream steps its units' stage and phase (stage + NS, wrapping with a phase flip) instead of
+    dividing the unit index: from any item start u and for every stream, the stepped values equal uu % S and
+    (uu / S) & 1 for each unit uu = u + i, u + i + NS, ... the stream takes."""
+    for u in range(0, 3 * S + 5):
+        for stream in range(NS):
+            i = (stream - u) % NS
+            s, ph = (u + i) % S, ((u + i) // S) & 1
+            for _ in range(4 * S):
+                uu = u + i
+                assert (s, ph) == (uu % S, (uu // S) & 1), (S, NS, u, stream, uu)
+                i += NS
+                s += NS
+                if s >= S:
+                    s -= S
+                    ph ^= 1
